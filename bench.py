@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark of the block-scaled FP4 path on B200.
+
+One step = one pass of the whole path over one synthetic tensor (default:
+the 4096 x 4096 bf16 LLM weight matrix, N(0, 0.02) with 0.1 % outliers x50):
+  tensor amax -> NVFP4 quantise + pack -> MXFP4 quantise + pack ->
+  NVFP4 dequantise (bf16) -> MXFP4 dequantise (bf16) -> NVFP4 scale search
+(7 kernel launches; the amax is shared by the NVFP4 quantiser and the
+search).  `value` is elements of x per second over the whole job, timed on
+the device with CUDA events around each step, L2 flushed (512 MiB write)
+between steps, max over ranks.  `e2e` times the same step through the same
+C-ABI calls starting from pinned host memory: host->device copy of x, the
+step, device->host copy of every quantised artefact and the status word.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle on host cores
+
+Multi-GPU (torchrun): every rank quantises its own tensor (independent
+weight matrices, seeds offset by rank): weak scaling, no collective on the
+data path; one max all-reduce of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "FP4 quantize elements/s and achieved HBM GB/s (fraction of B200 peak), 1 GPU"
+FLUSH_BYTES = 512 << 20
+WORKLOADS = {
+    "weight-4096x4096-bf16": workloads.WEIGHT_4K,
+    "act-8192x14336-bf16": workloads.ACT_8K,
+    "search-4096x14336-bf16": workloads.SEARCH_4K,
+    "tiny-f32-256x1024": workloads.TINY_F32,
+}
+DEFAULT_WORKLOAD = "weight-4096x4096-bf16"
+KERNEL_SOURCES = ["block_scaled_fp4_reduce_b200/csrc/fp4_kernels.cuh",
+                  "block_scaled_fp4_reduce_b200/csrc/fp4_codec.cuh"]
+OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize", "scale_search"]
+LAUNCHES_PER_STEP = 7  # amax partial + amax fold + 5 single-kernel entry points
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def algorithmic_bytes(w: workloads.Workload) -> dict:
+    """Bytes each kernel must move per launch (read + write), by definition:
+    x once per pass, packed codes 1/2 byte per element, one scale byte per
+    block, dequantised bf16 output 2 bytes per element."""
+    n, e = w.numel, (2 if w.dtype == torch.bfloat16 else 4)
+    return {
+        "amax": n * e,
+        "nvfp4_quantize": n * e + n // 2 + n // 16,
+        "mxfp4_quantize": n * e + n // 2 + n // 32,
+        "nvfp4_dequantize": n // 2 + n // 16 + 2 * n,
+        "mxfp4_dequantize": n // 2 + n // 32 + 2 * n,
+        "scale_search": n * e + n // 2 + n // 16,
+    }
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed
+    region (every 100 ms)."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.out = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            self.target = vis.split(",")[device] if vis else str(device)
+
+    def start(self):
+        try:
+            self.out = open(os.path.join("/tmp", f"clocks_{os.getpid()}.csv"), "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.target, f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == len(self.FIELDS):
+                    rows.append(parts)
+        os.unlink(self.out.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# -------------------------------------------------------------- the step --
+
+class Path:
+    """Device buffers and pre-bound C-ABI calls of one step."""
+
+    def __init__(self, x: torch.Tensor):
+        import block_scaled_fp4_reduce_b200 as fp4
+        self.fp4 = fp4
+        L = fp4.lib()
+        dev = x.device
+        R, C = x.shape
+        self.x = x
+        self.n = x.numel()
+        u8 = torch.uint8
+        self.amax = torch.empty(1, dtype=torch.float32, device=dev)
+        self.ws = fp4.workspace_for(x)
+        self.status = fp4.new_status(dev)
+        self.nv_p = torch.empty((R, C // 2), dtype=u8, device=dev)
+        self.nv_s = torch.empty((R, C // 16), dtype=u8, device=dev)
+        self.nv_g = torch.empty(1, dtype=torch.float32, device=dev)
+        self.mx_p = torch.empty((R, C // 2), dtype=u8, device=dev)
+        self.mx_s = torch.empty((R, C // 32), dtype=u8, device=dev)
+        self.y_nv = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
+        self.y_mx = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
+        self.ss_p = torch.empty((R, C // 2), dtype=u8, device=dev)
+        self.ss_s = torch.empty((R, C // 16), dtype=u8, device=dev)
+        self.ss_g = torch.empty(1, dtype=torch.float32, device=dev)
+        st = torch.cuda.current_stream().cuda_stream
+        dt = fp4._dtype_code(x)
+        P = lambda t: t.data_ptr()  # noqa: E731
+        self.calls = [
+            (L.fp4_tensor_amax, (P(x), dt, self.n, P(self.amax), P(self.ws), self.ws.numel(), P(self.status), st)),
+            (L.fp4_nvfp4_quantize_with_amax, (P(x), dt, R, C, P(self.amax), P(self.nv_p), P(self.nv_s),
+                                              P(self.nv_g), P(self.status), st)),
+            (L.fp4_mxfp4_quantize, (P(x), dt, R, C, P(self.mx_p), P(self.mx_s), P(self.status), st)),
+            (L.fp4_dequantize, (fp4.NVFP4, P(self.nv_p), P(self.nv_s), P(self.nv_g), R, C, P(self.y_nv),
+                                fp4.BF16, st)),
+            (L.fp4_dequantize, (fp4.MXFP4, P(self.mx_p), P(self.mx_s), None, R, C, P(self.y_mx), fp4.BF16, st)),
+            (L.fp4_scale_search_with_amax, (P(x), dt, R, C, P(self.amax), P(self.ss_p), P(self.ss_s),
+                                            P(self.ss_g), None, P(self.status), st)),
+        ]
+        self.results = [self.nv_p, self.nv_s, self.nv_g, self.mx_p, self.mx_s, self.ss_p, self.ss_s,
+                        self.status]
+
+    def step(self, events=None):
+        for i, (fn, args) in enumerate(self.calls):
+            st = fn(*args)
+            if st != 0:
+                raise self.fp4.FP4Error(st, fn.__name__)
+            if events is not None:
+                events[i + 1].record()
+
+    def check_status(self):
+        st = int(self.status.item())
+        if st:
+            raise self.fp4.FP4Error(st, "bench step")
+
+
+def flush_l2(buf: torch.Tensor):
+    buf.zero_()
+
+
+def run_ours(args, rank: int, world: int, local: int):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = WORKLOADS[args.workload]
+    if world > 1:
+        w = workloads.with_shape(w, w.rows, w.cols, seed_offset=1000 * rank)
+    x_host = workloads.generate(w).pin_memory()
+    x = x_host.to(dev, non_blocking=False)
+    path = Path(x)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    nops = len(path.calls)
+
+    warmup = max(args.warmup, 3)
+    for _ in range(warmup):
+        flush_l2(flush)
+        path.step()
+    torch.cuda.synchronize()
+    path.check_status()
+
+    # ---- timed region: K steps, events around every entry point ----------
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nops + 1)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(K):
+        flush_l2(flush)
+        evs[k][0].record()
+        path.step(evs[k])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    path.check_status()
+    per_op_ms = [0.0] * nops
+    total_ms = 0.0
+    for k in range(K):
+        total_ms += evs[k][0].elapsed_time(evs[k][nops])
+        for i in range(nops):
+            per_op_ms[i] += evs[k][i].elapsed_time(evs[k][i + 1])
+
+    # ---- end to end through the same calls from pinned host memory ---------
+    Ke = max(3, min(K, args.e2e_steps))
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in path.results]
+    h2d = x.numel() * x.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in path.results)
+    e2e_ms = 0.0
+    for k in range(Ke + 2):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        x.copy_(x_host, non_blocking=True)
+        path.step()
+        for h, t in zip(host_out, path.results):
+            h.copy_(t, non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        if int(host_out[-1].item()) != 0:
+            raise RuntimeError("device status set during the end-to-end run")
+        if k >= 2:
+            e2e_ms += e0.elapsed_time(e1)
+
+    stats = torch.tensor([total_ms, e2e_ms] + per_op_ms, dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.destroy_process_group()
+    total_ms, e2e_ms, per_op_ms = stats[0].item(), stats[1].item(), stats[2:].tolist()
+    if rank != 0:
+        return
+
+    n_all = w.numel * world
+    value = n_all * K / (total_ms / 1e3)
+    pk = peaks()
+    ab = algorithmic_bytes(w)
+    kernels = {}
+    for name, ms in zip(OPS, per_op_ms):
+        us = ms / K * 1e3
+        gbs = ab[name] / (us * 1e-6) / 1e9
+        kernels[name] = {"us": round(us, 3), "share": round(ms / total_ms, 4), "gbs": round(gbs, 1),
+                         "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
+    dom = max(kernels, key=lambda k: kernels[k]["us"])
+    roof = roofline_for(dom, kernels[dom], w, pk)
+    line = {
+        "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": K,
+        "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name if world == 1 else WORKLOADS[args.workload].name,
+                   "description": WORKLOADS[args.workload].description,
+                   "shape": [w.rows, w.cols], "input_dtype": str(w.dtype).replace("torch.", ""),
+                   "step": "amax, nvfp4 quantize, mxfp4 quantize, nvfp4 dequantize (bf16), "
+                           "mxfp4 dequantize (bf16), nvfp4 64-candidate scale search",
+                   "l2": "flushed between steps (512 MiB write), outside the timed events",
+                   "parallelism": f"replicas x{world} (independent tensors)" if world > 1 else "single GPU"},
+        "hbm_gbs_step": sum(ab.values()) / (total_ms / K * 1e-3) / 1e9,
+        "kernels": kernels,
+        "roofline": roof,
+        "e2e": {"value": n_all * Ke / (e2e_ms / 1e3), "unit": "elements/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "clocks": clk,
+        "wall_s_timed": wall,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    print(json.dumps(line), flush=True)
+
+
+def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict) -> dict:
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            t = json.load(f)
+        ent = t.get("kernels", {}).get(name)
+        if ent and ent.get("source_hash") == kernel_source_hash() and ent.get("workload") == w.name:
+            traffic = ent.get("bytes_per_launch")
+    if name == "scale_search":
+        # ALU-bound: lane operations of the candidate evaluations per second
+        # against 148 SMs x 128 FP32 lanes x the max SM clock.
+        return {"bound": "hbm", "achieved": k["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": k["frac_hbm"], "traffic": traffic, "kernel": name,
+                "note": "scale search is issue-bound (ALU); this is its HBM fraction",
+                "peak_source": pk["source"]}
+    return {"bound": "hbm", "achieved": k["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": k["frac_hbm"], "traffic": traffic, "kernel": name, "peak_source": pk["source"]}
+
+
+# ------------------------------------------------------- CPU oracle legs --
+
+def _oracle_step(xs):
+    import oracle
+    p, s, g = oracle.nvfp4_quantize(xs)
+    pm, sm = oracle.mxfp4_quantize(xs)
+    R, C = xs.shape
+    oracle.nvfp4_dequantize(p, s, g, R, C)
+    oracle.mxfp4_dequantize(pm, sm, R, C)
+    oracle.nvfp4_scale_search(xs)
+
+
+def cpu_baseline(w: workloads.Workload, budget_s: float = 15.0) -> dict:
+    """The oracle as it stands (single-threaded C) on a bounded row sample of
+    the same workload, the same five steps; elements/s."""
+    import oracle
+    oracle.build()
+    x = workloads.generate(w)
+    xo = workloads.as_oracle_array(x)
+    rows = 4
+    t0 = time.perf_counter()
+    _oracle_step(xo[:rows])
+    t1 = time.perf_counter() - t0
+    rows = int(max(4, min(w.rows, rows * budget_s / max(t1, 1e-3) / 2)))
+    t0 = time.perf_counter()
+    _oracle_step(xo[:rows])
+    dt = time.perf_counter() - t0
+    return {"value": rows * w.cols / dt, "unit": "elements/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} of {w.rows} rows ({rows * w.cols} elements), whole step, "
+                      f"{dt:.1f} s", "cpu": _cpu_model()}
+
+
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def run_reference(args, rank: int, world: int):
+    """--impl reference: the CPU oracle on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    w = WORKLOADS[args.workload]
+    x = workloads.generate(w)
+    xo = workloads.as_oracle_array(x)
+    total_budget = 120.0
+    t0 = time.perf_counter()
+    _oracle_step(xo[:2])
+    t_row = (time.perf_counter() - t0) / 2
+    steps, warm = args.steps, max(args.warmup, 0)
+    rows = int(max(1, min(w.rows, total_budget / max(t_row, 1e-4) / (steps + warm))))
+    for _ in range(warm):
+        _oracle_step(xo[:rows])
+    t0 = time.perf_counter()
+    for k in range(steps):
+        r0 = (k * rows) % max(1, w.rows - rows + 1)
+        _oracle_step(np.ascontiguousarray(xo[r0:r0 + rows]))
+    dt = time.perf_counter() - t0
+    value = rows * w.cols * steps / dt
+    line = {
+        "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": steps,
+        "warmup": warm, "ms_per_step": dt / steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "description": w.description, "shape": [w.rows, w.cols]},
+        "cpu_baseline": {"value": value, "unit": "elements/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} rows x {w.cols} per step (bounded sample of the workload)",
+                         "cpu": _cpu_model()},
+        "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+import numpy as np  # noqa: E402  (used by the reference leg)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * fp4.h -- C ABI of the B200 (sm_100a) block-scaled FP4 library.
+ *
+ * Block-scaled FP4 stores every element as a four-bit E2M1 code (1 sign,
+ * 2 exponent, 1 mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) and
+ * shares one scale per block of consecutive elements along the last
+ * dimension:
+ *   NVFP4  16-element blocks, E4M3 (FN) block scale s_b, FP32 global scale g;
+ *          x_hat = q * s_b * g.
+ *   MXFP4  32-element blocks, E8M0 power-of-two scale 2^e; x_hat = q * 2^e.
+ * Definitions: "NVFP4 与 MXFP4 格式" (charlestar.github.io, nvfp4-mxfp4-
+ * format) sections 1-5 and 8; "FP4 / NVFP4 数学总结" (devpress.csdn.net)
+ * sections 3, 9 and 10; "FP4、FP8 与 INT8/INT4" (tom-jerr.github.io)
+ * section 3.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.  Every pointer is a DEVICE pointer owned by the caller.  x,
+ * packed and y must be 16-byte aligned (else FP4_ERR_ALIGN); scales,
+ * global_scale, block_loss, status and workspace need only the alignment of
+ * their element type (workspace: 4 bytes).  The library never
+ * allocates, frees or synchronises; all work is queued on `stream`
+ * (a cudaStream_t; NULL = the legacy default stream) and the call returns
+ * as soon as it is queued.
+ *
+ * Layout.  x is a contiguous row-major [rows, cols] tensor of fp32 or bf16.
+ * Blocks run along a row: cols must be a multiple of 16 (NVFP4, scale
+ * search) or 32 (MXFP4), else FP4_ERR_SHAPE -- incomplete blocks are
+ * rejected, as the pages' reference programs do.  rows * cols may be zero
+ * (nothing is launched; a quantiser still writes g = 1 and no error).
+ *   packed  uint8 [rows, cols/2]: element 2i in the low nibble, 2i+1 in the
+ *           high nibble of byte i ("NVFP4 与 MXFP4 格式" section 1).
+ *   scales  uint8 [rows, cols/16] E4M3 (NVFP4) or [rows, cols/32] E8M0
+ *           (MXFP4), plain row-major, one byte per block.
+ *   global_scale  one fp32 in device memory holding g = fl32(A / (6*448)),
+ *           A = max|x| over the tensor: the DEQUANT multiplier (the page's
+ *           `a`, not the reciprocal some GEMM interfaces call global_scale).
+ *
+ * Errors.  Argument errors (NULL pointer, bad shape, misalignment, unknown
+ * dtype, workspace too small) are returned at once and nothing is queued.
+ * Launch failures return FP4_ERR_CUDA.  Data errors are found on the GPU
+ * and reported through `status`, a caller-owned device int32: a kernel
+ * that finds one stores its code there only if the word still holds FP4_OK,
+ * so the first error sticks until the CALLER clears the word (the library
+ * never does).  When *status != FP4_OK after a call, that call's outputs are
+ * unspecified.  Data errors: FP4_ERR_NONFINITE (a NaN or Inf in x) and
+ * FP4_ERR_RANGE (NVFP4 global scale below the smallest normal fp32 for a
+ * nonzero tensor, i.e. 0 < A < 2688 * 2^-126).
+ *
+ * Concurrency.  Calls on one stream are ordered.  Two calls that share a
+ * workspace must not run concurrently on different streams.
+ */
+#ifndef FP4_B200_H
+#define FP4_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fp4_status {
+    FP4_OK = 0,
+    FP4_ERR_INVALID_ARG = 1, /* NULL pointer, unknown enum, negative size */
+    FP4_ERR_SHAPE = 2,       /* cols not a multiple of the block size; overflow */
+    FP4_ERR_ALIGN = 3,       /* a tensor pointer is not 16-byte aligned */
+    FP4_ERR_NONFINITE = 4,   /* (device status) NaN or Inf in the input */
+    FP4_ERR_RANGE = 5,       /* (device status) NVFP4 global scale out of range */
+    FP4_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than required */
+    FP4_ERR_CUDA = 7         /* a CUDA launch or query failed */
+} fp4_status;
+
+typedef enum fp4_dtype { FP4_F32 = 0, FP4_BF16 = 1 } fp4_dtype;
+typedef enum fp4_format { FP4_NVFP4 = 0, FP4_MXFP4 = 1 } fp4_format;
+
+/* Human-readable name of a status value (static string). */
+const char *fp4_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int fp4_version(void);
+
+/* Bytes of device workspace the NVFP4 quantiser, the scale search and the
+ * tensor amax need for a [rows, cols] input: per-CTA partial maxima of the
+ * first pass.  Any caller-owned device buffer of at least this size, 4-byte
+ * aligned, works; it need not be initialised and its contents are scratch. */
+size_t fp4_workspace_bytes(fp4_format fmt, int64_t rows, int64_t cols);
+
+/* Tensor amax A = max |x| over n elements ("NVFP4 与 MXFP4 格式" section 3,
+ * A is the tensor absolute maximum; section 4 reference program, first
+ * step).  Writes A as one fp32 to device `amax`.  A NaN or Inf in x sets
+ * FP4_ERR_NONFINITE in *status (and *amax then holds a non-finite value).
+ * Two launches: per-CTA partial maxima into `workspace`, then a one-CTA
+ * reduction. */
+fp4_status fp4_tensor_amax(const void *x, fp4_dtype dtype, int64_t n, float *amax,
+                           void *workspace, size_t workspace_bytes, int32_t *status,
+                           cudaStream_t stream);
+
+/* NVFP4 quantise + pack ("NVFP4 与 MXFP4 格式" section 3, the two-scale
+ * quantiser; section 4 reference program; "FP4 / NVFP4 数学总结" section 10).
+ *   g   = fl32(A / 2688); A = 0 gives g = 1.
+ *   s_b = E4M3 code nearest (ties to even code) to the exact rational
+ *         A_b / (6 g), saturated at 448; A_b = block max |x|.
+ *   codes: zero scale -> all sixteen codes 0; else v = fl32(x / fl32(s_b*g))
+ *         (IEEE single division) rounded to the nearest E2M1 value, ties to
+ *         the even code, |v| > 6 saturating, the sign bit of x kept.
+ * Outputs packed [rows, cols/2], scales [rows, cols/16] (E4M3 codes) and
+ * *global_scale = g.  Two kernels: tensor amax into the workspace, then the
+ * fused block-amax / scale / divide / round / pack pass.  Data errors:
+ * NONFINITE, RANGE. */
+fp4_status fp4_nvfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                              uint8_t *packed, uint8_t *scales, float *global_scale,
+                              void *workspace, size_t workspace_bytes, int32_t *status,
+                              cudaStream_t stream);
+
+/* NVFP4 quantise + pack given a tensor amax already in device memory (for a
+ * tensor split across calls or devices whose amax was combined by the
+ * caller, e.g. a max all-reduce).  Same outputs and rules as
+ * fp4_nvfp4_quantize with A = *amax; a non-finite *amax sets NONFINITE. */
+fp4_status fp4_nvfp4_quantize_with_amax(const void *x, fp4_dtype dtype, int64_t rows,
+                                        int64_t cols, const float *amax, uint8_t *packed,
+                                        uint8_t *scales, float *global_scale, int32_t *status,
+                                        cudaStream_t stream);
+
+/* MXFP4 quantise + pack ("NVFP4 与 MXFP4 格式" section 2, E8M0 32-blocks;
+ * section 5, the OCP rounding-down scale rule).  Per 32-block:
+ * e = floor(log2 A_b) - 2 clamped to [-127, 127] (an all-zero block clamps
+ * to -127), scale byte e + 127, codes of v = x * 2^-e (exact) rounded as
+ * for NVFP4 (block maxima in [6, 8) * 2^e saturate to 6).  One kernel, one
+ * pass.  Data error: NONFINITE. */
+fp4_status fp4_mxfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                              uint8_t *packed, uint8_t *scales, int32_t *status,
+                              cudaStream_t stream);
+
+/* Dequantise ("FP4 / NVFP4 数学总结" section 3, x_hat = q * s_b * g;
+ * "FP4、FP8 与 INT8/INT4" section 3.2, x_hat = 2^e q).
+ *   NVFP4: y = fl32(fl32(p * s_b) * g), p the E2M1 value of the code
+ *          (code 8 = -0), s_b the E4M3 value of the scale byte (0x7F/0xFF
+ *          -> NaN), g = *global_scale.
+ *   MXFP4: y = p * 2^(byte - 127) (exact; byte 255 -> NaN); global_scale
+ *          is ignored and may be NULL.
+ * y is [rows, cols] of out_dtype: fp32 as computed, or bf16 rounded to
+ * nearest even.  No data errors (foreign NaN scale bytes give NaN). */
+fp4_status fp4_dequantize(fp4_format fmt, const uint8_t *packed, const uint8_t *scales,
+                          const float *global_scale, int64_t rows, int64_t cols, void *y,
+                          fp4_dtype out_dtype, cudaStream_t stream);
+
+/* MSE-minimising NVFP4 block-scale search ("FP4 / NVFP4 数学总结" section 9,
+ * Loss(s) = sum_i (x_i - s Round(x_i / s))^2; "NVFP4 与 MXFP4 格式" section 4,
+ * the max-based E4M3 scale need not minimise the block MSE).
+ * g as for fp4_nvfp4_quantize.  Candidates per 16-block: the E4M3 codes
+ * nearest to m_k * A_b / (6 g), m_k = (147 + k) / 210, k = 0..63 (64 points
+ * evenly spaced over [0.70, 1.00], each an exact rational rounded once).
+ * Each candidate's loss is that of the artefact the quantiser would emit at
+ * that scale (codes as in fp4_nvfp4_quantize, x_hat as in fp4_dequantize),
+ * summed in double; the smallest loss wins, exact ties go to the larger
+ * scale.  Emits the winner's packed codes, scale byte and g; block_loss
+ * (fp32 [rows, cols/16], may be NULL) receives the winning loss rounded to
+ * fp32.  Data errors: NONFINITE, RANGE. */
+fp4_status fp4_scale_search(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                            uint8_t *packed, uint8_t *scales, float *global_scale,
+                            float *block_loss, void *workspace, size_t workspace_bytes,
+                            int32_t *status, cudaStream_t stream);
+
+/* Scale search given a tensor amax already in device memory (e.g. from
+ * fp4_tensor_amax, shared with fp4_nvfp4_quantize_with_amax so the tensor
+ * is read once for both).  Same outputs and rules as fp4_scale_search with
+ * A = *amax; a non-finite *amax sets NONFINITE.  One kernel. */
+fp4_status fp4_scale_search_with_amax(const void *x, fp4_dtype dtype, int64_t rows,
+                                      int64_t cols, const float *amax, uint8_t *packed,
+                                      uint8_t *scales, float *global_scale, float *block_loss,
+                                      int32_t *status, cudaStream_t stream);
+
+/* Element encoder alone, for tests: codes[i] = E2M1 code of the fp32 value
+ * v[i] (nearest, ties to even code, saturating, sign bit kept).  A NaN or
+ * Inf in v gives an unspecified code.  codes is uint8 [n] (one code per
+ * byte, unpacked). */
+fp4_status fp4_e2m1_round(const float *v, uint8_t *codes, int64_t n, cudaStream_t stream);
+
+/* NVFP4 element quotient + encoder alone, for tests: codes[i] = E2M1 code
+ * of fl32(x[i] / d[i]) computed by the same device routine the NVFP4
+ * quantiser uses for one element (d[i] > 0 finite, x[i] finite). */
+fp4_status fp4_nv_encode_quotient(const float *x, const float *d, uint8_t *codes, int64_t n,
+                                  cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4_B200_H */

@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
             "oracle_nv_block_loss": (D, [P, I, F]),
             "oracle_search_candidate_code": (I, [F, F, I]),
             "oracle_nvfp4_scale_search": (I, [P, I, I64, I64, P, P, P, P]),
+            "oracle_nvfp4_scale_search_with_g": (I, [P, I, I64, I64, F, P, P, P]),
             "oracle_nvfp4_artefact_loss": (I, [P, I, I64, I64, P, P, F, P]),
             "oracle_storage_bytes": (I64, [I64, I64, I64]),
         }
@@ -299,6 +300,19 @@ def nvfp4_scale_search(x: np.ndarray):
     _check(lib().oracle_nvfp4_scale_search(_ptr(x), dt, R, C, _ptr(packed), _ptr(scales),
                                            ctypes.byref(g), _ptr(loss)))
     return packed, scales, g.value, loss
+
+
+def nvfp4_scale_search_with_g(x: np.ndarray, g: float):
+    """The search at a given global scale (for row samples of a large
+    tensor).  Returns (packed, scales, block_loss)."""
+    x, dt = _input(x)
+    R, C = _shape(x)
+    packed = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    loss = np.zeros((R, C // 16), np.float64)
+    _check(lib().oracle_nvfp4_scale_search_with_g(_ptr(x), dt, R, C, float(g), _ptr(packed),
+                                                  _ptr(scales), _ptr(loss)))
+    return packed, scales, loss
 
 
 def nvfp4_artefact_loss(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, g: float) -> np.ndarray:

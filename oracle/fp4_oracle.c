@@ -454,29 +454,24 @@ int oracle_search_candidate_code(float amax_b, float g, int k)
     return oracle_e4m3_encode(t);
 }
 
-/* Brute-force search over all 64 candidates of every block: the scale with
- * the smallest loss wins, exact ties go to the larger scale.  Emits packed
- * codes, scale codes, g and (optionally) the winning loss per block. */
-int oracle_nvfp4_scale_search(const void *x, int dtype, int64_t rows, int64_t cols,
-                              uint8_t *packed, uint8_t *scales, float *g_out,
-                              double *block_loss)
+/* Brute-force search over all 64 candidates of every block at a given
+ * global scale g: the scale with the smallest loss wins, exact ties go to
+ * the larger scale.  Emits packed codes, scale codes and (optionally) the
+ * winning loss per block. */
+int oracle_nvfp4_scale_search_with_g(const void *x, int dtype, int64_t rows, int64_t cols,
+                                     float g, uint8_t *packed, uint8_t *scales,
+                                     double *block_loss)
 {
     if (cols % 16 || rows < 0 || cols < 0)
         return ORACLE_ERR_SHAPE;
-    float amax, g;
-    int st = oracle_tensor_amax(x, dtype, rows * cols, &amax);
-    if (st)
-        return st;
-    st = oracle_nv_global_scale(amax, &g);
-    if (st)
-        return st;
-    *g_out = g;
     int64_t nblocks = rows * cols / 16;
     for (int64_t b = 0; b < nblocks; ++b) {
         float xb[16];
         float ab = 0.0f;
         for (int i = 0; i < 16; ++i) {
             xb[i] = load_elem(x, dtype, b * 16 + i);
+            if (!isfinite(xb[i]))
+                return ORACLE_ERR_NONFINITE;
             if (fabsf(xb[i]) > ab)
                 ab = fabsf(xb[i]);
         }
@@ -499,6 +494,24 @@ int oracle_nvfp4_scale_search(const void *x, int dtype, int64_t rows, int64_t co
             block_loss[b] = best_loss;
     }
     return ORACLE_OK;
+}
+
+/* The full search: tensor amax -> g (as for NVFP4) -> per-block search. */
+int oracle_nvfp4_scale_search(const void *x, int dtype, int64_t rows, int64_t cols,
+                              uint8_t *packed, uint8_t *scales, float *g_out,
+                              double *block_loss)
+{
+    if (cols % 16 || rows < 0 || cols < 0)
+        return ORACLE_ERR_SHAPE;
+    float amax, g;
+    int st = oracle_tensor_amax(x, dtype, rows * cols, &amax);
+    if (st)
+        return st;
+    st = oracle_nv_global_scale(amax, &g);
+    if (st)
+        return st;
+    *g_out = g;
+    return oracle_nvfp4_scale_search_with_g(x, dtype, rows, cols, g, packed, scales, block_loss);
 }
 
 /* Per-block loss of given (packed, scale) artefacts against x, for
