@@ -5,9 +5,9 @@ One step = one pass of the whole path over one synthetic tensor (default:
 the 4096 x 4096 bf16 LLM weight matrix, N(0, 0.02) with 0.1 % outliers x50):
   tensor amax -> NVFP4 quantise + pack -> MXFP4 quantise + pack ->
   NVFP4 dequantise (bf16) -> MXFP4 dequantise (bf16) -> NVFP4 scale search
-(7 kernel launches; the amax is shared by the NVFP4 quantiser and the
+(6 kernel launches; the amax is shared by the NVFP4 quantiser and the
 search).  `value` is elements of x per second over the whole job, timed on
-the device with CUDA events around each step, L2 flushed (512 MiB write)
+the device with CUDA events around each step, L2 flushed (512 MiB write, 256 MiB read)
 between steps, max over ranks.  `e2e` times the same step through the same
 C-ABI calls starting from pinned host memory: host->device copy of x, the
 step, device->host copy of every quantised artefact and the status word.
@@ -40,7 +40,6 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "FP4 quantize elements/s and achieved HBM GB/s (fraction of B200 peak), 1 GPU"
-FLUSH_BYTES = 512 << 20
 WORKLOADS = {
     "weight-4096x4096-bf16": workloads.WEIGHT_4K,
     "act-8192x14336-bf16": workloads.ACT_8K,
@@ -51,7 +50,7 @@ DEFAULT_WORKLOAD = "weight-4096x4096-bf16"
 KERNEL_SOURCES = ["block_scaled_fp4_reduce_b200/csrc/fp4_kernels.cuh",
                   "block_scaled_fp4_reduce_b200/csrc/fp4_codec.cuh"]
 OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize", "scale_search"]
-LAUNCHES_PER_STEP = 7  # amax partial + amax fold + 5 single-kernel entry points
+LAUNCHES_PER_STEP = 6  # one kernel per entry point (the amax folds in its last CTA)
 
 
 def peaks() -> dict:
@@ -205,8 +204,28 @@ class Path:
             raise self.fp4.FP4Error(st, "bench step")
 
 
-def flush_l2(buf: torch.Tensor):
-    buf.zero_()
+def max_over_ranks(values: list[float], device, world: int) -> list[float]:
+    """Element-wise max of per-rank timings (one all-reduce; identity at N=1)."""
+    if world == 1:
+        return list(values)
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+class L2Flush:
+    """Between timed steps: write a buffer larger than L2 (evicting x and the
+    outputs), then read a second one, so that the dirty lines of the write
+    are written back before the next step and L2 starts clean and cold."""
+
+    def __init__(self, mib: int, device):
+        self.w = torch.empty(mib << 20, dtype=torch.uint8, device=device) if mib else None
+        self.r = torch.ones((mib // 2) << 18, dtype=torch.int32, device=device) if mib else None
+
+    def __call__(self):
+        if self.w is not None:
+            self.w.zero_()
+            self.r.sum()
 
 
 def run_ours(args, rank: int, world: int, local: int):
@@ -215,18 +234,16 @@ def run_ours(args, rank: int, world: int, local: int):
     if world > 1:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    w = WORKLOADS[args.workload]
-    if world > 1:
-        w = workloads.with_shape(w, w.rows, w.cols, seed_offset=1000 * rank)
+    w = workloads.for_rank(WORKLOADS[args.workload], rank)
     x_host = workloads.generate(w).pin_memory()
     x = x_host.to(dev, non_blocking=False)
     path = Path(x)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_l2 = L2Flush(args.flush_mib, dev)
     nops = len(path.calls)
 
     warmup = max(args.warmup, 3)
     for _ in range(warmup):
-        flush_l2(flush)
+        flush_l2()
         path.step()
     torch.cuda.synchronize()
     path.check_status()
@@ -241,7 +258,7 @@ def run_ours(args, rank: int, world: int, local: int):
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     for k in range(K):
-        flush_l2(flush)
+        flush_l2()
         evs[k][0].record()
         path.step(evs[k])
     torch.cuda.synchronize()
@@ -264,7 +281,7 @@ def run_ours(args, rank: int, world: int, local: int):
     d2h = sum(t.numel() * t.element_size() for t in path.results)
     e2e_ms = 0.0
     for k in range(Ke + 2):
-        flush_l2(flush)
+        flush_l2()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         x.copy_(x_host, non_blocking=True)
@@ -278,11 +295,9 @@ def run_ours(args, rank: int, world: int, local: int):
         if k >= 2:
             e2e_ms += e0.elapsed_time(e1)
 
-    stats = torch.tensor([total_ms, e2e_ms] + per_op_ms, dtype=torch.float64, device=dev)
+    total_ms, e2e_ms, *per_op_ms = max_over_ranks([total_ms, e2e_ms] + per_op_ms, dev, world)
     if world > 1:
-        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.destroy_process_group()
-    total_ms, e2e_ms, per_op_ms = stats[0].item(), stats[1].item(), stats[2:].tolist()
     if rank != 0:
         return
 
@@ -297,7 +312,8 @@ def run_ours(args, rank: int, world: int, local: int):
         kernels[name] = {"us": round(us, 3), "share": round(ms / total_ms, 4), "gbs": round(gbs, 1),
                          "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
     dom = max(kernels, key=lambda k: kernels[k]["us"])
-    roof = roofline_for(dom, kernels[dom], w, pk)
+    n_cand = search_candidate_count(x, path.ss_g.item()) if dom == "scale_search" else None
+    roof = roofline_for(dom, kernels[dom], w, pk, n_cand)
     line = {
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": K,
         "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
@@ -307,7 +323,8 @@ def run_ours(args, rank: int, world: int, local: int):
                    "shape": [w.rows, w.cols], "input_dtype": str(w.dtype).replace("torch.", ""),
                    "step": "amax, nvfp4 quantize, mxfp4 quantize, nvfp4 dequantize (bf16), "
                            "mxfp4 dequantize (bf16), nvfp4 64-candidate scale search",
-                   "l2": "flushed between steps (512 MiB write), outside the timed events",
+                   "l2": f"flushed between steps outside the timed events ({args.flush_mib} MiB write, "
+                         f"then {args.flush_mib // 2} MiB read)",
                    "parallelism": f"replicas x{world} (independent tensors)" if world > 1 else "single GPU"},
         "hbm_gbs_step": sum(ab.values()) / (total_ms / K * 1e-3) / 1e9,
         "kernels": kernels,
@@ -323,7 +340,27 @@ def run_ours(args, rank: int, world: int, local: int):
     print(json.dumps(line), flush=True)
 
 
-def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict) -> dict:
+def search_candidate_count(x: torch.Tensor, g: float) -> int:
+    """Number of distinct scale candidates the search definition leaves after
+    merging duplicates, summed over the blocks of x: the candidates of a block
+    are the contiguous E4M3 codes from round(0.70 A_b/(6g)) to round(A_b/(6g)).
+    Counted with torch (fp32 quotients, torch's E4M3 rounding) once per
+    workload, outside the timed region; it sizes the work, not the output."""
+    ab = x.float().reshape(-1, 16).abs().amax(dim=1).double()
+    t_hi = (ab / (6.0 * g)).clamp(max=448.0).float()
+    t_lo = (ab * 147.0 / (1260.0 * g)).clamp(max=448.0).float()
+    c_hi = t_hi.to(torch.float8_e4m3fn).view(torch.uint8).long()
+    c_lo = t_lo.to(torch.float8_e4m3fn).view(torch.uint8).long()
+    return int((c_hi - c_lo + 1).sum().item())
+
+
+# fp32 operations of one candidate-element evaluation of the search: quotient
+# (one multiply by a reciprocal), round to the E2M1 grid, decode, two
+# reconstruction multiplies, subtract, square-accumulate.
+SEARCH_OPS_PER_EVAL = 7
+
+
+def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict, n_cand: int | None = None) -> dict:
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
@@ -332,13 +369,16 @@ def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict) -> dict:
         ent = t.get("kernels", {}).get(name)
         if ent and ent.get("source_hash") == kernel_source_hash() and ent.get("workload") == w.name:
             traffic = ent.get("bytes_per_launch")
-    if name == "scale_search":
-        # ALU-bound: lane operations of the candidate evaluations per second
-        # against 148 SMs x 128 FP32 lanes x the max SM clock.
-        return {"bound": "hbm", "achieved": k["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": k["frac_hbm"], "traffic": traffic, "kernel": name,
-                "note": "scale search is issue-bound (ALU); this is its HBM fraction",
-                "peak_source": pk["source"]}
+    if name == "scale_search" and n_cand:
+        # ALU-bound: fp32 lane operations of the distinct candidate
+        # evaluations per second, against SMs x 128 FP32 lanes x max SM clock.
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        peak = sms * 128 * pk["sm_max_mhz"] * 1e6 / 1e12
+        achieved = n_cand * 16 * SEARCH_OPS_PER_EVAL / (k["us"] * 1e-6) / 1e12
+        return {"bound": "alu", "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": "Tops/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": name,
+                "work": f"{n_cand} distinct candidates x 16 elements x {SEARCH_OPS_PER_EVAL} fp32 ops",
+                "peak_source": f"{sms} SMs x 128 FP32 lanes x {pk['sm_max_mhz']:.0f} MHz ({pk['source']})"}
     return {"bound": "hbm", "achieved": k["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": k["frac_hbm"], "traffic": traffic, "kernel": name, "peak_source": pk["source"]}
 
@@ -435,6 +475,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-mib", type=int, default=512,
+                    help="L2 flush size between steps (0 = no flush, for profiler runs only)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
             "fp4_scale_search": (I, [P, I, I64, I64, P, P, P, P, P, SZ, P, P]),
             "fp4_scale_search_with_amax": (I, [P, I, I64, I64, P, P, P, P, P, P, P]),
             "fp4_e2m1_round": (I, [P, P, I64, P]),
+            "fp4_e2m1_roundtrip": (I, [P, P, I64, P]),
             "fp4_nv_encode_quotient": (I, [P, P, P, I64, P]),
         }
         for name, (res, args) in sig.items():
@@ -156,6 +157,10 @@ def fp4_e2m1_round(v, codes, stream=None) -> int:
     return lib().fp4_e2m1_round(_p(v), _p(codes), v.numel(), _stream(stream))
 
 
+def fp4_e2m1_roundtrip(v, out, stream=None) -> int:
+    return lib().fp4_e2m1_roundtrip(_p(v), _p(out), v.numel(), _stream(stream))
+
+
 def fp4_nv_encode_quotient(x, d, codes, stream=None) -> int:
     return lib().fp4_nv_encode_quotient(_p(x), _p(d), _p(codes), x.numel(), _stream(stream))
 
@@ -183,8 +188,9 @@ class Quantized:
 
 
 def workspace_for(x: torch.Tensor) -> torch.Tensor:
+    """A zero-filled workspace (the library keeps its counter word at zero)."""
     n = lib().fp4_workspace_bytes(NVFP4, *_shape2(x))
-    return torch.empty(n, dtype=torch.uint8, device=x.device)
+    return torch.zeros(n, dtype=torch.uint8, device=x.device)
 
 
 def new_status(device) -> torch.Tensor:
@@ -246,6 +252,12 @@ def e2m1_round(v: torch.Tensor, stream=None) -> torch.Tensor:
     codes = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
     _check(fp4_e2m1_round(v, codes, stream), "fp4_e2m1_round")
     return codes
+
+
+def e2m1_roundtrip(v: torch.Tensor, stream=None) -> torch.Tensor:
+    out = torch.empty((v.numel(), 2), dtype=torch.float32, device=v.device)
+    _check(fp4_e2m1_roundtrip(v, out, stream), "fp4_e2m1_roundtrip")
+    return out
 
 
 def nv_encode_quotient(x: torch.Tensor, d: torch.Tensor, stream=None) -> torch.Tensor:

@@ -67,9 +67,27 @@ template <typename K> int grid_for(K kernel, int64_t work, int64_t per_cta)
     return (int)(want < cap ? want : cap);
 }
 
-fp4_status launched()
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel on the stream finishes; it waits for it
+// (griddepcontrol.wait) before touching memory.
+template <typename... KArgs, typename... Args>
+fp4_status launch(void (*kernel)(KArgs...), int grid, cudaStream_t stream, Args... args)
 {
-    return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return FP4_ERR_CUDA;
+    }
+    return FP4_OK;
 }
 
 bool valid_dtype(fp4_dtype t) { return t == FP4_F32 || t == FP4_BF16; }
@@ -86,57 +104,54 @@ fp4_status check_shape(int64_t rows, int64_t cols, int64_t block)
     return FP4_OK;
 }
 
-// Tensor amax, pass 1: returns the number of partials written (>= 0), or
-// -1 on a launch-configuration failure.
-int launch_amax_partials(const void *x, fp4_dtype dt, int64_t n, uint32_t *partials,
-                         cudaStream_t stream)
+// Workspace words: kMaxPartials per-CTA maxima, the wrapping CTA counter,
+// and the amax word the NVFP4 quantiser and the search read.
+constexpr size_t kWsAmax = kMaxPartials + 1; // kMaxPartials holds the counter
+constexpr size_t kWsWords = kMaxPartials + 8;
+
+// Tensor amax (one launch) into *amax.
+fp4_status launch_amax(const void *x, fp4_dtype dt, int64_t n, uint32_t *ws, float *amax,
+                       int32_t *status, cudaStream_t stream)
 {
-    if (n == 0)
-        return 0;
-    const int64_t elems_per_vec = dt == FP4_BF16 ? 8 : 4;
+    const int64_t elems_per_vec = dt == FP4_BF16 ? 16 : 8; // one 32-byte vector
     const int64_t nvec = n / elems_per_vec;
     const int64_t per_cta = (int64_t)kThreads * 4;
     int grid;
     if (dt == FP4_BF16)
-        grid = grid_for(fp4::amax_partial_kernel<uint16_t>, nvec, per_cta);
+        grid = grid_for(fp4::amax_kernel<uint16_t>, nvec, per_cta);
     else
-        grid = grid_for(fp4::amax_partial_kernel<float>, nvec, per_cta);
+        grid = grid_for(fp4::amax_kernel<float>, nvec, per_cta);
     if (grid <= 0)
-        return -1;
+        return FP4_ERR_CUDA;
     if (grid > kMaxPartials)
         grid = kMaxPartials;
     if (dt == FP4_BF16)
-        fp4::amax_partial_kernel<uint16_t>
-            <<<grid, kThreads, 0, stream>>>(static_cast<const uint16_t *>(x), n, partials);
-    else
-        fp4::amax_partial_kernel<float>
-            <<<grid, kThreads, 0, stream>>>(static_cast<const float *>(x), n, partials);
-    return grid;
+        return launch(fp4::amax_kernel<uint16_t>, grid, stream, static_cast<const uint16_t *>(x), n,
+                      ws, amax, status);
+    return launch(fp4::amax_kernel<float>, grid, stream, static_cast<const float *>(x), n, ws, amax,
+                  status);
 }
 
-fp4_status launch_nv_quantize(const void *x, fp4_dtype dt, int64_t n, const uint32_t *partials,
-                              int nparts, uint8_t *packed, uint8_t *scales, float *global_scale,
+fp4_status launch_nv_quantize(const void *x, fp4_dtype dt, int64_t n, const float *amax,
+                              uint8_t *packed, uint8_t *scales, float *global_scale,
                               int32_t *status, cudaStream_t stream)
 {
-    const int64_t n_units = n / 8;
+    const int64_t n_blocks = n / 16;
     const int64_t per_cta = (int64_t)kThreads * 2;
     int grid;
     if (dt == FP4_BF16)
-        grid = grid_for(fp4::nvfp4_quantize_kernel<uint16_t>, n_units, per_cta);
+        grid = grid_for(fp4::nvfp4_quantize_kernel<uint16_t>, n_blocks, per_cta);
     else
-        grid = grid_for(fp4::nvfp4_quantize_kernel<float>, n_units, per_cta);
+        grid = grid_for(fp4::nvfp4_quantize_kernel<float>, n_blocks, per_cta);
     if (grid <= 0)
         return FP4_ERR_CUDA;
-    uint32_t *pk = reinterpret_cast<uint32_t *>(packed);
+    uint2 *pk = reinterpret_cast<uint2 *>(packed);
     if (dt == FP4_BF16)
-        fp4::nvfp4_quantize_kernel<uint16_t><<<grid, kThreads, 0, stream>>>(
-            static_cast<const uint16_t *>(x), n_units, partials, nparts, pk, scales, global_scale,
-            status);
-    else
-        fp4::nvfp4_quantize_kernel<float><<<grid, kThreads, 0, stream>>>(
-            static_cast<const float *>(x), n_units, partials, nparts, pk, scales, global_scale,
-            status);
-    return launched();
+        return launch(fp4::nvfp4_quantize_kernel<uint16_t>, grid, stream,
+                      static_cast<const uint16_t *>(x), n_blocks, amax, pk, scales, global_scale,
+                      status);
+    return launch(fp4::nvfp4_quantize_kernel<float>, grid, stream, static_cast<const float *>(x),
+                  n_blocks, amax, pk, scales, global_scale, status);
 }
 
 } // namespace
@@ -149,7 +164,7 @@ const char *fp4_status_string(int status)
     case FP4_OK: return "ok";
     case FP4_ERR_INVALID_ARG: return "invalid argument";
     case FP4_ERR_SHAPE: return "shape: incomplete block or size overflow";
-    case FP4_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case FP4_ERR_ALIGN: return "pointer misaligned (x, y: 32 bytes; packed: 16 bytes)";
     case FP4_ERR_NONFINITE: return "non-finite input";
     case FP4_ERR_RANGE: return "global scale out of range";
     case FP4_ERR_WORKSPACE: return "workspace missing or too small";
@@ -165,7 +180,7 @@ size_t fp4_workspace_bytes(fp4_format fmt, int64_t rows, int64_t cols)
     (void)fmt;
     (void)rows;
     (void)cols;
-    return (size_t)kMaxPartials * sizeof(uint32_t);
+    return kWsWords * sizeof(uint32_t);
 }
 
 fp4_status fp4_tensor_amax(const void *x, fp4_dtype dtype, int64_t n, float *amax,
@@ -174,17 +189,12 @@ fp4_status fp4_tensor_amax(const void *x, fp4_dtype dtype, int64_t n, float *ama
 {
     if (!amax || !status || !valid_dtype(dtype) || n < 0 || (n > 0 && !x))
         return FP4_ERR_INVALID_ARG;
-    if (!aligned(x, 16))
+    if (!aligned(x, 32))
         return FP4_ERR_ALIGN;
     if (!workspace || workspace_bytes < fp4_workspace_bytes(FP4_NVFP4, 1, n) ||
         !aligned(workspace, 4))
         return FP4_ERR_WORKSPACE;
-    uint32_t *partials = static_cast<uint32_t *>(workspace);
-    const int nparts = launch_amax_partials(x, dtype, n, partials, stream);
-    if (nparts < 0)
-        return FP4_ERR_CUDA;
-    fp4::amax_finalize_kernel<<<1, kThreads, 0, stream>>>(partials, nparts, amax, status);
-    return launched();
+    return launch_amax(x, dtype, n, static_cast<uint32_t *>(workspace), amax, status, stream);
 }
 
 fp4_status fp4_nvfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
@@ -200,17 +210,17 @@ fp4_status fp4_nvfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int6
     const int64_t n = rows * cols;
     if (n > 0 && (!x || !packed || !scales))
         return FP4_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(packed, 16))
+    if (!aligned(x, 32) || !aligned(packed, 16))
         return FP4_ERR_ALIGN;
     if (!workspace || workspace_bytes < fp4_workspace_bytes(FP4_NVFP4, rows, cols) ||
         !aligned(workspace, 4))
         return FP4_ERR_WORKSPACE;
-    uint32_t *partials = static_cast<uint32_t *>(workspace);
-    const int nparts = launch_amax_partials(x, dtype, n, partials, stream);
-    if (nparts < 0)
-        return FP4_ERR_CUDA;
-    return launch_nv_quantize(x, dtype, n, partials, nparts, packed, scales, global_scale, status,
-                              stream);
+    uint32_t *ws = static_cast<uint32_t *>(workspace);
+    float *amax = reinterpret_cast<float *>(ws + kWsAmax);
+    st = launch_amax(x, dtype, n, ws, amax, status, stream);
+    if (st != FP4_OK)
+        return st;
+    return launch_nv_quantize(x, dtype, n, amax, packed, scales, global_scale, status, stream);
 }
 
 fp4_status fp4_nvfp4_quantize_with_amax(const void *x, fp4_dtype dtype, int64_t rows,
@@ -226,10 +236,9 @@ fp4_status fp4_nvfp4_quantize_with_amax(const void *x, fp4_dtype dtype, int64_t 
     const int64_t n = rows * cols;
     if (n > 0 && (!x || !packed || !scales))
         return FP4_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(amax, 4))
+    if (!aligned(x, 32) || !aligned(packed, 16) || !aligned(amax, 4))
         return FP4_ERR_ALIGN;
-    return launch_nv_quantize(x, dtype, n, reinterpret_cast<const uint32_t *>(amax), 1, packed,
-                              scales, global_scale, status, stream);
+    return launch_nv_quantize(x, dtype, n, amax, packed, scales, global_scale, status, stream);
 }
 
 fp4_status fp4_mxfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
@@ -246,25 +255,24 @@ fp4_status fp4_mxfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int6
         return FP4_OK;
     if (!x || !packed || !scales)
         return FP4_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(packed, 16))
+    if (!aligned(x, 32) || !aligned(packed, 16))
         return FP4_ERR_ALIGN;
-    const int64_t n_units = n / 8;
+    const int64_t n_blocks = n / 32;
     const int64_t per_cta = (int64_t)kThreads * 2;
-    uint32_t *pk = reinterpret_cast<uint32_t *>(packed);
+    uint4 *pk = reinterpret_cast<uint4 *>(packed);
     if (dtype == FP4_BF16) {
-        const int grid = grid_for(fp4::mxfp4_quantize_kernel<uint16_t>, n_units, per_cta);
+        const int grid = grid_for(fp4::mxfp4_quantize_kernel<uint16_t>, n_blocks, per_cta);
         if (grid <= 0)
             return FP4_ERR_CUDA;
-        fp4::mxfp4_quantize_kernel<uint16_t><<<grid, kThreads, 0, stream>>>(
-            static_cast<const uint16_t *>(x), n_units, pk, scales, status);
+        return launch(fp4::mxfp4_quantize_kernel<uint16_t>, grid, stream,
+                      static_cast<const uint16_t *>(x), n_blocks, pk, scales, status);
     } else {
-        const int grid = grid_for(fp4::mxfp4_quantize_kernel<float>, n_units, per_cta);
+        const int grid = grid_for(fp4::mxfp4_quantize_kernel<float>, n_blocks, per_cta);
         if (grid <= 0)
             return FP4_ERR_CUDA;
-        fp4::mxfp4_quantize_kernel<float><<<grid, kThreads, 0, stream>>>(
-            static_cast<const float *>(x), n_units, pk, scales, status);
+        return launch(fp4::mxfp4_quantize_kernel<float>, grid, stream,
+                      static_cast<const float *>(x), n_blocks, pk, scales, status);
     }
-    return launched();
 }
 
 fp4_status fp4_dequantize(fp4_format fmt, const uint8_t *packed, const uint8_t *scales,
@@ -282,18 +290,18 @@ fp4_status fp4_dequantize(fp4_format fmt, const uint8_t *packed, const uint8_t *
         return FP4_OK;
     if (!packed || !scales || !y || (nv && !global_scale))
         return FP4_ERR_INVALID_ARG;
-    if (!aligned(packed, 16) || !aligned(y, 16) || (nv && !aligned(global_scale, 4)))
+    if (!aligned(packed, 16) || !aligned(y, 32) || (nv && !aligned(global_scale, 4)))
         return FP4_ERR_ALIGN;
-    const int64_t n_units = n / 8;
-    const int64_t per_cta = (int64_t)kThreads * 4;
-    const uint32_t *pk = reinterpret_cast<const uint32_t *>(packed);
+    const int64_t n_units = n / 16;
+    const int64_t per_cta = (int64_t)kThreads * 2;
+    const uint2 *pk = reinterpret_cast<const uint2 *>(packed);
 #define FP4_DEQ_LAUNCH(NV, TOUT)                                                                \
     do {                                                                                        \
         const int grid = grid_for(fp4::dequantize_kernel<NV, TOUT>, n_units, per_cta);          \
         if (grid <= 0)                                                                          \
             return FP4_ERR_CUDA;                                                                \
-        fp4::dequantize_kernel<NV, TOUT><<<grid, kThreads, 0, stream>>>(                        \
-            pk, scales, global_scale, n_units, static_cast<TOUT *>(y));                         \
+        return launch(fp4::dequantize_kernel<NV, TOUT>, grid, stream, pk, scales, global_scale, \
+                      n_units, static_cast<TOUT *>(y));                                         \
     } while (0)
     if (nv && out_dtype == FP4_BF16)
         FP4_DEQ_LAUNCH(true, uint16_t);
@@ -304,12 +312,11 @@ fp4_status fp4_dequantize(fp4_format fmt, const uint8_t *packed, const uint8_t *
     else
         FP4_DEQ_LAUNCH(false, float);
 #undef FP4_DEQ_LAUNCH
-    return launched();
 }
 
 namespace {
-fp4_status launch_search(const void *x, fp4_dtype dtype, int64_t n, const uint32_t *partials,
-                         int nparts, uint8_t *packed, uint8_t *scales, float *global_scale,
+fp4_status launch_search(const void *x, fp4_dtype dtype, int64_t n, const float *amax,
+                         uint8_t *packed, uint8_t *scales, float *global_scale,
                          float *block_loss, int32_t *status, cudaStream_t stream)
 {
     const int64_t n_blocks = n / 16;
@@ -318,18 +325,17 @@ fp4_status launch_search(const void *x, fp4_dtype dtype, int64_t n, const uint32
         const int grid = grid_for(fp4::scale_search_kernel<uint16_t>, n_blocks, kThreads);
         if (grid <= 0)
             return FP4_ERR_CUDA;
-        fp4::scale_search_kernel<uint16_t><<<grid, kThreads, 0, stream>>>(
-            static_cast<const uint16_t *>(x), n_blocks, partials, nparts, pk, scales,
-            global_scale, block_loss, status);
+        return launch(fp4::scale_search_kernel<uint16_t>, grid, stream,
+                      static_cast<const uint16_t *>(x), n_blocks, amax, pk, scales, global_scale,
+                      block_loss, status);
     } else {
         const int grid = grid_for(fp4::scale_search_kernel<float>, n_blocks, kThreads);
         if (grid <= 0)
             return FP4_ERR_CUDA;
-        fp4::scale_search_kernel<float><<<grid, kThreads, 0, stream>>>(
-            static_cast<const float *>(x), n_blocks, partials, nparts, pk, scales, global_scale,
-            block_loss, status);
+        return launch(fp4::scale_search_kernel<float>, grid, stream,
+                      static_cast<const float *>(x), n_blocks, amax, pk, scales, global_scale,
+                      block_loss, status);
     }
-    return launched();
 }
 } // namespace
 
@@ -346,17 +352,18 @@ fp4_status fp4_scale_search(const void *x, fp4_dtype dtype, int64_t rows, int64_
     const int64_t n = rows * cols;
     if (n > 0 && (!x || !packed || !scales))
         return FP4_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(block_loss, 4))
+    if (!aligned(x, 32) || !aligned(packed, 16) || !aligned(block_loss, 4))
         return FP4_ERR_ALIGN;
     if (!workspace || workspace_bytes < fp4_workspace_bytes(FP4_NVFP4, rows, cols) ||
         !aligned(workspace, 4))
         return FP4_ERR_WORKSPACE;
-    uint32_t *partials = static_cast<uint32_t *>(workspace);
-    const int nparts = launch_amax_partials(x, dtype, n, partials, stream);
-    if (nparts < 0)
-        return FP4_ERR_CUDA;
-    return launch_search(x, dtype, n, partials, nparts, packed, scales, global_scale, block_loss,
-                         status, stream);
+    uint32_t *ws = static_cast<uint32_t *>(workspace);
+    float *amax = reinterpret_cast<float *>(ws + kWsAmax);
+    st = launch_amax(x, dtype, n, ws, amax, status, stream);
+    if (st != FP4_OK)
+        return st;
+    return launch_search(x, dtype, n, amax, packed, scales, global_scale, block_loss, status,
+                         stream);
 }
 
 fp4_status fp4_scale_search_with_amax(const void *x, fp4_dtype dtype, int64_t rows,
@@ -372,10 +379,10 @@ fp4_status fp4_scale_search_with_amax(const void *x, fp4_dtype dtype, int64_t ro
     const int64_t n = rows * cols;
     if (n > 0 && (!x || !packed || !scales))
         return FP4_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(block_loss, 4) || !aligned(amax, 4))
+    if (!aligned(x, 32) || !aligned(packed, 16) || !aligned(block_loss, 4) || !aligned(amax, 4))
         return FP4_ERR_ALIGN;
-    return launch_search(x, dtype, n, reinterpret_cast<const uint32_t *>(amax), 1, packed, scales,
-                         global_scale, block_loss, status, stream);
+    return launch_search(x, dtype, n, amax, packed, scales, global_scale, block_loss, status,
+                         stream);
 }
 
 fp4_status fp4_e2m1_round(const float *v, uint8_t *codes, int64_t n, cudaStream_t stream)
@@ -387,8 +394,19 @@ fp4_status fp4_e2m1_round(const float *v, uint8_t *codes, int64_t n, cudaStream_
     const int grid = grid_for(fp4::e2m1_round_kernel, (n + 7) / 8, kThreads);
     if (grid <= 0)
         return FP4_ERR_CUDA;
-    fp4::e2m1_round_kernel<<<grid, kThreads, 0, stream>>>(v, codes, n);
-    return launched();
+    return launch(fp4::e2m1_round_kernel, grid, stream, v, codes, n);
+}
+
+fp4_status fp4_e2m1_roundtrip(const float *v, float *out, int64_t n, cudaStream_t stream)
+{
+    if (n < 0 || (n > 0 && (!v || !out)))
+        return FP4_ERR_INVALID_ARG;
+    if (n == 0)
+        return FP4_OK;
+    const int grid = grid_for(fp4::e2m1_roundtrip_kernel, (n + 7) / 8, kThreads);
+    if (grid <= 0)
+        return FP4_ERR_CUDA;
+    return launch(fp4::e2m1_roundtrip_kernel, grid, stream, v, out, n);
 }
 
 fp4_status fp4_nv_encode_quotient(const float *x, const float *d, uint8_t *codes, int64_t n,
@@ -401,8 +419,7 @@ fp4_status fp4_nv_encode_quotient(const float *x, const float *d, uint8_t *codes
     const int grid = grid_for(fp4::nv_encode_quotient_kernel, n, kThreads);
     if (grid <= 0)
         return FP4_ERR_CUDA;
-    fp4::nv_encode_quotient_kernel<<<grid, kThreads, 0, stream>>>(x, d, codes, n);
-    return launched();
+    return launch(fp4::nv_encode_quotient_kernel, grid, stream, x, d, codes, n);
 }
 
 } // extern "C"

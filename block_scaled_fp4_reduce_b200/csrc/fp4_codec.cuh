@@ -21,7 +21,8 @@ namespace fp4 {
 // E2M1 encode: eight fp32 values -> eight packed codes in one u32.
 // Byte j holds element 2j in its low nibble and 2j+1 in its high nibble.
 // `cvt.rn.satfinite.e2m1x2.f32 d, a, b` rounds to nearest even, saturates
-// to +-6 and puts `a` in the high nibble, `b` in the low one.
+// to +-6 and puts `a` in the high nibble, `b` in the low one; the four bytes
+// are packed with one vector move.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4,
                                            float v5, float v6, float v7)
@@ -47,21 +48,30 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8])
 
 // ---------------------------------------------------------------------------
 // E2M1 decode: eight packed codes -> eight fp32 values (code 8 = -0).
-// `cvt.rn.f16x2.e2m1x2` widens a byte of two codes to f16x2 exactly (high
-// nibble -> high half); the f16 -> f32 widening is exact too.
+// `cvt.rn.f16x2.e2m1x2` widens one byte of two codes to f16x2 exactly (high
+// nibble -> high half); the f16 -> f32 widening is exact too.  Each byte is
+// shifted down in a 32-bit register and narrowed on its own (cvt.u8.u32):
+// unpacking a word with one vector move into four 8-bit registers straight
+// after the encoder packed it was seen to return wrong upper bytes.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte_in_low_bits)
+{
+    uint32_t h;
+    asm("{\n\t"
+        ".reg .b8 q;\n\t"
+        "cvt.u8.u32 q, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, q;\n\t"
+        "}"
+        : "=r"(h)
+        : "r"(byte_in_low_bits));
+    return h;
+}
+
 __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t packed, uint32_t (&h)[4])
 {
-    asm("{\n\t"
-        ".reg .b8 b0, b1, b2, b3;\n\t"
-        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t"
-        "}"
-        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-        : "r"(packed));
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        h[j] = e2m1x2_to_f16x2(packed >> (8 * j));
 }
 
 __device__ __forceinline__ void f16x2_to_f32(uint32_t h, float &lo, float &hi)
@@ -83,6 +93,27 @@ __device__ __forceinline__ void e2m1x8_decode(uint32_t packed, float (&p)[8])
 #pragma unroll
     for (int j = 0; j < 4; ++j)
         f16x2_to_f32(h[j], p[2 * j], p[2 * j + 1]);
+}
+
+// Round eight fp32 values to the E2M1 grid and return the grid values
+// (quantise-dequantise), each pair converted to codes and back inside one
+// asm block so that the codes never leave their 8-bit registers: the codes
+// are not needed, and a packed word built from `cvt ... e2m1x2` results that
+// is unpacked again straight away was seen to lose its upper two bytes.
+__device__ __forceinline__ void e2m1x8_qdq(const float (&v)[8], float (&p)[8])
+{
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t h;
+        asm("{\n\t"
+            ".reg .b8 q;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 q, %2, %1;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %0, q;\n\t"
+            "}"
+            : "=r"(h)
+            : "f"(v[2 * j]), "f"(v[2 * j + 1]));
+        f16x2_to_f32(h, p[2 * j], p[2 * j + 1]);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -123,23 +154,35 @@ __device__ __forceinline__ uint32_t e4m3_code_from_f64(double t)
     return (uint32_t)((E + 6) * 8) + m;
 }
 
-// NVFP4 block-scale code: E4M3 nearest to the exact rational A_b / (6 g).
-// Fast path: t = RN(A_b * RN(1/(6g))) is within 2^-23 relative of the
-// rational, i.e. a few units in its last place, and `cvt.rn.satfinite.e4m3x2`
-// rounds t once to E4M3 (saturating at 448).  Every E4M3 midpoint, and every
-// E4M3 value, is an fp32 pattern whose 19 low fraction bits are zero; when t
-// lies more than 16 units from such a pattern, t and the rational round to
-// the same code.  Otherwise (and never for t < 2^-11, which is always code
-// 0) the rational is formed as one correctly rounded double quotient.
-__device__ __forceinline__ uint32_t nv_scale_code(float amax_b, float inv6g, double six_g)
+// Block-scale code: E4M3 nearest to the exact rational num * A_b / den
+// (NVFP4: num = 1, den = 6g; the search's smallest candidate: num = 147,
+// den = 1260 g), given inv = RN32(num / den).
+// Fast path: t = RN(A_b * inv) is within 2^-23 relative of the rational, a
+// few units in its last place, and `cvt.rn.satfinite.e4m3x2` rounds t once
+// to E4M3 (saturating at 448).  Every E4M3 midpoint, and every E4M3 value,
+// is an fp32 pattern whose 19 low fraction bits are zero; when t lies more
+// than 16 units from such a pattern, t and the rational round to the same
+// code.  Otherwise (never for t < 2^-11, which is always code 0) the rational
+// is formed as one correctly rounded double quotient (num * A_b and den are
+// exact in double).
+__device__ __forceinline__ uint32_t nv_scale_code(float amax_b, float inv, double num, double den)
 {
-    float t = __fmul_rn(amax_b, inv6g);
-    uint32_t tb = __float_as_uint(t);
+    const float t = __fmul_rn(amax_b, inv);
+    const uint32_t tb = __float_as_uint(t);
     if (tb > 0x3A000000u && ((tb + 16u) & 0x7FFFFu) < 32u)
-        return e4m3_code_from_f64(__ddiv_rn((double)amax_b, six_g));
+        return e4m3_code_from_f64(__ddiv_rn(num * (double)amax_b, den));
     uint16_t c;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(0.0f), "f"(t));
     return (uint32_t)(c & 0xFFu);
+}
+
+// Value of a positive E4M3 code 0..126: codes >= 8 are normal, exponent
+// field e = c / 8 and fraction f = c % 8 give the fp32 pattern
+// (e + 120) << 23 | f << 20 = (c << 20) + (120 << 23); codes below 8 are
+// the subnormals c * 2^-9.
+__device__ __forceinline__ float e4m3_pos_to_f32(uint32_t c)
+{
+    return c >= 8u ? __uint_as_float((c << 20) + 0x3C000000u) : (float)c * 0x1p-9f;
 }
 
 // ---------------------------------------------------------------------------
@@ -176,30 +219,46 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t byte)
 // NVFP4 element quotient v = fl32(x / d) followed by E2M1 rounding, for
 // eight elements sharing d = fl32(s_b * g) > 0.
 //
-// Bracketing instead of dividing: with r = RN(1/d) (IEEE reciprocal) the
-// neighbours r_lo = pred(r) and r_hi = succ(r) satisfy r_lo <= 1/d <= r_hi
-// exactly, so x*r_lo and x*r_hi bracket x/d, and since rounding to nearest
-// is monotone, RN(x*r_lo) and RN(x*r_hi) bracket v = RN(x/d) in magnitude,
-// all three with the sign of x.  The E2M1 code is a monotone function of
-// the magnitude, so when both brackets give the same code, v has it too.
-// Only when a midpoint of the E2M1 grid falls inside the two-ulp bracket
-// (about one element in a million for random data, and exact ties) do the
-// eight elements take the IEEE single division.  A d below the smallest
-// normal fp32 (1/d could overflow) always takes the division.
+// Bracketing instead of dividing: with r_lo <= 1/d <= r_hi (exact reals,
+// see nv_recip), x*r_lo and x*r_hi bracket x/d, and since rounding to
+// nearest is monotone, RN(x*r_lo) and RN(x*r_hi) bracket v = RN(x/d) in
+// magnitude, all three with the sign of x.  The E2M1 code is a monotone
+// function of the magnitude, so when both brackets give the same code, v
+// has it too.  Only when a midpoint of the E2M1 grid falls inside the
+// eight-ulp bracket (a few elements in a million for random data, and exact
+// ties) do the eight elements take the IEEE single division.  A d below the
+// smallest normal fp32 always takes the division.
 // ---------------------------------------------------------------------------
 struct NvRecip {
     float d, lo, hi;
     bool exact_only;
 };
 
+__device__ __forceinline__ float rcp_approx(float d)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+    return r;
+}
+
+// Reciprocal bracket of d.  r0 = rcp.approx(d) has a relative error far
+// below 2^-12; one Newton step r1 = r0 + r0 (1 - d r0) (two FMAs) leaves
+// |r1 d - 1| <= delta^2 + delta u + u < 2^-23 (u = 2^-24), i.e. at most two
+// units in the last place of r1, four bit patterns when 1/d sits just below a
+// power of two.  So r1 - 4 and r1 + 4 (as bit patterns) bracket 1/d exactly.
+// d is normal here (>= 2^-126) and at most 2^125.5 (448 g, g <= FLT_MAX/2688),
+// so 1/d and its neighbours are normal.
 __device__ __forceinline__ NvRecip nv_recip(float d)
 {
     NvRecip q;
     q.d = d;
     q.exact_only = !(d >= 0x1p-126f);
-    float r = __frcp_rn(q.exact_only ? 1.0f : d);
-    q.lo = __uint_as_float(__float_as_uint(r) - 1u);
-    q.hi = __uint_as_float(__float_as_uint(r) + 1u);
+    const float dd = q.exact_only ? 1.0f : d;
+    const float r0 = rcp_approx(dd);
+    const float e = fmaf(-dd, r0, 1.0f);
+    const float r1 = fmaf(r0, e, r0);
+    q.lo = __uint_as_float(__float_as_uint(r1) - 4u);
+    q.hi = __uint_as_float(__float_as_uint(r1) + 4u);
     return q;
 }
 
@@ -212,7 +271,7 @@ __device__ __forceinline__ uint32_t nv_encode8(const float (&x)[8], const NvReci
         b[i] = __fmul_rn(x[i], q.hi);
     }
     uint32_t ca = e2m1x8(a);
-    uint32_t cb = e2m1x8(b);
+    const uint32_t cb = e2m1x8(b);
     if (ca != cb || q.exact_only) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
@@ -229,59 +288,24 @@ __device__ __forceinline__ float nv_dequant(float p, float sb, float g)
 }
 
 // ---------------------------------------------------------------------------
-// Loads: eight consecutive input elements as fp32.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 &w, float (&x)[8])
+// 32-byte (256-bit) vector load / store, sm_100 and later.  Loads are
+// cached in L2 only (.cg): data is streamed once, and with launch chaining a
+// kernel may start while its predecessor still runs, so inputs are never
+// read through the non-coherent path.
+__device__ __forceinline__ void ldg_v8(const void *p, uint32_t *w)
 {
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        x[2 * j] = __uint_as_float(ws[j] << 16);
-        x[2 * j + 1] = __uint_as_float(ws[j] & 0xFFFF0000u);
-    }
+    asm volatile("ld.global.cg.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+          "=r"(w[7])
+        : "l"(p));
 }
 
-// max over eight bf16 of the |x| bit pattern, as an fp32 bit pattern.
-// Non-negative floats order like their bit patterns; NaN / Inf patterns
-// (>= 0x7F80 in bf16) sort above every finite value.
-__device__ __forceinline__ uint32_t bf16x8_absmax_bits(const uint4 &w)
+__device__ __forceinline__ void stg_v8(void *p, const uint32_t *w)
 {
-    uint32_t m = __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
-                          __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
-    return max(m & 0xFFFFu, m >> 16) << 16;
-}
-
-__device__ __forceinline__ uint32_t f32x4_absmax_bits(const uint4 &w)
-{
-    return max(max(w.x & 0x7FFFFFFFu, w.y & 0x7FFFFFFFu),
-               max(w.z & 0x7FFFFFFFu, w.w & 0x7FFFFFFFu));
-}
-
-__device__ __forceinline__ uint4 ldg_stream(const void *p)
-{
-    uint4 v;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-// Store one 16-byte vector without keeping it in L1 / with streaming hint.
-__device__ __forceinline__ void stg_stream(void *p, const uint4 &v)
-{
-    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w)
+    asm volatile("st.global.cs.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+                 "r"(w[7])
                  : "memory");
-}
-
-// Eight fp32 -> eight bf16 (round to nearest even) packed in a uint4.
-__device__ __forceinline__ uint4 f32x8_to_bf16x8(const float (&y)[8])
-{
-    uint32_t o[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(y[2 * j + 1]), "f"(y[2 * j]));
-    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 } // namespace fp4

@@ -1,9 +1,8 @@
 // fp4_kernels.cuh -- sm_100a kernels of the block-scaled FP4 path.
 //
-//   amax_partial_kernel   tensor amax, first pass: per-CTA max |x| bit
-//                         pattern into a workspace word ("NVFP4 与 MXFP4 格式"
-//                         section 3: A, the tensor absolute maximum)
-//   amax_finalize_kernel  one CTA folds the partials into one fp32
+//   amax_kernel           tensor amax ("NVFP4 与 MXFP4 格式" section 3: A, the
+//                         tensor absolute maximum): per-CTA maxima, folded by
+//                         the last CTA to finish, in one launch
 //   nvfp4_quantize_kernel block amax, E4M3 scale, element quotient, E2M1
 //                         rounding and nibble packing in one pass (section 3)
 //   mxfp4_quantize_kernel the same for 32-blocks with an E8M0 scale (section 5)
@@ -11,13 +10,20 @@
 //   scale_search_kernel   per-block MSE-minimising E4M3 scale
 //                         ("FP4 / NVFP4 数学总结" section 9)
 //
-// All of the path is HBM-bound streaming except the scale search.  Loads
-// are 16-byte vectors through the non-coherent path with no L1 allocation;
-// one thread handles eight consecutive elements (one 16-byte bf16 vector)
-// per unit, so two adjacent lanes share an NVFP4 block and four an MXFP4
-// block, and a warp reads 512 contiguous bytes per load instruction.
-// Grids are persistent: SM count x resident CTAs, grid-striding over the
-// tensor.
+// Layout of the work: one thread owns one whole block (16 elements for
+// NVFP4 and the search, 32 for MXFP4) and reads it with 256-bit loads
+// (`ld.global.cg.v8`, new on sm_100), so consecutive lanes
+// read consecutive 32-byte sectors and every per-block step (amax, scale,
+// reciprocal) runs once per block.  Grids are persistent: SMs x resident
+// CTAs, grid-striding over the blocks, two blocks in flight per thread.
+// Everything is HBM-bound streaming except the scale search (issue-bound).
+//
+// Launch chaining: every kernel is launched with programmatic stream
+// serialisation.  It lets the next kernel on the stream launch at once
+// (griddepcontrol.launch_dependents) and waits for the previous one
+// (griddepcontrol.wait) before its first global memory access, so launch
+// latency and the CTA ramp overlap the previous kernel's tail.  Loads after
+// the wait go through L2 (.cg / coherent), never the non-coherent path.
 #pragma once
 
 #include <cstdint>
@@ -59,112 +65,170 @@ __device__ __forceinline__ uint32_t cta_max_u32(uint32_t v)
     return s_res;
 }
 
-// Elements of type T in one 16-byte vector, and the vectors of one unit of
-// eight elements.
-template <typename T> struct Vec;
-template <> struct Vec<float> {
-    static constexpr int kPerUnit = 2;
-};
-template <> struct Vec<uint16_t> { // bf16 bit patterns
-    static constexpr int kPerUnit = 1;
+// ---------------------------------------------------------------------------
+// A block of N input elements of type T (float, or uint16_t = bf16 bits) as
+// raw 32-bit words, loaded with 256-bit vectors.
+// ---------------------------------------------------------------------------
+template <typename T, int N> struct Blk {
+    static constexpr int kWords = N * (int)sizeof(T) / 4;
+    static_assert(kWords % 8 == 0, "blocks are whole 32-byte vectors");
+    uint32_t w[kWords];
 };
 
-template <typename T>
-__device__ __forceinline__ void load_unit(const uint4 *xv, int64_t unit, bool valid, uint4 (&w)[2])
+template <typename T, int N>
+__device__ __forceinline__ void load_blk(const T *x, int64_t b, Blk<T, N> &k)
 {
+    const char *p = reinterpret_cast<const char *>(x) + b * (int64_t)(N * sizeof(T));
 #pragma unroll
-    for (int k = 0; k < Vec<T>::kPerUnit; ++k)
-        w[k] = valid ? ldg_stream(xv + unit * Vec<T>::kPerUnit + k) : make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < Blk<T, N>::kWords; j += 8)
+        ldg_v8(p + 4 * j, &k.w[j]);
 }
 
-template <typename T>
-__device__ __forceinline__ uint32_t unit_to_f32(const uint4 (&w)[2], float (&x)[8])
+// max |x| over the block as an fp32 bit pattern.  Non-negative floats order
+// like their bit patterns; NaN / Inf patterns sort above every finite value.
+template <typename T, int N>
+__device__ __forceinline__ uint32_t absmax_bits(const Blk<T, N> &k)
 {
-    if constexpr (Vec<T>::kPerUnit == 1) {
-        bf16x8_to_f32(w[0], x);
-        return bf16x8_absmax_bits(w[0]);
-    } else {
-        const uint32_t ws[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+    constexpr int W = Blk<T, N>::kWords;
+    uint32_t m[W];
+    if constexpr (sizeof(T) == 2) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            x[i] = __uint_as_float(ws[i]);
-        return max(f32x4_absmax_bits(w[0]), f32x4_absmax_bits(w[1]));
+        for (int j = 0; j < W; ++j)
+            m[j] = k.w[j] & 0x7FFF7FFFu;
+#pragma unroll
+        for (int s = W / 2; s >= 1; s /= 2)
+#pragma unroll
+            for (int j = 0; j < s; ++j)
+                m[j] = __vmaxu2(m[j], m[j + s]);
+        return max(m[0] & 0xFFFFu, m[0] >> 16) << 16;
+    } else {
+#pragma unroll
+        for (int j = 0; j < W; ++j)
+            m[j] = k.w[j] & 0x7FFFFFFFu;
+#pragma unroll
+        for (int s = W / 2; s >= 1; s /= 2)
+#pragma unroll
+            for (int j = 0; j < s; ++j)
+                m[j] = max(m[j], m[j + s]);
+        return m[0];
     }
 }
 
+// max |x| over a block known to be finite, as an fp32 bit pattern: bf16
+// pairs go through packed `max.bf16x2` on absolute values (two elements per
+// instruction); fp32 through the integer path above.
+template <typename T, int N>
+__device__ __forceinline__ uint32_t absmax_bits_finite(const Blk<T, N> &k)
+{
+    if constexpr (sizeof(T) == 2) {
+        constexpr int W = Blk<T, N>::kWords;
+        uint32_t m[W];
+#pragma unroll
+        for (int j = 0; j < W; ++j)
+            m[j] = k.w[j] & 0x7FFF7FFFu;
+#pragma unroll
+        for (int s = W / 2; s >= 1; s /= 2)
+#pragma unroll
+            for (int j = 0; j < s; ++j)
+                asm("max.bf16x2 %0, %1, %2;" : "=r"(m[j]) : "r"(m[j]), "r"(m[j + s]));
+        uint32_t r;
+        asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(m[0]), "r"(__funnelshift_l(m[0], m[0], 16)));
+        return r << 16;
+    } else {
+        return absmax_bits(k);
+    }
+}
+
+// Element i of the block as fp32 (exact).
+template <typename T, int N>
+__device__ __forceinline__ float elem(const Blk<T, N> &k, int i)
+{
+    if constexpr (sizeof(T) == 2)
+        return __uint_as_float((i & 1) ? (k.w[i >> 1] & 0xFFFF0000u) : (k.w[i >> 1] << 16));
+    else
+        return __uint_as_float(k.w[i]);
+}
+
+template <typename T, int N>
+__device__ __forceinline__ void elems8(const Blk<T, N> &k, int first, float (&x)[8])
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        x[i] = elem(k, first + i);
+}
+
+__device__ __forceinline__ void pdl_begin()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
-// Tensor amax, pass 1: partials[blockIdx.x] = max over the CTA's share of
-// the |x| bit pattern (an fp32 pattern; >= 0x7F800000 flags NaN / Inf).
+// Tensor amax in one launch.  Each CTA writes the max |x| bit pattern of its
+// share to ws[blockIdx.x]; the last CTA to finish (counted with a wrapping
+// atomicInc on ws[kMaxPartials], which returns to 0 after every launch)
+// folds the partials and writes A as fp32 to *amax (NaN / Inf flags
+// FP4_ERR_NONFINITE).  32-byte loads, four in flight per thread.
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-    amax_partial_kernel(const T *__restrict__ x, int64_t n, uint32_t *__restrict__ partials)
+    amax_kernel(const T *__restrict__ x, int64_t n, uint32_t *ws, float *amax, int32_t *status)
 {
-    constexpr int kElemsPerVec = 16 / (int)sizeof(T);
+    pdl_begin();
+    constexpr int kPerVec = 32 / (int)sizeof(T);
     constexpr int kUnroll = 4;
-    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
-    const int64_t nvec = n / kElemsPerVec;
+    const int64_t nvec = n / kPerVec;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     uint32_t m = 0;
     for (; i + (kUnroll - 1) * stride < nvec; i += kUnroll * stride) {
-        uint4 w[kUnroll];
+        Blk<T, kPerVec> v[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u)
-            w[u] = ldg_stream(xv + i + u * stride);
+            load_blk(x, i + u * stride, v[u]);
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            if constexpr (sizeof(T) == 2)
-                m = max(m, bf16x8_absmax_bits(w[u]));
-            else
-                m = max(m, f32x4_absmax_bits(w[u]));
-        }
+        for (int u = 0; u < kUnroll; ++u)
+            m = max(m, absmax_bits(v[u]));
     }
     for (; i < nvec; i += stride) {
-        uint4 w = ldg_stream(xv + i);
-        if constexpr (sizeof(T) == 2)
-            m = max(m, bf16x8_absmax_bits(w));
-        else
-            m = max(m, f32x4_absmax_bits(w));
+        Blk<T, kPerVec> v;
+        load_blk(x, i, v);
+        m = max(m, absmax_bits(v));
     }
-    if (blockIdx.x == 0) { // elements past the last whole vector
-        for (int64_t j = nvec * kElemsPerVec + threadIdx.x; j < n; j += blockDim.x) {
+    if (blockIdx.x == 0) { // elements past the last whole 32-byte vector
+        for (int64_t j = nvec * kPerVec + threadIdx.x; j < n; j += blockDim.x) {
             uint32_t b;
             if constexpr (sizeof(T) == 2)
-                b = ((uint32_t)x[j] & 0x7FFFu) << 16;
+                b = ((uint32_t)__ldcg(x + j) & 0x7FFFu) << 16;
             else
-                b = __float_as_uint(x[j]) & 0x7FFFFFFFu;
+                b = __float_as_uint(__ldcg(x + j)) & 0x7FFFFFFFu;
             m = max(m, b);
         }
     }
     m = cta_max_u32(m);
-    if (threadIdx.x == 0)
-        partials[blockIdx.x] = m;
-}
-
-// Fold nparts partial maxima (every thread of the CTA gets the result).
-__device__ __forceinline__ uint32_t fold_partials(const uint32_t *partials, int nparts)
-{
-    uint32_t m = 0;
-    for (int i = threadIdx.x; i < nparts; i += blockDim.x)
-        m = max(m, partials[i] & 0x7FFFFFFFu);
-    return cta_max_u32(m);
-}
-
-__global__ void __launch_bounds__(kThreads)
-    amax_finalize_kernel(const uint32_t *__restrict__ partials, int nparts, float *amax,
-                         int32_t *status)
-{
-    uint32_t m = fold_partials(partials, nparts);
+    __shared__ bool s_last;
     if (threadIdx.x == 0) {
-        *amax = __uint_as_float(m);
-        if (m >= kNonFiniteBits)
-            raise_status(status, kStatusNonFinite);
+        ws[blockIdx.x] = m;
+        __threadfence();
+        s_last = atomicInc(&ws[kMaxPartials], gridDim.x - 1) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (s_last) {
+        __threadfence();
+        uint32_t a = 0;
+        for (int k = threadIdx.x; k < (int)gridDim.x; k += blockDim.x)
+            a = max(a, __ldcg(ws + k));
+        a = cta_max_u32(a);
+        if (threadIdx.x == 0) {
+            *amax = __uint_as_float(a);
+            if (a >= kNonFiniteBits)
+                raise_status(status, kStatusNonFinite);
+        }
     }
 }
 
-// The NVFP4 global scale from the folded amax pattern: g = fl32(A / 2688),
-// A = 0 -> 1.  Returns 0 and sets *err for a non-finite A or a g below the
+// The NVFP4 global scale from the amax bit pattern: g = fl32(A / 2688),
+// A = 0 -> 1.  Returns 0 and sets err for a non-finite A or a g below the
 // smallest normal fp32.
 __device__ __forceinline__ float nv_global_scale(uint32_t amax_bits, int32_t &err)
 {
@@ -183,189 +247,195 @@ __device__ __forceinline__ float nv_global_scale(uint32_t amax_bits, int32_t &er
     return g;
 }
 
-// CTA prologue shared by the NVFP4 quantiser and the scale search: fold the
-// amax partials, derive g, publish g / the error from CTA 0.  Returns false
-// when the CTA must stop (data error).
-__device__ __forceinline__ bool nv_prologue(const uint32_t *partials, int nparts,
-                                            float *global_scale, int32_t *status, float &g)
+// Prologue shared by the NVFP4 quantiser and the scale search: read the
+// tensor amax, derive g, publish g / the error from thread 0 of CTA 0.
+// Returns false when the kernel must stop (data error).
+__device__ __forceinline__ bool nv_prologue(const float *amax, float *global_scale,
+                                            int32_t *status, float &g)
 {
-    __shared__ float s_g;
-    __shared__ int32_t s_err;
-    uint32_t a = fold_partials(partials, nparts);
-    if (threadIdx.x == 0) {
-        int32_t err;
-        float gg = nv_global_scale(a, err);
-        if (blockIdx.x == 0) {
-            if (err)
-                raise_status(status, err);
-            else
-                *global_scale = gg;
-        }
-        s_g = gg;
-        s_err = err;
+    int32_t err;
+    g = nv_global_scale(__float_as_uint(__ldcg(amax)) & 0x7FFFFFFFu, err);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (err)
+            raise_status(status, err);
+        else
+            *global_scale = g;
     }
-    __syncthreads();
-    g = s_g;
-    return s_err == 0;
+    return err == 0;
+}
+
+// Per-CTA constants of the NVFP4 block-scale rounding.
+struct NvScaleConsts {
+    float g;
+    float inv6g;  // RN32(1 / (6 g))
+    double six_g; // 6 g, exact in double
+};
+
+__device__ __forceinline__ NvScaleConsts nv_scale_consts(float g)
+{
+    NvScaleConsts c;
+    c.g = g;
+    c.six_g = 6.0 * (double)g;
+    c.inv6g = (float)(1.0 / c.six_g);
+    return c;
+}
+
+// Exact NVFP4 codes of a 16-block at positive scale code c (zero scale ->
+// zero codes): v = fl32(x / fl32(s_b g)), E2M1.
+template <typename T>
+__device__ __forceinline__ uint2 nv_block_codes(const Blk<T, 16> &b, uint32_t c, float g)
+{
+    if (c == 0u)
+        return make_uint2(0u, 0u);
+    const NvRecip q = nv_recip(__fmul_rn(e4m3_pos_to_f32(c), g));
+    float h[8];
+    uint2 pk;
+    elems8(b, 0, h);
+    pk.x = nv_encode8(h, q);
+    elems8(b, 8, h);
+    pk.y = nv_encode8(h, q);
+    return pk;
 }
 
 // ---------------------------------------------------------------------------
-// NVFP4 quantise + pack.  Unit = eight elements (half a block); lanes 2i and
-// 2i+1 of a warp hold one 16-element block.  Per unit: one (bf16) or two
-// (fp32) 16-byte loads, one 4-byte packed store; the even lane stores the
-// scale byte.  The loop bound is warp-uniform so the pair shuffle always
-// sees both lanes.
+// NVFP4 quantise + pack.  One thread per 16-element block: one 32-byte load
+// (bf16) or two (fp32), one 8-byte packed store, one scale byte.
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-    nvfp4_quantize_kernel(const T *__restrict__ x, int64_t n_units,
-                          const uint32_t *__restrict__ partials, int nparts,
-                          uint32_t *__restrict__ packed, uint8_t *__restrict__ scales,
+    nvfp4_quantize_kernel(const T *__restrict__ x, int64_t n_blocks, const float *amax,
+                          uint2 *__restrict__ packed, uint8_t *__restrict__ scales,
                           float *global_scale, int32_t *status)
 {
+    pdl_begin();
     float g;
-    if (!nv_prologue(partials, nparts, global_scale, status, g))
+    if (!nv_prologue(amax, global_scale, status, g))
         return;
-    const double six_g = 6.0 * (double)g;            // exact in double
-    const float inv6g = (float)(1.0 / six_g);        // RN32(RN64(1/(6g)))
-
+    const NvScaleConsts sc = nv_scale_consts(g);
     constexpr int kUnroll = 2;
-    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t base = warp * 32 * kUnroll; base < n_units; base += nwarps * 32 * kUnroll) {
-        uint4 w[kUnroll][2];
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b0 < n_blocks;
+         b0 += kUnroll * stride) {
+        Blk<T, 16> blk[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            if (b0 + u * stride < n_blocks)
+                load_blk(x, b0 + u * stride, blk[u]);
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int64_t unit = base + u * 32 + lane;
-            load_unit<T>(xv, unit, unit < n_units, w[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t unit = base + u * 32 + lane;
-            float xf[8];
-            uint32_t ab = unit_to_f32<T>(w[u], xf);
-            ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, 1));
-            const float amax_b = __uint_as_float(ab);
-            const uint32_t code = nv_scale_code(amax_b, inv6g, six_g);
-            uint32_t pk = 0u;
-            if (code != 0u) {
-                const float sb = e4m3_to_f32(code);
-                pk = nv_encode8(xf, nv_recip(__fmul_rn(sb, g)));
-            }
-            if (unit < n_units) {
-                packed[unit] = pk;
-                if (!(lane & 1))
-                    scales[unit >> 1] = (uint8_t)code;
+            const int64_t b = b0 + u * stride;
+            if (b < n_blocks) {
+                const float amax_b = __uint_as_float(absmax_bits_finite(blk[u]));
+                const uint32_t code = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
+                packed[b] = nv_block_codes(blk[u], code, g);
+                scales[b] = (uint8_t)code;
             }
         }
     }
 }
 
-// NVFP4 quantise with a caller-provided amax (device fp32): same kernel,
-// the amax word acts as a single partial.
-
 // ---------------------------------------------------------------------------
-// MXFP4 quantise + pack.  Lanes 4i..4i+3 hold one 32-element block.
+// MXFP4 quantise + pack.  One thread per 32-element block: two 32-byte loads
+// (bf16) or four (fp32), one 16-byte packed store, one scale byte.
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-    mxfp4_quantize_kernel(const T *__restrict__ x, int64_t n_units,
-                          uint32_t *__restrict__ packed, uint8_t *__restrict__ scales,
+    mxfp4_quantize_kernel(const T *__restrict__ x, int64_t n_blocks,
+                          uint4 *__restrict__ packed, uint8_t *__restrict__ scales,
                           int32_t *status)
 {
+    pdl_begin();
     constexpr int kUnroll = 2;
-    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     bool bad = false;
-    for (int64_t base = warp * 32 * kUnroll; base < n_units; base += nwarps * 32 * kUnroll) {
-        uint4 w[kUnroll][2];
+    for (int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b0 < n_blocks;
+         b0 += kUnroll * stride) {
+        Blk<T, 32> blk[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            if (b0 + u * stride < n_blocks)
+                load_blk(x, b0 + u * stride, blk[u]);
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int64_t unit = base + u * 32 + lane;
-            load_unit<T>(xv, unit, unit < n_units, w[u]);
-        }
+            const int64_t b = b0 + u * stride;
+            if (b < n_blocks) {
+                const uint32_t ab = absmax_bits(blk[u]);
+                bad |= ab >= kNonFiniteBits;
+                const uint32_t byte = e8m0_byte_floor(ab);
+                const float inv = e8m0_inverse(byte);
+                uint32_t pk[4];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t unit = base + u * 32 + lane;
-            float xf[8];
-            uint32_t ab = unit_to_f32<T>(w[u], xf);
-            ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, 1));
-            ab = max(ab, __shfl_xor_sync(0xFFFFFFFFu, ab, 2));
-            bad |= ab >= kNonFiniteBits;
-            const uint32_t byte = e8m0_byte_floor(ab);
-            const float inv = e8m0_inverse(byte);
-            float v[8];
+                for (int j = 0; j < 4; ++j) {
+                    float v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                v[i] = __fmul_rn(xf[i], inv); // exact: multiplication by 2^-e
-            const uint32_t pk = e2m1x8(v);
-            if (unit < n_units) {
-                packed[unit] = pk;
-                if (!(lane & 3))
-                    scales[unit >> 2] = (uint8_t)byte;
+                    for (int i = 0; i < 8; ++i)
+                        v[i] = __fmul_rn(elem(blk[u], 8 * j + i), inv); // exact: 2^-e
+                    pk[j] = e2m1x8(v);
+                }
+                packed[b] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                scales[b] = (uint8_t)byte;
             }
         }
     }
-    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0)
+    if (bad)
         raise_status(status, kStatusNonFinite);
 }
 
 // ---------------------------------------------------------------------------
-// Dequantise.  Unit = eight codes (one 4-byte word) -> eight outputs.
+// Dequantise.  One thread per 16 codes (8 packed bytes) -> 16 outputs (one
+// 32-byte bf16 store or two fp32 ones).
 // ---------------------------------------------------------------------------
 template <bool kNv, typename TOut>
 __global__ void __launch_bounds__(kThreads)
-    dequantize_kernel(const uint32_t *__restrict__ packed, const uint8_t *__restrict__ scales,
+    dequantize_kernel(const uint2 *__restrict__ packed, const uint8_t *__restrict__ scales,
                       const float *__restrict__ global_scale, int64_t n_units,
                       TOut *__restrict__ y)
 {
-    constexpr int kUnroll = 4;
-    const float g = kNv ? *global_scale : 1.0f;
+    pdl_begin();
+    constexpr int kUnroll = 2;
+    const float g = kNv ? __ldcg(global_scale) : 1.0f;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (; i < n_units; i += kUnroll * stride) {
-        uint32_t pk[kUnroll];
+    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n_units;
+         i0 += kUnroll * stride) {
+        uint2 pk[kUnroll];
         uint32_t sbyte[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int64_t unit = i + u * stride;
+            const int64_t unit = i0 + u * stride;
             if (unit < n_units) {
-                pk[u] = __ldg(packed + unit);
-                sbyte[u] = __ldg(scales + (kNv ? (unit >> 1) : (unit >> 2)));
-            } else {
-                pk[u] = 0u;
-                sbyte[u] = 0u;
+                pk[u] = __ldcg(packed + unit);
+                sbyte[u] = __ldcg(scales + (kNv ? unit : (unit >> 1)));
             }
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int64_t unit = i + u * stride;
-            float p[8], yv[8];
-            e2m1x8_decode(pk[u], p);
-            if (kNv) {
-                const float sb = e4m3_to_f32(sbyte[u]);
+            const int64_t unit = i0 + u * stride;
+            if (unit >= n_units)
+                continue;
+            const float s = kNv ? e4m3_to_f32(sbyte[u]) : e8m0_to_f32(sbyte[u]);
+            float y16[16];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float p[8];
+                e2m1x8_decode(h ? pk[u].y : pk[u].x, p);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    yv[k] = nv_dequant(p[k], sb, g);
-            } else {
-                const float s = e8m0_to_f32(sbyte[u]);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    yv[k] = __fmul_rn(p[k], s); // exact
+                    y16[8 * h + k] = kNv ? nv_dequant(p[k], s, g) : __fmul_rn(p[k], s);
             }
-            if (unit < n_units) {
-                if constexpr (sizeof(TOut) == 2) {
-                    stg_stream(reinterpret_cast<uint4 *>(y) + unit, f32x8_to_bf16x8(yv));
-                } else {
-                    uint4 *yo = reinterpret_cast<uint4 *>(y) + 2 * unit;
-                    stg_stream(yo, make_uint4(__float_as_uint(yv[0]), __float_as_uint(yv[1]),
-                                              __float_as_uint(yv[2]), __float_as_uint(yv[3])));
-                    stg_stream(yo + 1, make_uint4(__float_as_uint(yv[4]), __float_as_uint(yv[5]),
-                                                  __float_as_uint(yv[6]), __float_as_uint(yv[7])));
+            if constexpr (sizeof(TOut) == 2) {
+                uint32_t o[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(y16[2 * j + 1]), "f"(y16[2 * j]));
+                stg_v8(reinterpret_cast<char *>(y) + unit * 32, o);
+            } else {
+                uint32_t o[8];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        o[j] = __float_as_uint(y16[8 * h + j]);
+                    stg_v8(reinterpret_cast<char *>(y) + unit * 64 + 32 * h, o);
                 }
             }
         }
@@ -375,141 +445,141 @@ __global__ void __launch_bounds__(kThreads)
 // ---------------------------------------------------------------------------
 // Scale search.  One thread owns one 16-element block, kept in registers.
 //
-// Candidate codes: c_k = E4M3(m_k A_b / (6g)), m_k = (147 + k)/210.  The
-// raw candidates grow by a factor of at most 148/147 from one k to the next
+// Candidate set: c_k = E4M3(m_k A_b / (6g)), m_k = (147 + k)/210.  The raw
+// candidates grow by a factor of at most 148/147 from one k to the next
 // while every E4M3 rounding interval spans a factor above 1 + 1/16, so the
-// 64 candidates hit exactly the codes c_0 .. c_63, all of them: only two
-// roundings per block are needed (c_63 is the max-based NVFP4 scale).
+// 64 candidates hit exactly the codes c_0 .. c_63, all of them: two
+// roundings per block (c_63 is the max-based NVFP4 scale).
 //
-// Losses: each candidate's loss is first accumulated in fp32 on the block
-// scaled by a power of two (2^(127-f), f the exponent field of A_b, which
-// changes no comparison); its error is below 2e-6 relative plus 2^-140.
-// A comparison the fp32 sums cannot settle with that margin is redone on
-// the double loss the definition uses (same operations, same order), so
-// the winner equals the winner of the exact-in-double search.  Candidates
-// run in increasing scale order and a tie goes to the later one, i.e. to
-// the larger scale.
+// Order and pruning: codes run from c_63 down.  For a scale whose largest
+// reconstruction T7 = fl32(fl32(6 s_b) g) is below A_b, the block maximum
+// alone contributes (A_b - T7)^2 to the loss, a lower bound that only grows
+// as the scale shrinks; once it exceeds the best loss so far no smaller
+// candidate can win or tie, and the loop stops (about 2.3 of 5 candidates
+// evaluated on Laplace data).
+//
+// Screening loss: the block scaled by k = 2^(127 - f) (f the exponent field
+// of A_b: A_b k in [1, 2), changing no comparison) with the reconstruction
+// x_hat k = fl32(fl32(p s_b) g k) (exact while g >= 2^-116) and codes from
+// one reciprocal product per element (misrounded only within a few ulps of
+// an E2M1 midpoint, where the two neighbouring reconstructions are
+// equidistant from x: their squared errors differ by at most 1.2e-5 of
+// that element's term), summed in fp32 (error < 1e-6).  A comparison the
+// screening sums cannot settle with a 5e-5 relative margin is redone on the
+// exact double loss of the definition -- exact codes, x_hat as dequantised,
+// sum_i ((double)x_i - (double)x_hat_i)^2 in element order -- so the winner
+// is the winner of the exact-in-double search, and on equal loss the larger
+// scale (the one met first) stays.
 // ---------------------------------------------------------------------------
-struct BlockX {
-    float x[16];
-};
-
-// Codes of the block at scale code c (zero scale -> zero codes).
-__device__ __forceinline__ uint2 block_codes(const BlockX &b, uint32_t c, float g)
+template <typename T>
+__device__ __forceinline__ double exact_block_loss(const Blk<T, 16> &b, const uint2 &pk,
+                                                   uint32_t c, float g)
 {
-    if (c == 0u)
-        return make_uint2(0u, 0u);
-    const NvRecip q = nv_recip(__fmul_rn(e4m3_to_f32(c), g));
-    float lo[8], hi[8];
+    const float sb = e4m3_pos_to_f32(c);
+    double acc = 0.0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        lo[i] = b.x[i];
-        hi[i] = b.x[8 + i];
-    }
-    return make_uint2(nv_encode8(lo, q), nv_encode8(hi, q));
-}
-
-__device__ __forceinline__ void block_recon(const uint2 &pk, uint32_t c, float g, float (&xh)[16])
-{
-    const float sb = e4m3_to_f32(c);
-    float p[8];
-    e2m1x8_decode(pk.x, p);
+    for (int h = 0; h < 2; ++h) {
+        float p[8];
+        e2m1x8_decode(h ? pk.y : pk.x, p);
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-        xh[i] = nv_dequant(p[i], sb, g);
-    e2m1x8_decode(pk.y, p);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        xh[8 + i] = nv_dequant(p[i], sb, g);
-}
-
-// Scaled fp32 loss of codes pk at scale code c.
-__device__ __forceinline__ float block_loss32(const BlockX &b, const uint2 &pk, uint32_t c,
-                                             float g, float k)
-{
-    float xh[16];
-    block_recon(pk, c, g, xh);
-    float acc = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float ds = __fmul_rn(__fsub_rn(b.x[i], xh[i]), k);
-        acc = fmaf(ds, ds, acc);
+        for (int i = 0; i < 8; ++i) {
+            const double dd = __dsub_rn((double)elem(b, 8 * h + i), (double)nv_dequant(p[i], sb, g));
+            acc = __dadd_rn(acc, __dmul_rn(dd, dd));
+        }
     }
     return acc;
 }
 
-// The definition's loss: sum_i ((double)x_i - (double)x_hat_i)^2 in double,
-// summed in element order.
-__device__ __forceinline__ double block_loss64(const BlockX &b, const uint2 &pk, uint32_t c,
-                                               float g)
+// Screening loss of scale code c on the scaled block xk.
+__device__ __forceinline__ float screen_loss(const float (&xk)[16], uint32_t c, float g, float k,
+                                             float gk)
 {
-    float xh[16];
-    block_recon(pk, c, g, xh);
-    double acc = 0.0;
+    float acc = 0.0f;
+    if (c == 0u) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const double dd = __dsub_rn((double)b.x[i], (double)xh[i]);
-        acc = __dadd_rn(acc, __dmul_rn(dd, dd));
+        for (int i = 0; i < 16; ++i)
+            acc = fmaf(xk[i], xk[i], acc);
+        return acc;
+    }
+    const float sb = e4m3_pos_to_f32(c);
+    const float dk = __fmul_rn(__fmul_rn(sb, g), k);
+    const float r0 = rcp_approx(dk);
+    const float r = fmaf(r0, fmaf(-dk, r0, 1.0f), r0);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float v[8], p[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            v[i] = __fmul_rn(xk[8 * h + i], r);
+        e2m1x8_qdq(v, p);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float d = __fsub_rn(xk[8 * h + i], __fmul_rn(__fmul_rn(p[i], sb), gk));
+            acc = fmaf(d, d, acc);
+        }
     }
     return acc;
 }
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-    scale_search_kernel(const T *__restrict__ x, int64_t n_blocks,
-                        const uint32_t *__restrict__ partials, int nparts,
+    scale_search_kernel(const T *__restrict__ x, int64_t n_blocks, const float *amax,
                         uint2 *__restrict__ packed, uint8_t *__restrict__ scales,
                         float *global_scale, float *__restrict__ block_loss, int32_t *status)
 {
+    pdl_begin();
     float g;
-    if (!nv_prologue(partials, nparts, global_scale, status, g))
+    if (!nv_prologue(amax, global_scale, status, g))
         return;
-    const double g1260 = 1260.0 * (double)g; // exact: 9 + 24 significant bits
-    const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+    const NvScaleConsts sc = nv_scale_consts(g);
+    const double g1260 = 1260.0 * (double)g;      // exact: 9 + 24 significant bits
+    const float inv_lo = (float)(147.0 / g1260);  // RN32(0.7 / (6g))
+    const bool exact_always = !(g >= 0x1p-116f);
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < n_blocks;
          blk += stride) {
-        BlockX b;
-        uint32_t ab;
-        {
-            uint4 w[2][2];
-            load_unit<T>(xv, 2 * blk, true, w[0]);
-            load_unit<T>(xv, 2 * blk + 1, true, w[1]);
-            float h0[8], h1[8];
-            ab = max(unit_to_f32<T>(w[0], h0), unit_to_f32<T>(w[1], h1));
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                b.x[i] = h0[i];
-                b.x[8 + i] = h1[i];
-            }
-        }
-        const double amax_b = (double)__uint_as_float(ab);
-        const uint32_t c_lo = e4m3_code_from_f64(__ddiv_rn(147.0 * amax_b, g1260));
-        const uint32_t c_hi = e4m3_code_from_f64(__ddiv_rn(210.0 * amax_b, g1260));
+        Blk<T, 16> b;
+        load_blk(x, blk, b);
+        const uint32_t ab = absmax_bits_finite(b);
+        const float amax_b = __uint_as_float(ab);
+        const uint32_t c_hi = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
+        const uint32_t c_lo = nv_scale_code(amax_b, inv_lo, 147.0, g1260);
         const float k = __uint_as_float((254u - min(ab >> 23, 253u)) << 23);
+        const float gk = __fmul_rn(g, k);
+        const float ak = __fmul_rn(amax_b, k);
+        float xk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            xk[i] = __fmul_rn(elem(b, i), k);
 
-        uint32_t best_c = c_lo;
-        uint2 best_pk = block_codes(b, c_lo, g);
-        float best_l = block_loss32(b, best_pk, c_lo, g, k);
-        for (uint32_t c = c_lo + 1; c <= c_hi; ++c) {
-            const uint2 pk = block_codes(b, c, g);
-            const float l = block_loss32(b, pk, c, g, k);
-            const float hi = fmaxf(l, best_l), lo = fminf(l, best_l);
+        uint32_t best_c = c_hi;
+        float best = screen_loss(xk, c_hi, g, k, gk);
+        for (uint32_t c = c_hi; c > c_lo;) {
+            --c;
+            const float t7 = __fmul_rn(__fmul_rn(6.0f, e4m3_pos_to_f32(c)), gk);
+            if (ak > t7) {
+                const float e = __fsub_rn(ak, t7);
+                if (__fmul_rn(e, e) > fmaf(best, 6e-5f, best) + 0x1p-130f)
+                    break;
+            }
+            const float l = screen_loss(xk, c, g, k, gk);
+            const float hi = fmaxf(l, best), lo = fminf(l, best);
             bool take;
-            if (hi - lo > 8e-6f * hi + 0x1p-140f)
-                take = l < best_l;
+            if (!exact_always && __fsub_rn(hi, lo) > fmaf(hi, 5e-5f, 0x1p-130f))
+                take = l < best;
             else
-                take = block_loss64(b, pk, c, g) <= block_loss64(b, best_pk, best_c, g);
+                take = exact_block_loss(b, nv_block_codes(b, c, g), c, g) <
+                       exact_block_loss(b, nv_block_codes(b, best_c, g), best_c, g);
             if (take) {
                 best_c = c;
-                best_pk = pk;
-                best_l = l;
+                best = l;
             }
         }
-        packed[blk] = best_pk;
+        const uint2 pk = nv_block_codes(b, best_c, g);
+        packed[blk] = pk;
         scales[blk] = (uint8_t)best_c;
         if (block_loss)
-            block_loss[blk] = (float)block_loss64(b, best_pk, best_c, g);
+            block_loss[blk] = (float)exact_block_loss(b, pk, best_c, g);
     }
 }
 
@@ -519,6 +589,7 @@ __global__ void __launch_bounds__(kThreads)
 __global__ void e2m1_round_kernel(const float *__restrict__ v, uint8_t *__restrict__ codes,
                                   int64_t n)
 {
+    pdl_begin();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u * 8 < n; u += stride) {
         float a[8];
@@ -533,9 +604,33 @@ __global__ void e2m1_round_kernel(const float *__restrict__ v, uint8_t *__restri
     }
 }
 
+// decode(encode(v)) with the codes passed from one helper to the other in
+// registers, as the kernels do.
+__global__ void e2m1_roundtrip_kernel(const float *__restrict__ v, float *__restrict__ out,
+                                      int64_t n)
+{
+    pdl_begin();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u * 8 < n; u += stride) {
+        float a[8], p[8], q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            a[i] = (u * 8 + i < n) ? v[u * 8 + i] : 0.0f;
+        e2m1x8_decode(e2m1x8(a), p);
+        e2m1x8_qdq(a, q);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (u * 8 + i < n) {
+                out[2 * (u * 8 + i)] = p[i];
+                out[2 * (u * 8 + i) + 1] = q[i];
+            }
+    }
+}
+
 __global__ void nv_encode_quotient_kernel(const float *__restrict__ x, const float *__restrict__ d,
                                           uint8_t *__restrict__ codes, int64_t n)
 {
+    pdl_begin();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
         float a[8] = {x[i], 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};

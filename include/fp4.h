@@ -15,8 +15,9 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- * Pointers.  Every pointer is a DEVICE pointer owned by the caller.  x,
- * packed and y must be 16-byte aligned (else FP4_ERR_ALIGN); scales,
+ * Pointers.  Every pointer is a DEVICE pointer owned by the caller.  x and
+ * y must be 32-byte aligned and packed 16-byte aligned (else FP4_ERR_ALIGN:
+ * the kernels move whole blocks with 256-bit vector loads and stores); scales,
  * global_scale, block_loss, status and workspace need only the alignment of
  * their element type (workspace: 4 bytes).  The library never
  * allocates, frees or synchronises; all work is queued on `stream`
@@ -66,7 +67,7 @@ typedef enum fp4_status {
     FP4_OK = 0,
     FP4_ERR_INVALID_ARG = 1, /* NULL pointer, unknown enum, negative size */
     FP4_ERR_SHAPE = 2,       /* cols not a multiple of the block size; overflow */
-    FP4_ERR_ALIGN = 3,       /* a tensor pointer is not 16-byte aligned */
+    FP4_ERR_ALIGN = 3,       /* x / y not 32-byte or packed not 16-byte aligned */
     FP4_ERR_NONFINITE = 4,   /* (device status) NaN or Inf in the input */
     FP4_ERR_RANGE = 5,       /* (device status) NVFP4 global scale out of range */
     FP4_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than required */
@@ -83,17 +84,18 @@ const char *fp4_status_string(int status);
 int fp4_version(void);
 
 /* Bytes of device workspace the NVFP4 quantiser, the scale search and the
- * tensor amax need for a [rows, cols] input: per-CTA partial maxima of the
- * first pass.  Any caller-owned device buffer of at least this size, 4-byte
- * aligned, works; it need not be initialised and its contents are scratch. */
+ * tensor amax need for a [rows, cols] input: per-CTA partial maxima, a CTA
+ * counter and the amax word.  Any caller-owned device buffer of at least
+ * this size, 4-byte aligned, works.  It must be zero-filled once before its
+ * first use (e.g. cudaMemset after allocation); every call leaves the counter
+ * at zero again, and the rest of the buffer is scratch. */
 size_t fp4_workspace_bytes(fp4_format fmt, int64_t rows, int64_t cols);
 
 /* Tensor amax A = max |x| over n elements ("NVFP4 与 MXFP4 格式" section 3,
  * A is the tensor absolute maximum; section 4 reference program, first
  * step).  Writes A as one fp32 to device `amax`.  A NaN or Inf in x sets
  * FP4_ERR_NONFINITE in *status (and *amax then holds a non-finite value).
- * Two launches: per-CTA partial maxima into `workspace`, then a one-CTA
- * reduction. */
+ * One launch: per-CTA maxima into `workspace`, folded by the last CTA. */
 fp4_status fp4_tensor_amax(const void *x, fp4_dtype dtype, int64_t n, float *amax,
                            void *workspace, size_t workspace_bytes, int32_t *status,
                            cudaStream_t stream);
@@ -109,7 +111,11 @@ fp4_status fp4_tensor_amax(const void *x, fp4_dtype dtype, int64_t n, float *ama
  * Outputs packed [rows, cols/2], scales [rows, cols/16] (E4M3 codes) and
  * *global_scale = g.  Two kernels: tensor amax into the workspace, then the
  * fused block-amax / scale / divide / round / pack pass.  Data errors:
- * NONFINITE, RANGE. */
+ * NONFINITE, RANGE.
+ *
+ * Every kernel of the library is launched with programmatic stream
+ * serialisation: it may start while the previous kernel on the stream is
+ * finishing and waits for it before touching memory. */
 fp4_status fp4_nvfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
                               uint8_t *packed, uint8_t *scales, float *global_scale,
                               void *workspace, size_t workspace_bytes, int32_t *status,
@@ -178,6 +184,12 @@ fp4_status fp4_scale_search_with_amax(const void *x, fp4_dtype dtype, int64_t ro
  * Inf in v gives an unspecified code.  codes is uint8 [n] (one code per
  * byte, unpacked). */
 fp4_status fp4_e2m1_round(const float *v, uint8_t *codes, int64_t n, cudaStream_t stream);
+
+/* E2M1 round trip alone, for tests: out[2i] = value of the code of v[i]
+ * decoded from the packed codes the encoder returns in registers, and
+ * out[2i+1] = the same value from the fused quantise-dequantise routine the
+ * scale search uses.  out is fp32 [2n]. */
+fp4_status fp4_e2m1_roundtrip(const float *v, float *out, int64_t n, cudaStream_t stream);
 
 /* NVFP4 element quotient + encoder alone, for tests: codes[i] = E2M1 code
  * of fl32(x[i] / d[i]) computed by the same device routine the NVFP4

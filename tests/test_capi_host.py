@@ -43,7 +43,7 @@ def test_status_strings_and_version(L):
 
 P = 1 << 20          # a fake, 16-byte aligned "device" address (never dereferenced)
 Q = P + 4            # misaligned
-WS = 4096
+WS = 1 << 16
 
 
 def test_argument_errors_return_before_any_launch(L):

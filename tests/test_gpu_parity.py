@@ -164,6 +164,22 @@ def test_e2m1_round_every_finite_fp32_outside_the_decisive_range():
         del bits, v, c, mag, neg, small, big
 
 
+def test_e2m1_register_roundtrip():
+    """Codes handed from the encoder to the decoder in registers (the
+    kernels' own chain), and the fused quantise-dequantise of the search,
+    both give the oracle's decode(encode(v)) for every bf16 pattern and a
+    dense fp32 sweep."""
+    b = torch.arange(1 << 16, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float()
+    v = torch.cat([b[torch.isfinite(b)], torch.linspace(-8, 8, 1 << 20)]).contiguous()
+    out = fp4.e2m1_roundtrip(v.to(DEV)).cpu().numpy()
+    codes = oracle.e2m1_encode_f32(v.numpy())
+    mag = np.array([oracle.e2m1_decode(c) for c in range(16)], np.float32)
+    want = mag[codes]
+    ok_chain = np.array_equal(out[:, 0].view(np.uint32), want.view(np.uint32))
+    ok_fused = np.array_equal(out[:, 1].view(np.uint32), want.view(np.uint32))
+    assert ok_chain and ok_fused, f"decode(encode) in registers: {ok_chain}, fused quantise-dequantise: {ok_fused}"
+
+
 def test_nv_quotient_bracket_matches_ieee_division():
     """codes of fl32(x / d) for random pairs and for pairs placed exactly
     on, and a few ulps either side of, every E2M1 midpoint."""

@@ -76,6 +76,14 @@ def with_shape(w: Workload, rows: int, cols: int, seed_offset: int = 0) -> Workl
                                name=f"{w.name}@{rows}x{cols}" + (f"+{seed_offset}" if seed_offset else ""))
 
 
+def for_rank(w: Workload, rank: int) -> Workload:
+    """The tensor rank `rank` works on when N ranks each take their own
+    tensor of the workload (independent problems, no data exchange): same
+    shape and distribution, seed offset by 1000 per rank (rank 0 keeps the
+    workload's own seed)."""
+    return w if rank == 0 else with_shape(w, w.rows, w.cols, seed_offset=1000 * rank)
+
+
 def generate(w: Workload, device: str | torch.device = "cpu") -> torch.Tensor:
     """The workload's tensor, [rows, cols] in its dtype, drawn from a
     torch.Generator seeded with w.seed on `device`."""
