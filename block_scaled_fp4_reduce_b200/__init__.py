@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
             "fp4_tensor_amax": (I, [P, I, I64, P, P, SZ, P, P]),
             "fp4_nvfp4_quantize": (I, [P, I, I64, I64, P, P, P, P, SZ, P, P]),
             "fp4_nvfp4_quantize_with_amax": (I, [P, I, I64, I64, P, P, P, P, P, P]),
+            "fp4_nvfp4_quantize_noalloc": (I, [P, I, I64, I64, P, P, P, P, P]),
             "fp4_mxfp4_quantize": (I, [P, I, I64, I64, P, P, P, P]),
             "fp4_dequantize": (I, [I, P, P, P, I64, I64, P, I, P]),
             "fp4_scale_search": (I, [P, I, I64, I64, P, P, P, P, P, SZ, P, P]),
@@ -127,6 +128,12 @@ def fp4_nvfp4_quantize_with_amax(x, amax, packed, scales, global_scale, status, 
     R, C = _shape2(x)
     return lib().fp4_nvfp4_quantize_with_amax(_p(x), _dtype_code(x), R, C, _p(amax), _p(packed), _p(scales),
                                               _p(global_scale), _p(status), _stream(stream))
+
+
+def fp4_nvfp4_quantize_noalloc(x, packed, scales, global_scale, status, stream=None) -> int:
+    R, C = _shape2(x)
+    return lib().fp4_nvfp4_quantize_noalloc(_p(x), _dtype_code(x), R, C, _p(packed), _p(scales),
+                                            _p(global_scale), _p(status), _stream(stream))
 
 
 def fp4_mxfp4_quantize(x, packed, scales, status, stream=None) -> int:

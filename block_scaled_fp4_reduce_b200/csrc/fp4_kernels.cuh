@@ -584,9 +584,10 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Test-only element kernels.
+// Test-only element kernels (internal linkage: this header is included by
+// more than one translation unit).
 // ---------------------------------------------------------------------------
-__global__ void e2m1_round_kernel(const float *__restrict__ v, uint8_t *__restrict__ codes,
+static __global__ void e2m1_round_kernel(const float *__restrict__ v, uint8_t *__restrict__ codes,
                                   int64_t n)
 {
     pdl_begin();
@@ -606,7 +607,7 @@ __global__ void e2m1_round_kernel(const float *__restrict__ v, uint8_t *__restri
 
 // decode(encode(v)) with the codes passed from one helper to the other in
 // registers, as the kernels do.
-__global__ void e2m1_roundtrip_kernel(const float *__restrict__ v, float *__restrict__ out,
+static __global__ void e2m1_roundtrip_kernel(const float *__restrict__ v, float *__restrict__ out,
                                       int64_t n)
 {
     pdl_begin();
@@ -627,7 +628,7 @@ __global__ void e2m1_roundtrip_kernel(const float *__restrict__ v, float *__rest
     }
 }
 
-__global__ void nv_encode_quotient_kernel(const float *__restrict__ x, const float *__restrict__ d,
+static __global__ void nv_encode_quotient_kernel(const float *__restrict__ x, const float *__restrict__ d,
                                           uint8_t *__restrict__ codes, int64_t n)
 {
     pdl_begin();

@@ -179,6 +179,24 @@ fp4_status fp4_scale_search_with_amax(const void *x, fp4_dtype dtype, int64_t ro
                                       uint8_t *scales, float *global_scale, float *block_loss,
                                       int32_t *status, cudaStream_t stream);
 
+/* NVFP4 quantise + pack without a caller workspace.  No counterpart in the
+ * pages: it exists for callers that cannot allocate device memory -- code
+ * running where cudaMalloc is off limits (an inference-engine plugin's
+ * execute callback, a serving loop that must not allocate once requests
+ * flow) or whose device memory was all reserved up front and handed out as
+ * tensors.  Same arguments, outputs, rules and errors as fp4_nvfp4_quantize
+ * minus the workspace, which lives instead in a 4128-byte __device__ array
+ * inside the library (held on every GPU that loads it until exit; enough
+ * for every shape -- a shape needing more would get FP4_ERR_WORKSPACE).
+ * All calls on a device share that array: calls whose kernels overlap on
+ * the GPU race and must be ordered by the caller.  Each call clears the
+ * array's counter word on `stream` before its kernels.  The first call on a
+ * device looks up the array's address with that device current; make it
+ * before any stream capture. */
+fp4_status fp4_nvfp4_quantize_noalloc(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                      uint8_t *packed, uint8_t *scales, float *global_scale,
+                                      int32_t *status, cudaStream_t stream);
+
 /* Element encoder alone, for tests: codes[i] = E2M1 code of the fp32 value
  * v[i] (nearest, ties to even code, saturating, sign bit kept).  A NaN or
  * Inf in v gives an unspecified code.  codes is uint8 [n] (one code per
