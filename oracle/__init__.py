@@ -79,6 +79,9 @@ def lib() -> ctypes.CDLL:
             "oracle_nvfp4_dequantize": (None, [P, P, F, I64, I64, P]),
             "oracle_mx_block_exponent": (I, [F]),
             "oracle_mxfp4_quantize": (I, [P, I, I64, I64, P, P]),
+            "oracle_mx_block_exponent_ceil": (I, [F, P]),
+            "oracle_mxfp4_quantize_rule": (I, [P, I, I64, I64, I, P, P]),
+            "oracle_nvfp4_quantize_four_over_six": (I, [P, I, I64, I64, P, P, P, P]),
             "oracle_mxfp4_dequantize": (None, [P, P, I64, I64, P]),
             "oracle_nv_block_loss": (D, [P, I, F]),
             "oracle_search_candidate_code": (I, [F, F, I]),
@@ -256,6 +259,38 @@ def mxfp4_quantize(x: np.ndarray):
     scales = np.zeros((R, C // 32), np.uint8)
     _check(lib().oracle_mxfp4_quantize(_ptr(x), dt, R, C, _ptr(packed), _ptr(scales)))
     return packed, scales
+
+
+MX_FLOOR, MX_CEIL = 0, 1
+
+
+def mx_block_exponent_ceil(amax_b: float) -> int:
+    e = ctypes.c_int()
+    _check(lib().oracle_mx_block_exponent_ceil(float(amax_b), ctypes.byref(e)))
+    return e.value
+
+
+def mxfp4_quantize_rule(x: np.ndarray, rule: int):
+    """MXFP4 with scale rule MX_FLOOR (OCP) or MX_CEIL (the page's mx_scale)."""
+    x, dt = _input(x)
+    R, C = _shape(x)
+    packed = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 32), np.uint8)
+    _check(lib().oracle_mxfp4_quantize_rule(_ptr(x), dt, R, C, int(rule), _ptr(packed), _ptr(scales)))
+    return packed, scales
+
+
+def nvfp4_quantize_four_over_six(x: np.ndarray):
+    """Returns (packed, scales, g, block_loss float64)."""
+    x, dt = _input(x)
+    R, C = _shape(x)
+    packed = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    loss = np.zeros((R, C // 16), np.float64)
+    g = ctypes.c_float()
+    _check(lib().oracle_nvfp4_quantize_four_over_six(_ptr(x), dt, R, C, _ptr(packed), _ptr(scales),
+                                                     ctypes.byref(g), _ptr(loss)))
+    return packed, scales, g.value, loss
 
 
 def nvfp4_dequantize(packed: np.ndarray, scales: np.ndarray, g: float, rows: int, cols: int) -> np.ndarray:

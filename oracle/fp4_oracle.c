@@ -19,6 +19,8 @@
  *   [MATH]  "FP4 / NVFP4 数学总结" (devpress.csdn.net): S3 NVFP4 formula,
  *           S7-S8 max/6 scale worked example, S9 Loss(s), S10 quantise /
  *           dequantise formulas.
+ *   [TJ]    "FP4、FP8 与 INT8/INT4：数值范围、块缩放与推理计算精度"
+ *           (tom-jerr.github.io): S4 "Scale 怎么选" (four over six).
  *
  * Arithmetic: double for every step the pages write as real arithmetic;
  * IEEE single (C `float`, FLT_EVAL_METHOD == 0, no contraction) for the
@@ -380,6 +382,72 @@ int oracle_mx_block_exponent(float amax_b)
     return e;
 }
 
+/* Shared exponent of a 32-block under the ceil rule of the page's
+ * `mx_scale` helper ([NVMX] S5-S6: the ModelOpt-style 2^ceil(log2(A_b/6))):
+ * an all-zero block gets scale 1 (e = 0); otherwise e = max(-127, E - 3)
+ * with frexp(A_b) = m 2^E, then e + 1 if A_b > 6 * 2^e (the threshold
+ * compare avoids rounding log2 near integers); e > 127 is rejected. */
+int oracle_mx_block_exponent_ceil(float amax_b, int *e_out)
+{
+    if (amax_b == 0.0f) {
+        *e_out = 0;
+        return ORACLE_OK;
+    }
+    int E;
+    frexp((double)amax_b, &E);
+    int e = E - 3;
+    if (e < -127)
+        e = -127;
+    if ((double)amax_b > 6.0 * ldexp(1.0, e))
+        e += 1;
+    if (e > 127)
+        return ORACLE_ERR_RANGE;
+    *e_out = e;
+    return ORACLE_OK;
+}
+
+/* MXFP4 with the scale rule chosen: rule 0 = OCP rounding-down (floor),
+ * rule 1 = the ceil rule above. */
+int oracle_mxfp4_quantize_rule(const void *x, int dtype, int64_t rows, int64_t cols, int rule,
+                               uint8_t *packed, uint8_t *scales)
+{
+    if (cols % 32 || rows < 0 || cols < 0)
+        return ORACLE_ERR_SHAPE;
+    if (rule != 0 && rule != 1)
+        return ORACLE_ERR_ARG;
+    int64_t n = rows * cols;
+    for (int64_t i = 0; i < n; ++i)
+        if (!isfinite(load_elem(x, dtype, i)))
+            return ORACLE_ERR_NONFINITE;
+    int64_t nblocks = n / 32;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        float ab = 0.0f;
+        for (int i = 0; i < 32; ++i) {
+            float m = fabsf(load_elem(x, dtype, b * 32 + i));
+            if (m > ab)
+                ab = m;
+        }
+        int e;
+        if (rule == 0) {
+            e = oracle_mx_block_exponent(ab);
+        } else {
+            int st = oracle_mx_block_exponent_ceil(ab, &e);
+            if (st)
+                return st;
+        }
+        double scale = ldexp(1.0, e);
+        uint8_t codes[32];
+        for (int i = 0; i < 32; ++i) {
+            int c = 0;
+            oracle_e2m1_encode((double)load_elem(x, dtype, b * 32 + i) / scale, &c);
+            codes[i] = (uint8_t)c;
+        }
+        scales[b] = (uint8_t)(e + 127);
+        oracle_pack4(codes, 32, packed + b * 16);
+    }
+    return ORACLE_OK;
+}
+
 int oracle_mxfp4_quantize(const void *x, int dtype, int64_t rows, int64_t cols,
                           uint8_t *packed, uint8_t *scales)
 {
@@ -512,6 +580,50 @@ int oracle_nvfp4_scale_search(const void *x, int dtype, int64_t rows, int64_t co
         return st;
     *g_out = g;
     return oracle_nvfp4_scale_search_with_g(x, dtype, rows, cols, g, packed, scales, block_loss);
+}
+
+/* NVFP4 "four over six" ([TJ] S4: mapping the block maximum to 4 instead
+ * of 6 can place the other values on better grid points; neither rule wins
+ * on every block).  Per 16-block the two candidate scales are the E4M3
+ * codes nearest to A_b / (6g) (the max-based scale) and A_b / (4g); the
+ * second is taken only when its artefact loss is strictly smaller.  g as
+ * for NVFP4.  Emits codes, scale codes, g and the chosen loss. */
+int oracle_nvfp4_quantize_four_over_six(const void *x, int dtype, int64_t rows, int64_t cols,
+                                        uint8_t *packed, uint8_t *scales, float *g_out,
+                                        double *block_loss)
+{
+    if (cols % 16 || rows < 0 || cols < 0)
+        return ORACLE_ERR_SHAPE;
+    float amax, g;
+    int st = oracle_tensor_amax(x, dtype, rows * cols, &amax);
+    if (st)
+        return st;
+    st = oracle_nv_global_scale(amax, &g);
+    if (st)
+        return st;
+    *g_out = g;
+    int64_t nblocks = rows * cols / 16;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        float xb[16];
+        float ab = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+            xb[i] = load_elem(x, dtype, b * 16 + i);
+            if (fabsf(xb[i]) > ab)
+                ab = fabsf(xb[i]);
+        }
+        int c6 = oracle_e4m3_encode((double)ab / (6.0 * (double)g));
+        int c4 = oracle_e4m3_encode((double)ab / (4.0 * (double)g));
+        double l6 = oracle_nv_block_loss(xb, c6, g);
+        double l4 = oracle_nv_block_loss(xb, c4, g);
+        int best = l4 < l6 ? c4 : c6;
+        uint8_t codes[16];
+        nv_block_codes(xb, 16, best, g, codes);
+        scales[b] = (uint8_t)best;
+        oracle_pack4(codes, 16, packed + b * 8);
+        if (block_loss)
+            block_loss[b] = l4 < l6 ? l4 : l6;
+    }
+    return ORACLE_OK;
 }
 
 /* Per-block loss of given (packed, scale) artefacts against x, for
