@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
             "fp4_nvfp4_quantize_with_amax": (I, [P, I, I64, I64, P, P, P, P, P, P]),
             "fp4_nvfp4_quantize_noalloc": (I, [P, I, I64, I64, P, P, P, P, P]),
             "fp4_mxfp4_quantize": (I, [P, I, I64, I64, P, P, P, P]),
+            "fp4_mxfp4_quantize_ceil": (I, [P, I, I64, I64, P, P, P, P]),
+            "fp4_nvfp4_quantize_four_over_six": (I, [P, I, I64, I64, P, P, P, P, P, SZ, P, P]),
             "fp4_dequantize": (I, [I, P, P, P, I64, I64, P, I, P]),
             "fp4_scale_search": (I, [P, I, I64, I64, P, P, P, P, P, SZ, P, P]),
             "fp4_scale_search_with_amax": (I, [P, I, I64, I64, P, P, P, P, P, P, P]),
@@ -142,6 +144,21 @@ def fp4_mxfp4_quantize(x, packed, scales, status, stream=None) -> int:
                                     _stream(stream))
 
 
+def fp4_mxfp4_quantize_ceil(x, packed, scales, status, stream=None) -> int:
+    R, C = _shape2(x)
+    return lib().fp4_mxfp4_quantize_ceil(_p(x), _dtype_code(x), R, C, _p(packed), _p(scales), _p(status),
+                                         _stream(stream))
+
+
+def fp4_nvfp4_quantize_four_over_six(x, packed, scales, global_scale, block_loss, workspace, status,
+                                     stream=None) -> int:
+    R, C = _shape2(x)
+    return lib().fp4_nvfp4_quantize_four_over_six(_p(x), _dtype_code(x), R, C, _p(packed), _p(scales),
+                                                  _p(global_scale), _p(block_loss), _p(workspace),
+                                                  workspace.numel() * workspace.element_size(),
+                                                  _p(status), _stream(stream))
+
+
 def fp4_dequantize(fmt, packed, scales, global_scale, rows, cols, y, stream=None) -> int:
     return lib().fp4_dequantize(fmt, _p(packed), _p(scales), _p(global_scale), rows, cols, _p(y),
                                 _dtype_code(y), _stream(stream))
@@ -224,6 +241,31 @@ def mxfp4_quantize(x: torch.Tensor, status=None, stream=None) -> Quantized:
     st = status if status is not None else new_status(dev)
     _check(fp4_mxfp4_quantize(x, packed, scales, st, stream), "fp4_mxfp4_quantize")
     return Quantized(MXFP4, packed, scales, None, st, R, C)
+
+
+def mxfp4_quantize_ceil(x: torch.Tensor, status=None, stream=None) -> Quantized:
+    R, C = _shape2(x)
+    dev = x.device
+    packed = torch.empty((R, C // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((R, C // 32), dtype=torch.uint8, device=dev)
+    st = status if status is not None else new_status(dev)
+    _check(fp4_mxfp4_quantize_ceil(x, packed, scales, st, stream), "fp4_mxfp4_quantize_ceil")
+    return Quantized(MXFP4, packed, scales, None, st, R, C)
+
+
+def nvfp4_quantize_four_over_six(x: torch.Tensor, with_loss: bool = True, workspace=None, status=None,
+                                 stream=None) -> Quantized:
+    R, C = _shape2(x)
+    dev = x.device
+    packed = torch.empty((R, C // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((R, C // 16), dtype=torch.uint8, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    loss = torch.empty((R, C // 16), dtype=torch.float32, device=dev) if with_loss else None
+    ws = workspace if workspace is not None else workspace_for(x)
+    st = status if status is not None else new_status(dev)
+    _check(fp4_nvfp4_quantize_four_over_six(x, packed, scales, g, loss, ws, st, stream),
+           "fp4_nvfp4_quantize_four_over_six")
+    return Quantized(NVFP4, packed, scales, g, st, R, C, block_loss=loss)
 
 
 def dequantize(q: Quantized, out_dtype=torch.bfloat16, out=None, stream=None) -> torch.Tensor:

@@ -156,6 +156,42 @@ fp4_status launch_nv_quantize(const void *x, fp4_dtype dt, int64_t n, const floa
 
 } // namespace
 
+namespace {
+template <bool kCeil>
+fp4_status mxfp4_quantize_rule(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                               uint8_t *packed, uint8_t *scales, int32_t *status,
+                               cudaStream_t stream)
+{
+    if (!status || !valid_dtype(dtype))
+        return FP4_ERR_INVALID_ARG;
+    fp4_status st = check_shape(rows, cols, 32);
+    if (st != FP4_OK)
+        return st;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4_OK;
+    if (!x || !packed || !scales)
+        return FP4_ERR_INVALID_ARG;
+    if (!aligned(x, 32) || !aligned(packed, 16))
+        return FP4_ERR_ALIGN;
+    const int64_t n_blocks = n / 32;
+    const int64_t per_cta = (int64_t)kThreads * 2;
+    uint4 *pk = reinterpret_cast<uint4 *>(packed);
+    if (dtype == FP4_BF16) {
+        const int grid = grid_for(fp4::mxfp4_quantize_kernel<uint16_t, kCeil>, n_blocks, per_cta);
+        if (grid <= 0)
+            return FP4_ERR_CUDA;
+        return launch(fp4::mxfp4_quantize_kernel<uint16_t, kCeil>, grid, stream,
+                      static_cast<const uint16_t *>(x), n_blocks, pk, scales, status);
+    }
+    const int grid = grid_for(fp4::mxfp4_quantize_kernel<float, kCeil>, n_blocks, per_cta);
+    if (grid <= 0)
+        return FP4_ERR_CUDA;
+    return launch(fp4::mxfp4_quantize_kernel<float, kCeil>, grid, stream,
+                  static_cast<const float *>(x), n_blocks, pk, scales, status);
+}
+} // namespace
+
 extern "C" {
 
 const char *fp4_status_string(int status)
@@ -245,34 +281,14 @@ fp4_status fp4_mxfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int6
                               uint8_t *packed, uint8_t *scales, int32_t *status,
                               cudaStream_t stream)
 {
-    if (!status || !valid_dtype(dtype))
-        return FP4_ERR_INVALID_ARG;
-    fp4_status st = check_shape(rows, cols, 32);
-    if (st != FP4_OK)
-        return st;
-    const int64_t n = rows * cols;
-    if (n == 0)
-        return FP4_OK;
-    if (!x || !packed || !scales)
-        return FP4_ERR_INVALID_ARG;
-    if (!aligned(x, 32) || !aligned(packed, 16))
-        return FP4_ERR_ALIGN;
-    const int64_t n_blocks = n / 32;
-    const int64_t per_cta = (int64_t)kThreads * 2;
-    uint4 *pk = reinterpret_cast<uint4 *>(packed);
-    if (dtype == FP4_BF16) {
-        const int grid = grid_for(fp4::mxfp4_quantize_kernel<uint16_t>, n_blocks, per_cta);
-        if (grid <= 0)
-            return FP4_ERR_CUDA;
-        return launch(fp4::mxfp4_quantize_kernel<uint16_t>, grid, stream,
-                      static_cast<const uint16_t *>(x), n_blocks, pk, scales, status);
-    } else {
-        const int grid = grid_for(fp4::mxfp4_quantize_kernel<float>, n_blocks, per_cta);
-        if (grid <= 0)
-            return FP4_ERR_CUDA;
-        return launch(fp4::mxfp4_quantize_kernel<float>, grid, stream,
-                      static_cast<const float *>(x), n_blocks, pk, scales, status);
-    }
+    return mxfp4_quantize_rule<false>(x, dtype, rows, cols, packed, scales, status, stream);
+}
+
+fp4_status fp4_mxfp4_quantize_ceil(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                   uint8_t *packed, uint8_t *scales, int32_t *status,
+                                   cudaStream_t stream)
+{
+    return mxfp4_quantize_rule<true>(x, dtype, rows, cols, packed, scales, status, stream);
 }
 
 fp4_status fp4_dequantize(fp4_format fmt, const uint8_t *packed, const uint8_t *scales,
@@ -383,6 +399,48 @@ fp4_status fp4_scale_search_with_amax(const void *x, fp4_dtype dtype, int64_t ro
         return FP4_ERR_ALIGN;
     return launch_search(x, dtype, n, amax, packed, scales, global_scale, block_loss, status,
                          stream);
+}
+
+fp4_status fp4_nvfp4_quantize_four_over_six(const void *x, fp4_dtype dtype, int64_t rows,
+                                            int64_t cols, uint8_t *packed, uint8_t *scales,
+                                            float *global_scale, float *block_loss,
+                                            void *workspace, size_t workspace_bytes,
+                                            int32_t *status, cudaStream_t stream)
+{
+    if (!global_scale || !status || !valid_dtype(dtype))
+        return FP4_ERR_INVALID_ARG;
+    fp4_status st = check_shape(rows, cols, 16);
+    if (st != FP4_OK)
+        return st;
+    const int64_t n = rows * cols;
+    if (n > 0 && (!x || !packed || !scales))
+        return FP4_ERR_INVALID_ARG;
+    if (!aligned(x, 32) || !aligned(packed, 16) || !aligned(block_loss, 4))
+        return FP4_ERR_ALIGN;
+    if (!workspace || workspace_bytes < fp4_workspace_bytes(FP4_NVFP4, rows, cols) ||
+        !aligned(workspace, 4))
+        return FP4_ERR_WORKSPACE;
+    uint32_t *ws = static_cast<uint32_t *>(workspace);
+    float *amax = reinterpret_cast<float *>(ws + kWsAmax);
+    st = launch_amax(x, dtype, n, ws, amax, status, stream);
+    if (st != FP4_OK)
+        return st;
+    const int64_t n_blocks = n / 16;
+    uint2 *pk = reinterpret_cast<uint2 *>(packed);
+    if (dtype == FP4_BF16) {
+        const int grid = grid_for(fp4::nvfp4_four_over_six_kernel<uint16_t>, n_blocks, kThreads);
+        if (grid <= 0)
+            return FP4_ERR_CUDA;
+        return launch(fp4::nvfp4_four_over_six_kernel<uint16_t>, grid, stream,
+                      static_cast<const uint16_t *>(x), n_blocks, static_cast<const float *>(amax),
+                      pk, scales, global_scale, block_loss, status);
+    }
+    const int grid = grid_for(fp4::nvfp4_four_over_six_kernel<float>, n_blocks, kThreads);
+    if (grid <= 0)
+        return FP4_ERR_CUDA;
+    return launch(fp4::nvfp4_four_over_six_kernel<float>, grid, stream,
+                  static_cast<const float *>(x), n_blocks, static_cast<const float *>(amax), pk,
+                  scales, global_scale, block_loss, status);
 }
 
 fp4_status fp4_e2m1_round(const float *v, uint8_t *codes, int64_t n, cudaStream_t stream)

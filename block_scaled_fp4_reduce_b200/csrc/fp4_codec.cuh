@@ -198,7 +198,26 @@ __device__ __forceinline__ uint32_t e8m0_byte_floor(uint32_t amax_bits)
     return (uint32_t)max(f - 2, 0);
 }
 
-// 2^-e as fp32 for the E8M0 byte b = e + 127 (b <= 252 from finite input):
+// E8M0 block scale, ceil rule (the NVFP4/MXFP4 format page's `mx_scale`,
+// ModelOpt-style 2^ceil(log2(A_b/6))): an all-zero block gets e = 0 (scale
+// 1); otherwise e = max(E - 3, -127) with A_b = m 2^E, m in [0.5, 1), then
+// e + 1 if A_b > 6 * 2^e, so that A_b never exceeds 6 * 2^e.  For finite
+// fp32 input E <= 128, so e <= 126 and the E8M0 range is never exceeded.
+__device__ __forceinline__ uint32_t e8m0_byte_ceil(uint32_t amax_bits)
+{
+    if (amax_bits == 0u)
+        return 127u;
+    const int E = amax_bits >= 0x00800000u ? (int)(amax_bits >> 23) - 126
+                                           : (32 - __clz((int)amax_bits)) - 149;
+    int e = max(E - 3, -127);
+    const float p2 = e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23)
+                               : __uint_as_float(0x00400000u); // 2^-127
+    if (__uint_as_float(amax_bits) > __fmul_rn(6.0f, p2))
+        ++e;
+    return (uint32_t)(e + 127);
+}
+
+// 2^-e as fp32 for the E8M0 byte b = e + 127 (b <= 253 from finite input):
 // biased exponent 127 - e = 254 - b, always normal.
 __device__ __forceinline__ float e8m0_inverse(uint32_t byte)
 {

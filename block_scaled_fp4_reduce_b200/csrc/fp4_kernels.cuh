@@ -5,7 +5,8 @@
 //                         the last CTA to finish, in one launch
 //   nvfp4_quantize_kernel block amax, E4M3 scale, element quotient, E2M1
 //                         rounding and nibble packing in one pass (section 3)
-//   mxfp4_quantize_kernel the same for 32-blocks with an E8M0 scale (section 5)
+//   mxfp4_quantize_kernel the same for 32-blocks with an E8M0 scale (section 5;
+//                         OCP rounding-down rule, or the page's ceil rule)
 //   dequantize_kernel     x_hat = q * s_b * g (NVFP4) or q * 2^e (MXFP4)
 //   scale_search_kernel   per-block MSE-minimising E4M3 scale
 //                         ("FP4 / NVFP4 数学总结" section 9)
@@ -336,9 +337,10 @@ __global__ void __launch_bounds__(kThreads)
 
 // ---------------------------------------------------------------------------
 // MXFP4 quantise + pack.  One thread per 32-element block: two 32-byte loads
-// (bf16) or four (fp32), one 16-byte packed store, one scale byte.
+// (bf16) or four (fp32), one 16-byte packed store, one scale byte.  kCeil
+// selects the ceil scale rule instead of the OCP rounding-down one.
 // ---------------------------------------------------------------------------
-template <typename T>
+template <typename T, bool kCeil = false>
 __global__ void __launch_bounds__(kThreads)
     mxfp4_quantize_kernel(const T *__restrict__ x, int64_t n_blocks,
                           uint4 *__restrict__ packed, uint8_t *__restrict__ scales,
@@ -361,7 +363,7 @@ __global__ void __launch_bounds__(kThreads)
             if (b < n_blocks) {
                 const uint32_t ab = absmax_bits(blk[u]);
                 bad |= ab >= kNonFiniteBits;
-                const uint32_t byte = e8m0_byte_floor(ab);
+                const uint32_t byte = kCeil ? e8m0_byte_ceil(ab) : e8m0_byte_floor(ab);
                 const float inv = e8m0_inverse(byte);
                 uint32_t pk[4];
 #pragma unroll
@@ -455,71 +457,232 @@ __global__ void __launch_bounds__(kThreads)
 // reconstruction T7 = fl32(fl32(6 s_b) g) is below A_b, the block maximum
 // alone contributes (A_b - T7)^2 to the loss, a lower bound that only grows
 // as the scale shrinks; once it exceeds the best loss so far no smaller
-// candidate can win or tie, and the loop stops (about 2.3 of 5 candidates
-// evaluated on Laplace data).
+// candidate can win or tie, and the search of the block stops (about 2.3 of
+// 5 candidates evaluated on Laplace data).
 //
-// Screening loss: the block scaled by k = 2^(127 - f) (f the exponent field
-// of A_b: A_b k in [1, 2), changing no comparison) with the reconstruction
-// x_hat k = fl32(fl32(p s_b) g k) (exact while g >= 2^-116) and codes from
-// one reciprocal product per element (misrounded only within a few ulps of
-// an E2M1 midpoint, where the two neighbouring reconstructions are
-// equidistant from x: their squared errors differ by at most 1.2e-5 of
-// that element's term), summed in fp32 (error < 1e-6).  A comparison the
-// screening sums cannot settle with a 5e-5 relative margin is redone on the
-// exact double loss of the definition -- exact codes, x_hat as dequantised,
-// sum_i ((double)x_i - (double)x_hat_i)^2 in element order -- so the winner
-// is the winner of the exact-in-double search, and on equal loss the larger
-// scale (the one met first) stays.
+// Screening: the block is scaled by k = 2^(127 - f) (f the exponent field
+// of A_b, so A_b k is in [1, 2); scaling changes no comparison).  With d_k =
+// fl32(s_b g) k, v_i = RN(x_i k r) (r within two ulps of 1/d_k) and p_i the
+// E2M1 grid value of v_i, the screening loss is S = d_k^2 sum_i (v_i - p_i)^2.
+// Against the exact scaled loss L = sum_i (x_i k - x_hat_i k)^2 it differs by
+// at most B(S, d_k) = 1e-6 S + 6e-6 sqrt(S) + 7e-5 d_k^2 + 1e-11: per element
+// the two differences agree within 2^-23 (1.5 |x k| + |x_hat k|) <= 7.2e-7;
+// an element within a few ulps of an E2M1 midpoint may round to the other
+// neighbour, whose squared error differs by at most 4.3e-6 d_k^2; the fp32
+// sum adds 1e-6 S.  A comparison with |S_a - S_b| <= B_a + B_b, and every
+// comparison when g < 2^-116 (reconstructions could be subnormal), is redone
+// on the exact double loss of the definition -- exact codes, x_hat as
+// dequantised, sum_i ((double)x_i - (double)x_hat_i)^2 in element order --
+// so the winner is the winner of the exact-in-double search, and on equal
+// loss the larger scale (the one met first) stays.
 // ---------------------------------------------------------------------------
+// Eight consecutive elements (half a block) reloaded from memory as fp32.
 template <typename T>
-__device__ __forceinline__ double exact_block_loss(const Blk<T, 16> &b, const uint2 &pk,
-                                                   uint32_t c, float g)
+__device__ __forceinline__ void load_half(const T *x, int64_t blk, int h, float (&v)[8])
+{
+    const char *p = reinterpret_cast<const char *>(x) + (blk * 16 + 8 * h) * (int64_t)sizeof(T);
+    uint32_t w[8];
+    if constexpr (sizeof(T) == 2) {
+        asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "l"(p));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[2 * j] = __uint_as_float(w[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    } else {
+        ldg_v8(p, w);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            v[j] = __uint_as_float(w[j]);
+    }
+}
+
+// Exact codes of one half-block at scale code c (zero scale -> zero codes).
+template <typename T>
+__device__ __forceinline__ uint32_t exact_half_codes(const T *x, int64_t blk, int h, uint32_t c,
+                                                     float g, float (&v)[8])
+{
+    load_half(x, blk, h, v);
+    if (c == 0u)
+        return 0u;
+    return nv_encode8(v, nv_recip(__fmul_rn(e4m3_pos_to_f32(c), g)));
+}
+
+// The definition's loss of scale code c over one block, in double, in
+// element order: exact codes, x_hat = fl32(fl32(p s_b) g), sum of
+// ((double)x - (double)x_hat)^2.  Reloads the block (an L2 hit); one half
+// at a time to stay light on registers (inlined: it is small, and ptxas
+// 12.9 crashed on an out-of-line version called from two kernels).
+template <typename T>
+__device__ __forceinline__ double exact_loss_of(const T *x, int64_t blk, uint32_t c, float g)
 {
     const float sb = e4m3_pos_to_f32(c);
     double acc = 0.0;
-#pragma unroll
+#pragma unroll 1
     for (int h = 0; h < 2; ++h) {
-        float p[8];
-        e2m1x8_decode(h ? pk.y : pk.x, p);
+        float v[8], p[8];
+        e2m1x8_decode(exact_half_codes(x, blk, h, c, g, v), p);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const double dd = __dsub_rn((double)elem(b, 8 * h + i), (double)nv_dequant(p[i], sb, g));
+            const double dd = __dsub_rn((double)v[i], (double)nv_dequant(p[i], sb, g));
             acc = __dadd_rn(acc, __dmul_rn(dd, dd));
         }
     }
     return acc;
 }
 
-// Screening loss of scale code c on the scaled block xk.
-__device__ __forceinline__ float screen_loss(const float (&xk)[16], uint32_t c, float g, float k,
-                                             float gk)
+// Exact codes of a whole block at scale code c (used when g is so small that
+// the scaled encode could see subnormal reconstructions).
+template <typename T>
+__device__ __forceinline__ uint2 exact_codes_of(const T *x, int64_t blk, uint32_t c, float g)
 {
-    float acc = 0.0f;
-    if (c == 0u) {
+    float v[8];
+    uint2 pk;
+    pk.x = exact_half_codes(x, blk, 0, c, g, v);
+    pk.y = exact_half_codes(x, blk, 1, c, g, v);
+    return pk;
+}
+
+// Screening loss of candidate code c and its error bound.
+struct Screen {
+    float s, bound;
+};
+
+__device__ __forceinline__ Screen screen(const float (&xk)[16], uint32_t c, float g, float k)
+{
+    Screen r;
+    if (c == 0u) { // zero scale: x_hat = 0, the sum of squares in fp32
+        float acc = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             acc = fmaf(xk[i], xk[i], acc);
-        return acc;
+        r.s = acc;
+        r.bound = fmaf(acc, 1e-6f, 1e-11f);
+        return r;
     }
-    const float sb = e4m3_pos_to_f32(c);
-    const float dk = __fmul_rn(__fmul_rn(sb, g), k);
+    const float dk = __fmul_rn(__fmul_rn(e4m3_pos_to_f32(c), g), k);
     const float r0 = rcp_approx(dk);
-    const float r = fmaf(r0, fmaf(-dk, r0, 1.0f), r0);
+    const float rc = fmaf(r0, fmaf(-dk, r0, 1.0f), r0);
+    float acc = 0.0f;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         float v[8], p[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            v[i] = __fmul_rn(xk[8 * h + i], r);
+            v[i] = __fmul_rn(xk[8 * h + i], rc);
         e2m1x8_qdq(v, p);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float d = __fsub_rn(xk[8 * h + i], __fmul_rn(__fmul_rn(p[i], sb), gk));
-            acc = fmaf(d, d, acc);
+            const float e = __fsub_rn(v[i], p[i]);
+            acc = fmaf(e, e, acc);
         }
     }
-    return acc;
+    const float d2 = __fmul_rn(dk, dk);
+    r.s = __fmul_rn(acc, d2);
+    r.bound = fmaf(r.s, 1e-6f, fmaf(sqrtf(r.s), 6e-6f, fmaf(d2, 7e-5f, 1e-11f)));
+    return r;
 }
+
+// One block's search.  Only the scaled block x k stays in registers: the
+// codes of x/d and of (x k)/(d k) are the same (the two quotients are the same
+// real number, and an x k that underflowed is tiny, code 0 with x's sign,
+// like x/d), so the final encode runs on x k; the exact comparisons and the
+// optional loss output reload the block.
+template <typename T> struct BlockSearch {
+    const T *x;
+    int64_t blk;
+    float xk[16];
+    float g, k, ak, gk;
+    uint32_t c_lo, best_c, next_c;
+    float best, best_bound;
+    bool exact_always;
+
+    // Loads the block; returns max |x| over it.
+    __device__ __forceinline__ float setup(const T *x_, int64_t blk_, float g_, bool exact_always_)
+    {
+        x = x_;
+        blk = blk_;
+        g = g_;
+        exact_always = exact_always_;
+        Blk<T, 16> b;
+        load_blk(x, blk, b);
+        const uint32_t ab = absmax_bits_finite(b);
+        k = __uint_as_float((254u - min(ab >> 23, 253u)) << 23);
+        gk = __fmul_rn(g, k);
+        ak = __fmul_rn(__uint_as_float(ab), k);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            xk[i] = __fmul_rn(elem(b, i), k);
+        return __uint_as_float(ab);
+    }
+
+    // Screen candidate c against the best so far; returns false when the
+    // lower bound ends the search.
+    __device__ __forceinline__ bool step(uint32_t c)
+    {
+        const float t7 = __fmul_rn(__fmul_rn(6.0f, e4m3_pos_to_f32(c)), gk);
+        if (ak > t7) {
+            const float e = __fsub_rn(ak, t7);
+            if (__fmul_rn(e, e) > __fmul_rn(__fadd_rn(best, best_bound), 1.0000003f))
+                return false;
+        }
+        const Screen sc = screen(xk, c, g, k);
+        bool take;
+        if (!exact_always && fabsf(__fsub_rn(sc.s, best)) > __fadd_rn(sc.bound, best_bound))
+            take = sc.s < best;
+        else
+            take = exact_loss_of(x, blk, c, g) < exact_loss_of(x, blk, best_c, g);
+        if (take) {
+            best_c = c;
+            best = sc.s;
+            best_bound = sc.bound;
+        }
+        return true;
+    }
+
+    // Continue from next_c down to c_lo for at most max_steps candidates;
+    // true when the search is complete.
+    __device__ __forceinline__ bool run(int max_steps)
+    {
+#pragma unroll 1
+        for (int n = 0; n < max_steps; ++n) {
+            if (next_c <= c_lo)
+                return true;
+            const uint32_t c = next_c - 1;
+            if (!step(c)) {
+                next_c = c_lo;
+                return true;
+            }
+            next_c = c;
+        }
+        return next_c <= c_lo;
+    }
+
+    __device__ __forceinline__ void finish(uint2 *packed, uint8_t *scales, float *block_loss)
+    {
+        uint2 pk = make_uint2(0u, 0u);
+        if (exact_always) {
+            pk = exact_codes_of(x, blk, best_c, g);
+        } else if (best_c != 0u) {
+            const NvRecip q = nv_recip(__fmul_rn(__fmul_rn(e4m3_pos_to_f32(best_c), g), k));
+            float h[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                h[i] = xk[i];
+            pk.x = nv_encode8(h, q);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                h[i] = xk[8 + i];
+            pk.y = nv_encode8(h, q);
+        }
+        packed[blk] = pk;
+        scales[blk] = (uint8_t)best_c;
+        if (block_loss)
+            block_loss[blk] = (float)exact_loss_of(x, blk, best_c, g);
+    }
+};
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -538,48 +701,57 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < n_blocks;
          blk += stride) {
-        Blk<T, 16> b;
-        load_blk(x, blk, b);
-        const uint32_t ab = absmax_bits_finite(b);
-        const float amax_b = __uint_as_float(ab);
+        BlockSearch<T> bs;
+        const float amax_b = bs.setup(x, blk, g, exact_always);
         const uint32_t c_hi = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
-        const uint32_t c_lo = nv_scale_code(amax_b, inv_lo, 147.0, g1260);
-        const float k = __uint_as_float((254u - min(ab >> 23, 253u)) << 23);
-        const float gk = __fmul_rn(g, k);
-        const float ak = __fmul_rn(amax_b, k);
-        float xk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            xk[i] = __fmul_rn(elem(b, i), k);
+        bs.c_lo = nv_scale_code(amax_b, inv_lo, 147.0, g1260);
+        bs.best_c = c_hi;
+        bs.next_c = c_hi;
+        const Screen s0 = screen(bs.xk, c_hi, g, bs.k);
+        bs.best = s0.s;
+        bs.best_bound = s0.bound;
+        bs.run(128);
+        bs.finish(packed, scales, block_loss);
+    }
+}
 
-        uint32_t best_c = c_hi;
-        float best = screen_loss(xk, c_hi, g, k, gk);
-        for (uint32_t c = c_hi; c > c_lo;) {
-            --c;
-            const float t7 = __fmul_rn(__fmul_rn(6.0f, e4m3_pos_to_f32(c)), gk);
-            if (ak > t7) {
-                const float e = __fsub_rn(ak, t7);
-                if (__fmul_rn(e, e) > fmaf(best, 6e-5f, best) + 0x1p-130f)
-                    break;
-            }
-            const float l = screen_loss(xk, c, g, k, gk);
-            const float hi = fmaxf(l, best), lo = fminf(l, best);
-            bool take;
-            if (!exact_always && __fsub_rn(hi, lo) > fmaf(hi, 5e-5f, 0x1p-130f))
-                take = l < best;
-            else
-                take = exact_block_loss(b, nv_block_codes(b, c, g), c, g) <
-                       exact_block_loss(b, nv_block_codes(b, best_c, g), best_c, g);
-            if (take) {
-                best_c = c;
-                best = l;
-            }
-        }
-        const uint2 pk = nv_block_codes(b, best_c, g);
-        packed[blk] = pk;
-        scales[blk] = (uint8_t)best_c;
-        if (block_loss)
-            block_loss[blk] = (float)exact_block_loss(b, pk, best_c, g);
+// ---------------------------------------------------------------------------
+// NVFP4 "four over six" ("FP4、FP8 与 INT8/INT4" section 4: mapping the block
+// maximum to 4 instead of 6 can put the other values on better grid points;
+// neither wins on every block).  Per block the E4M3 codes nearest to
+// A_b/(6g) (the max-based scale) and A_b/(4g) are compared on the loss of the
+// emitted artefact, screened and, when close, settled exactly as in the
+// search; the max-to-4 scale is taken only when strictly better.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+    nvfp4_four_over_six_kernel(const T *__restrict__ x, int64_t n_blocks, const float *amax,
+                               uint2 *__restrict__ packed, uint8_t *__restrict__ scales,
+                               float *global_scale, float *__restrict__ block_loss,
+                               int32_t *status)
+{
+    pdl_begin();
+    float g;
+    if (!nv_prologue(amax, global_scale, status, g))
+        return;
+    const NvScaleConsts sc = nv_scale_consts(g);
+    const double four_g = 4.0 * (double)g;    // exact
+    const float inv4g = (float)(1.0 / four_g); // RN32(1 / (4g))
+    const bool exact_always = !(g >= 0x1p-116f);
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < n_blocks;
+         blk += stride) {
+        BlockSearch<T> bs;
+        const float amax_b = bs.setup(x, blk, g, exact_always);
+        const uint32_t c6 = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
+        const uint32_t c4 = nv_scale_code(amax_b, inv4g, 1.0, four_g);
+        bs.best_c = c6;
+        const Screen s0 = screen(bs.xk, c6, g, bs.k);
+        bs.best = s0.s;
+        bs.best_bound = s0.bound;
+        if (c4 != c6)
+            bs.step(c4);
+        bs.finish(packed, scales, block_loss);
     }
 }
 

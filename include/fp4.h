@@ -140,6 +140,29 @@ fp4_status fp4_mxfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int6
                               uint8_t *packed, uint8_t *scales, int32_t *status,
                               cudaStream_t stream);
 
+/* MXFP4 quantise + pack with the ceil scale rule of "NVFP4 与 MXFP4 格式"
+ * section 5 and its section 6 helper (ModelOpt-style 2^ceil(log2(A_b/6))):
+ * e = max(E - 3, -127) with A_b = m 2^E (m in [0.5, 1)), plus 1 when
+ * A_b > 6 * 2^e; an all-zero block gets scale 1 (byte 127).  No element
+ * clips.  Otherwise as fp4_mxfp4_quantize; dequantise with FP4_MXFP4. */
+fp4_status fp4_mxfp4_quantize_ceil(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                   uint8_t *packed, uint8_t *scales, int32_t *status,
+                                   cudaStream_t stream);
+
+/* NVFP4 quantise + pack with the "four over six" block scale
+ * ("FP4、FP8 与 INT8/INT4" section 4: mapping the block maximum to 4 rather
+ * than 6 can place the other values on better grid points).  g as for
+ * fp4_nvfp4_quantize; per block the E4M3 codes nearest to A_b/(6g) and to
+ * A_b/(4g) are compared on the loss of the emitted artefact (as in
+ * fp4_scale_search, summed in double); the max-to-4 scale is taken only
+ * when strictly better.  block_loss (nullable) gets the chosen loss in
+ * fp32.  Dequantise with FP4_NVFP4.  Data errors: NONFINITE, RANGE. */
+fp4_status fp4_nvfp4_quantize_four_over_six(const void *x, fp4_dtype dtype, int64_t rows,
+                                            int64_t cols, uint8_t *packed, uint8_t *scales,
+                                            float *global_scale, float *block_loss,
+                                            void *workspace, size_t workspace_bytes,
+                                            int32_t *status, cudaStream_t stream);
+
 /* Dequantise ("FP4 / NVFP4 数学总结" section 3, x_hat = q * s_b * g;
  * "FP4、FP8 与 INT8/INT4" section 3.2, x_hat = 2^e q).
  *   NVFP4: y = fl32(fl32(p * s_b) * g), p the E2M1 value of the code

@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
             "oracle_mx_block_exponent_ceil": (I, [F, P]),
             "oracle_mxfp4_quantize_rule": (I, [P, I, I64, I64, I, P, P]),
             "oracle_nvfp4_quantize_four_over_six": (I, [P, I, I64, I64, P, P, P, P]),
+            "oracle_nvfp4_quantize_four_over_six_with_g": (I, [P, I, I64, I64, F, P, P, P]),
             "oracle_mxfp4_dequantize": (None, [P, P, I64, I64, P]),
             "oracle_nv_block_loss": (D, [P, I, F]),
             "oracle_search_candidate_code": (I, [F, F, I]),
@@ -291,6 +292,18 @@ def nvfp4_quantize_four_over_six(x: np.ndarray):
     _check(lib().oracle_nvfp4_quantize_four_over_six(_ptr(x), dt, R, C, _ptr(packed), _ptr(scales),
                                                      ctypes.byref(g), _ptr(loss)))
     return packed, scales, g.value, loss
+
+
+def nvfp4_quantize_four_over_six_with_g(x: np.ndarray, g: float):
+    """Four over six at a given global scale.  Returns (packed, scales, loss)."""
+    x, dt = _input(x)
+    R, C = _shape(x)
+    packed = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    loss = np.zeros((R, C // 16), np.float64)
+    _check(lib().oracle_nvfp4_quantize_four_over_six_with_g(_ptr(x), dt, R, C, float(g), _ptr(packed),
+                                                            _ptr(scales), _ptr(loss)))
+    return packed, scales, loss
 
 
 def nvfp4_dequantize(packed: np.ndarray, scales: np.ndarray, g: float, rows: int, cols: int) -> np.ndarray:

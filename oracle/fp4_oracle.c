@@ -588,26 +588,20 @@ int oracle_nvfp4_scale_search(const void *x, int dtype, int64_t rows, int64_t co
  * codes nearest to A_b / (6g) (the max-based scale) and A_b / (4g); the
  * second is taken only when its artefact loss is strictly smaller.  g as
  * for NVFP4.  Emits codes, scale codes, g and the chosen loss. */
-int oracle_nvfp4_quantize_four_over_six(const void *x, int dtype, int64_t rows, int64_t cols,
-                                        uint8_t *packed, uint8_t *scales, float *g_out,
-                                        double *block_loss)
+int oracle_nvfp4_quantize_four_over_six_with_g(const void *x, int dtype, int64_t rows,
+                                               int64_t cols, float g, uint8_t *packed,
+                                               uint8_t *scales, double *block_loss)
 {
     if (cols % 16 || rows < 0 || cols < 0)
         return ORACLE_ERR_SHAPE;
-    float amax, g;
-    int st = oracle_tensor_amax(x, dtype, rows * cols, &amax);
-    if (st)
-        return st;
-    st = oracle_nv_global_scale(amax, &g);
-    if (st)
-        return st;
-    *g_out = g;
     int64_t nblocks = rows * cols / 16;
     for (int64_t b = 0; b < nblocks; ++b) {
         float xb[16];
         float ab = 0.0f;
         for (int i = 0; i < 16; ++i) {
             xb[i] = load_elem(x, dtype, b * 16 + i);
+            if (!isfinite(xb[i]))
+                return ORACLE_ERR_NONFINITE;
             if (fabsf(xb[i]) > ab)
                 ab = fabsf(xb[i]);
         }
@@ -624,6 +618,24 @@ int oracle_nvfp4_quantize_four_over_six(const void *x, int dtype, int64_t rows, 
             block_loss[b] = l4 < l6 ? l4 : l6;
     }
     return ORACLE_OK;
+}
+
+int oracle_nvfp4_quantize_four_over_six(const void *x, int dtype, int64_t rows, int64_t cols,
+                                        uint8_t *packed, uint8_t *scales, float *g_out,
+                                        double *block_loss)
+{
+    if (cols % 16 || rows < 0 || cols < 0)
+        return ORACLE_ERR_SHAPE;
+    float amax, g;
+    int st = oracle_tensor_amax(x, dtype, rows * cols, &amax);
+    if (st)
+        return st;
+    st = oracle_nv_global_scale(amax, &g);
+    if (st)
+        return st;
+    *g_out = g;
+    return oracle_nvfp4_quantize_four_over_six_with_g(x, dtype, rows, cols, g, packed, scales,
+                                                      block_loss);
 }
 
 /* Per-block loss of given (packed, scale) artefacts against x, for
