@@ -90,6 +90,11 @@ def lib() -> ctypes.CDLL:
             "oracle_nvfp4_scale_search_with_g": (I, [P, I, I64, I64, F, P, P, P]),
             "oracle_nvfp4_artefact_loss": (I, [P, I, I64, I64, P, P, F, P]),
             "oracle_storage_bytes": (I64, [I64, I64, I64]),
+            "oracle_padded_blocks": (I64, [I64, I64, I64]),
+            "oracle_padded_storage_bytes": (I64, [I64, I64, I64, I64]),
+            "oracle_pad_rows": (I, [P, I, I64, I64, I64, P]),
+            "oracle_crop_rows": (I, [P, I64, I64, I64, P]),
+            "oracle_transpose": (I, [P, I, I64, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -380,3 +385,79 @@ def storage_bytes(elements: int, group: int, global_bytes: int) -> int:
     if n < 0:
         raise OracleError(ERR_SHAPE, "complete blocks required")
     return n
+
+
+# --------------------------------------------------------------------------
+# Ragged rows and column-wise grouping ("NVFP4 与 MXFP4 格式" sections 6-8)
+# --------------------------------------------------------------------------
+
+def padded_cols(cols: int, group: int) -> int:
+    """Row length after padding to whole blocks: ceil(cols / G) * G."""
+    return -(-int(cols) // group) * group
+
+
+def padded_blocks(rows: int, cols: int, group: int) -> int:
+    return lib().oracle_padded_blocks(int(rows), int(cols), int(group))
+
+
+def padded_storage_bytes(rows: int, cols: int, group: int, global_bytes: int) -> int:
+    n = lib().oracle_padded_storage_bytes(int(rows), int(cols), int(group), int(global_bytes))
+    if n < 0:
+        raise OracleError(ERR_ARG, "group must be 16 or 32")
+    return n
+
+
+def pad_rows(x: np.ndarray, group: int) -> np.ndarray:
+    """x [R, K] with every row padded by +0 to whole blocks of `group`."""
+    x, dt = _input(x)
+    R, K = _shape(x)
+    Kp = padded_cols(K, group)
+    out = np.zeros((R, Kp), x.dtype)
+    _check(lib().oracle_pad_rows(_ptr(x), dt, R, K, Kp, _ptr(out)))
+    return out
+
+
+def crop_rows(y: np.ndarray, cols: int) -> np.ndarray:
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    R, Kp = y.shape
+    out = np.zeros((R, cols), np.float32)
+    _check(lib().oracle_crop_rows(_ptr(y), R, Kp, int(cols), _ptr(out)))
+    return out
+
+
+def transpose(x: np.ndarray) -> np.ndarray:
+    x, dt = _input(x)
+    R, C = _shape(x)
+    out = np.zeros((C, R), x.dtype)
+    _check(lib().oracle_transpose(_ptr(x), dt, R, C, _ptr(out)))
+    return out
+
+
+def nvfp4_quantize_padded(x: np.ndarray):
+    """NVFP4 of x [R, K] with rows padded by +0 to whole 16-blocks: packed
+    [R, ceil(K/16)*8], scales [R, ceil(K/16)], g (pads do not change A)."""
+    return nvfp4_quantize(pad_rows(x, 16))
+
+
+def mxfp4_quantize_padded(x: np.ndarray, rule: int = 0):
+    """MXFP4 of x [R, K] with rows padded by +0 to whole 32-blocks."""
+    return mxfp4_quantize_rule(pad_rows(x, 32), rule)
+
+
+def nvfp4_dequantize_padded(packed, scales, g, rows: int, cols: int) -> np.ndarray:
+    """Dequantise the padded layout, then crop every row to `cols`."""
+    return crop_rows(nvfp4_dequantize(packed, scales, g, rows, padded_cols(cols, 16)), cols)
+
+
+def mxfp4_dequantize_padded(packed, scales, rows: int, cols: int) -> np.ndarray:
+    return crop_rows(mxfp4_dequantize(packed, scales, rows, padded_cols(cols, 32)), cols)
+
+
+def nvfp4_quantize_columns(x: np.ndarray):
+    """NVFP4 of x [R, C] grouped along columns: the padded row-wise
+    quantisation of the transpose, packed [C, ceil(R/16)*8]."""
+    return nvfp4_quantize_padded(transpose(x))
+
+
+def mxfp4_quantize_columns(x: np.ndarray, rule: int = 0):
+    return mxfp4_quantize_padded(transpose(x), rule)

@@ -669,3 +669,77 @@ int64_t oracle_storage_bytes(int64_t elements, int64_t group, int64_t global_byt
         return -1;
     return elements / 2 + elements / group + global_bytes;
 }
+
+/* ------------------------------------------------------------------ */
+/* Ragged rows and the other grouping axis ([NVMX] S6, S7, S8).        */
+/* ------------------------------------------------------------------ */
+
+/* Blocks of a row-padded [rows, cols] matrix, B = rows * ceil(cols / G)
+ * ([NVMX] S8: padding each row gives this count, not ceil(rows*cols/G)). */
+int64_t oracle_padded_blocks(int64_t rows, int64_t cols, int64_t group)
+{
+    if (rows < 0 || cols < 0 || group <= 0)
+        return -1;
+    return rows * ((cols + group - 1) / group);
+}
+
+/* Storage of a row-padded matrix ([NVMX] S8): B (G/2 + 1) bytes of payload
+ * and block scales, plus the bytes of any tensor-level scale. */
+int64_t oracle_padded_storage_bytes(int64_t rows, int64_t cols, int64_t group,
+                                    int64_t global_bytes)
+{
+    if ((group != 16 && group != 32) || global_bytes < 0)
+        return -1;
+    int64_t b = oracle_padded_blocks(rows, cols, group);
+    if (b < 0)
+        return -1;
+    return b * (group / 2 + 1) + global_bytes;
+}
+
+/* Pads every row of x [rows, cols] to padded_cols >= cols elements with +0
+ * (the pad value is not given on the page; +0 leaves every block maximum as
+ * it was).  out holds rows * padded_cols elements of x's type. */
+int oracle_pad_rows(const void *x, int dtype, int64_t rows, int64_t cols, int64_t padded_cols,
+                    void *out)
+{
+    if (rows < 0 || cols < 0 || padded_cols < cols || (dtype != ORACLE_F32 && dtype != ORACLE_BF16))
+        return ORACLE_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < padded_cols; ++c) {
+            if (dtype == ORACLE_F32)
+                ((float *)out)[r * padded_cols + c] = c < cols ? ((const float *)x)[r * cols + c] : 0.0f;
+            else
+                ((uint16_t *)out)[r * padded_cols + c] =
+                    c < cols ? ((const uint16_t *)x)[r * cols + c] : (uint16_t)0;
+        }
+    return ORACLE_OK;
+}
+
+/* Keeps the first cols of every padded row ([NVMX] S7: decode the padded
+ * layout, then cut each row back to the original shape). */
+int oracle_crop_rows(const float *y_padded, int64_t rows, int64_t padded_cols, int64_t cols,
+                     float *y)
+{
+    if (rows < 0 || cols < 0 || padded_cols < cols)
+        return ORACLE_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            y[r * cols + c] = y_padded[r * padded_cols + c];
+    return ORACLE_OK;
+}
+
+/* out [cols, rows] = x [rows, cols] transposed ([NVMX] S6: grouping the
+ * transposed matrix by rows groups the original by columns). */
+int oracle_transpose(const void *x, int dtype, int64_t rows, int64_t cols, void *out)
+{
+    if (rows < 0 || cols < 0 || (dtype != ORACLE_F32 && dtype != ORACLE_BF16))
+        return ORACLE_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            if (dtype == ORACLE_F32)
+                ((float *)out)[c * rows + r] = ((const float *)x)[r * cols + c];
+            else
+                ((uint16_t *)out)[c * rows + r] = ((const uint16_t *)x)[r * cols + c];
+        }
+    return ORACLE_OK;
+}
