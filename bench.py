@@ -45,12 +45,19 @@ WORKLOADS = {
     "act-8192x14336-bf16": workloads.ACT_8K,
     "search-4096x14336-bf16": workloads.SEARCH_4K,
     "tiny-f32-256x1024": workloads.TINY_F32,
+    "model-7b-weights-bf16": workloads.MODEL_WEIGHTS,
+    "columns-4096x14336-bf16": workloads.COLUMNS_4K,
+    "ragged-8192x14335-bf16": workloads.RAGGED_8K,
+    "variants-8192x14336-bf16": workloads.VARIANTS_8K,
 }
+LAYOUT_WORKLOADS = {"columns-4096x14336-bf16": "columns", "ragged-8192x14335-bf16": "padded",
+                    "variants-8192x14336-bf16": "variants"}
+MODEL_WEIGHTS = "model-7b-weights-bf16"  # the whole weight set, grouped calls
 DEFAULT_WORKLOAD = "weight-4096x4096-bf16"
 KERNEL_SOURCES = ["block_scaled_fp4_reduce_b200/csrc/fp4_kernels.cuh",
-                  "block_scaled_fp4_reduce_b200/csrc/fp4_codec.cuh"]
+                  "block_scaled_fp4_reduce_b200/csrc/fp4_codec.cuh",
+                  "block_scaled_fp4_reduce_b200/csrc/fp4_grouped.cuh"]
 OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize", "scale_search"]
-LAUNCHES_PER_STEP = 6  # one kernel per entry point (the amax folds in its last CTA)
 
 
 def peaks() -> dict:
@@ -74,7 +81,8 @@ def kernel_source_hash() -> str:
 def algorithmic_bytes(w: workloads.Workload) -> dict:
     """Bytes each kernel must move per launch (read + write), by definition:
     x once per pass, packed codes 1/2 byte per element, one scale byte per
-    block, dequantised bf16 output 2 bytes per element."""
+    block, dequantised bf16 output 2 bytes per element (the grouped weight
+    set: the same per element over all its matrices)."""
     n, e = w.numel, (2 if w.dtype == torch.bfloat16 else 4)
     return {
         "amax": n * e,
@@ -190,6 +198,9 @@ class Path:
         self.results = [self.nv_p, self.nv_s, self.nv_g, self.mx_p, self.mx_s, self.ss_p, self.ss_s,
                         self.status]
 
+    OPS = OPS
+    LAUNCHES = 6  # one kernel per entry point (the amax folds in its last CTA)
+
     def step(self, events=None):
         for i, (fn, args) in enumerate(self.calls):
             st = fn(*args)
@@ -202,6 +213,141 @@ class Path:
         st = int(self.status.item())
         if st:
             raise self.fp4.FP4Error(st, "bench step")
+
+
+class GroupedPath:
+    """The whole 7B-class weight set (32 layers x 4 x 4096^2 + 3 x 4096x14336
+    bf16 matrices, each generated from its own seed) in one flat device
+    buffer; one step = grouped amax, grouped NVFP4 quantise (per-matrix g),
+    grouped MXFP4 quantise, grouped NVFP4 and MXFP4 dequantise to bf16: five
+    entry points, one kernel each (plus the clear of the amax words)."""
+    OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize"]
+    LAUNCHES = 5
+
+    def __init__(self, device, rank: int = 0):
+        import block_scaled_fp4_reduce_b200 as fp4
+        self.fp4 = fp4
+        L = fp4.lib()
+        self.ws_list = [workloads.model_matrix(l, i) for l in range(workloads.MODEL_LAYERS)
+                        for i in range(len(workloads.MODEL_MATRICES))]
+        if rank:
+            self.ws_list = [workloads.for_rank(w, rank) for w in self.ws_list]
+        sizes = [w.numel for w in self.ws_list]
+        self.n = sum(sizes)
+        u8, bf = torch.uint8, torch.bfloat16
+        self.x = torch.empty(self.n, dtype=bf, device=device)
+        off, self.xs = 0, []
+        for w, m in zip(self.ws_list, sizes):
+            v = self.x[off:off + m].view(w.rows, w.cols)
+            v.copy_(workloads.generate(w, device=device))
+            self.xs.append(v)
+            off += m
+        n = self.n
+        self.nv_p, self.nv_s = torch.empty(n // 2, dtype=u8, device=device), torch.empty(n // 16, dtype=u8, device=device)
+        self.mx_p, self.mx_s = torch.empty(n // 2, dtype=u8, device=device), torch.empty(n // 32, dtype=u8, device=device)
+        self.nv_g = torch.empty(len(sizes), dtype=torch.float32, device=device)
+        self.y_nv = torch.empty(n, dtype=bf, device=device)
+        self.y_mx = torch.empty(n, dtype=bf, device=device)
+        self.ws = torch.empty(L.fp4_grouped_workspace_bytes(len(sizes)), dtype=u8, device=device)
+        self.status = fp4.new_status(device)
+        k = len(sizes)
+        self.q_nv = (fp4.QuantItem * k)()
+        self.q_mx = (fp4.QuantItem * k)()
+        self.d_nv = (fp4.DequantItem * k)()
+        self.d_mx = (fp4.DequantItem * k)()
+        off = 0
+        for j, (w, m) in enumerate(zip(self.ws_list, sizes)):
+            P = lambda t, o: t.data_ptr() + o * t.element_size()  # noqa: E731
+            self.q_nv[j] = fp4.QuantItem(P(self.x, off), w.rows, w.cols, P(self.nv_p, off // 2),
+                                         P(self.nv_s, off // 16), P(self.nv_g, j))
+            self.q_mx[j] = fp4.QuantItem(P(self.x, off), w.rows, w.cols, P(self.mx_p, off // 2),
+                                         P(self.mx_s, off // 32), None)
+            self.d_nv[j] = fp4.DequantItem(P(self.nv_p, off // 2), P(self.nv_s, off // 16), P(self.nv_g, j),
+                                           P(self.y_nv, off), w.rows, w.cols)
+            self.d_mx[j] = fp4.DequantItem(P(self.mx_p, off // 2), P(self.mx_s, off // 32), None,
+                                           P(self.y_mx, off), w.rows, w.cols)
+            off += m
+        st = torch.cuda.current_stream().cuda_stream
+        cp = lambda a: ctypes.cast(a, ctypes.c_void_p)  # noqa: E731
+        ws, stp = self.ws.data_ptr(), self.status.data_ptr()
+        self.calls = [
+            (L.fp4_tensor_amax_grouped, (cp(self.q_nv), k, fp4.BF16, ws, self.ws.numel(), stp, st)),
+            (L.fp4_nvfp4_quantize_grouped_with_amax, (cp(self.q_nv), k, fp4.BF16, ws, stp, st)),
+            (L.fp4_mxfp4_quantize_grouped, (cp(self.q_mx), k, fp4.BF16, stp, st)),
+            (L.fp4_dequantize_grouped, (fp4.NVFP4, cp(self.d_nv), k, fp4.BF16, st)),
+            (L.fp4_dequantize_grouped, (fp4.MXFP4, cp(self.d_mx), k, fp4.BF16, st)),
+        ]
+        self.results = [self.nv_p, self.nv_s, self.nv_g, self.mx_p, self.mx_s, self.status]
+
+    step = Path.step
+    check_status = Path.check_status
+
+
+class LayoutPath:
+    """The other block layouts and scale rules on one tensor x [R, K]:
+    "variants" = amax, NVFP4 four over six (it runs its own amax: two
+    launches), MXFP4 with the ceil scale rule, dequantisation of both to
+    bf16; "columns" = amax,
+    column-wise NVFP4 quantise (Q(W^T), g from the amax), column-wise MXFP4
+    quantise, dequantisation of both padded layouts of the [K, R] transpose
+    to bf16; "padded" = amax, NVFP4 and MXFP4 quantise of rows padded to
+    whole blocks, dequantisation of both back to the logical [R, K] bf16."""
+    OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize"]
+    LAUNCHES = 5
+
+    def __init__(self, x: torch.Tensor, kind: str):
+        import block_scaled_fp4_reduce_b200 as fp4
+        self.fp4 = fp4
+        L = fp4.lib()
+        dev = x.device
+        R, K = x.shape
+        self.x, self.n, self.kind = x, x.numel(), kind
+        u8 = torch.uint8
+        if kind == "columns":  # outputs describe the [K, R] transpose
+            OR, OC = K, R
+        else:
+            OR, OC = R, K
+        pad = lambda c, gsz: -(-c // gsz) * gsz  # noqa: E731
+        self.amax = torch.empty(1, dtype=torch.float32, device=dev)
+        self.ws = fp4.workspace_for(x)
+        self.status = fp4.new_status(dev)
+        self.nv_p = torch.empty((OR, pad(OC, 16) // 2), dtype=u8, device=dev)
+        self.nv_s = torch.empty((OR, pad(OC, 16) // 16), dtype=u8, device=dev)
+        self.nv_g = torch.empty(1, dtype=torch.float32, device=dev)
+        self.mx_p = torch.empty((OR, pad(OC, 32) // 2), dtype=u8, device=dev)
+        self.mx_s = torch.empty((OR, pad(OC, 32) // 32), dtype=u8, device=dev)
+        self.y_nv = torch.empty((OR, OC), dtype=torch.bfloat16, device=dev)
+        self.y_mx = torch.empty((OR, OC), dtype=torch.bfloat16, device=dev)
+        st = torch.cuda.current_stream().cuda_stream
+        dt = fp4._dtype_code(x)
+        P = lambda t: t.data_ptr()  # noqa: E731
+        ws_bytes = self.ws.numel()
+        if kind == "variants":  # four over six (its own amax inside) and the MXFP4 ceil rule
+            nv_call = (L.fp4_nvfp4_quantize_four_over_six, (P(x), dt, R, K, P(self.nv_p), P(self.nv_s), P(self.nv_g),
+                                                           None, P(self.ws), ws_bytes, P(self.status), st))
+            mx_call = (L.fp4_mxfp4_quantize_ceil, (P(x), dt, R, K, P(self.mx_p), P(self.mx_s), P(self.status), st))
+        else:
+            nvq = L.fp4_nvfp4_quantize_columns if kind == "columns" else L.fp4_nvfp4_quantize_padded
+            mxq = L.fp4_mxfp4_quantize_columns if kind == "columns" else L.fp4_mxfp4_quantize_padded
+            nv_call = (nvq, (P(x), dt, R, K, P(self.nv_p), P(self.nv_s), P(self.nv_g), P(self.ws), ws_bytes,
+                             P(self.status), st))
+            mx_call = (mxq, (P(x), dt, R, K, fp4.MX_FLOOR, P(self.mx_p), P(self.mx_s), P(self.status), st))
+        self.calls = [
+            (L.fp4_tensor_amax, (P(x), dt, self.n, P(self.amax), P(self.ws), ws_bytes, P(self.status), st)),
+            nv_call,
+            mx_call,
+            (L.fp4_dequantize_padded, (fp4.NVFP4, P(self.nv_p), P(self.nv_s), P(self.nv_g), OR, OC,
+                                       P(self.y_nv), fp4.BF16, st)),
+            (L.fp4_dequantize_padded, (fp4.MXFP4, P(self.mx_p), P(self.mx_s), None, OR, OC, P(self.y_mx),
+                                       fp4.BF16, st)),
+        ]
+        self.results = [self.nv_p, self.nv_s, self.nv_g, self.mx_p, self.mx_s, self.status]
+
+        if kind == "variants":
+            self.LAUNCHES = 6
+
+    step = Path.step
+    check_status = Path.check_status
 
 
 def max_over_ranks(values: list[float], device, world: int) -> list[float]:
@@ -235,9 +381,16 @@ def run_ours(args, rank: int, world: int, local: int):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     w = workloads.for_rank(WORKLOADS[args.workload], rank)
-    x_host = workloads.generate(w).pin_memory()
-    x = x_host.to(dev, non_blocking=False)
-    path = Path(x)
+    if args.workload == MODEL_WEIGHTS:
+        path = GroupedPath(dev, rank)
+        x = path.x
+        x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+        x_host.copy_(x)
+    else:
+        x_host = workloads.generate(w).pin_memory()
+        x = x_host.to(dev, non_blocking=False)
+        kind = LAYOUT_WORKLOADS.get(args.workload)
+        path = LayoutPath(x, kind) if kind else Path(x)
     flush_l2 = L2Flush(args.flush_mib, dev)
     nops = len(path.calls)
 
@@ -306,13 +459,26 @@ def run_ours(args, rank: int, world: int, local: int):
     pk = peaks()
     ab = algorithmic_bytes(w)
     kernels = {}
-    for name, ms in zip(OPS, per_op_ms):
+    for name, ms in zip(path.OPS, per_op_ms):
         us = ms / K * 1e3
         gbs = ab[name] / (us * 1e-6) / 1e9
         kernels[name] = {"us": round(us, 3), "share": round(ms / total_ms, 4), "gbs": round(gbs, 1),
                          "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
     dom = max(kernels, key=lambda k: kernels[k]["us"])
     n_cand = search_candidate_count(x, path.ss_g.item()) if dom == "scale_search" else None
+    step_desc = ("amax, nvfp4 quantize, mxfp4 quantize, nvfp4 dequantize (bf16), mxfp4 dequantize (bf16), "
+                 "nvfp4 64-candidate scale search")
+    if args.workload in LAYOUT_WORKLOADS:
+        step_desc = {"columns": "amax, column-wise nvfp4 quantize (Q(W^T)), column-wise mxfp4 quantize, "
+                                "nvfp4 and mxfp4 dequantize of the transposed padded layouts (bf16)",
+                     "padded": "amax, nvfp4 and mxfp4 quantize of rows padded to whole blocks, nvfp4 and "
+                               "mxfp4 dequantize back to the logical shape (bf16)",
+                     "variants": "amax, nvfp4 four-over-six quantize (its own amax + the two-candidate kernel), "
+                                 "mxfp4 quantize with the ceil scale rule, nvfp4 and mxfp4 dequantize (bf16)"
+                     }[LAYOUT_WORKLOADS[args.workload]]
+    if args.workload == MODEL_WEIGHTS:
+        step_desc = ("grouped over all 224 matrices (one kernel per pass): per-matrix amax, nvfp4 quantize "
+                     "(per-matrix g), mxfp4 quantize, nvfp4 dequantize (bf16), mxfp4 dequantize (bf16)")
     roof = roofline_for(dom, kernels[dom], w, pk, n_cand)
     line = {
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": K,
@@ -320,18 +486,19 @@ def run_ours(args, rank: int, world: int, local: int):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name if world == 1 else WORKLOADS[args.workload].name,
                    "description": WORKLOADS[args.workload].description,
-                   "shape": [w.rows, w.cols], "input_dtype": str(w.dtype).replace("torch.", ""),
-                   "step": "amax, nvfp4 quantize, mxfp4 quantize, nvfp4 dequantize (bf16), "
-                           "mxfp4 dequantize (bf16), nvfp4 64-candidate scale search",
+                   "shape": ([[r, c] for r, c in workloads.MODEL_MATRICES] if args.workload == MODEL_WEIGHTS
+                             else [w.rows, w.cols]),
+                   "input_dtype": str(w.dtype).replace("torch.", ""),
+                   "step": step_desc,
                    "l2": f"flushed between steps outside the timed events ({args.flush_mib} MiB write, "
                          f"then {args.flush_mib // 2} MiB read)",
                    "parallelism": f"replicas x{world} (independent tensors)" if world > 1 else "single GPU"},
-        "hbm_gbs_step": sum(ab.values()) / (total_ms / K * 1e-3) / 1e9,
+        "hbm_gbs_step": sum(ab[o] for o in path.OPS) / (total_ms / K * 1e-3) / 1e9,
         "kernels": kernels,
         "roofline": roof,
         "e2e": {"value": n_all * Ke / (e2e_ms / 1e3), "unit": "elements/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "gpu_launches": path.LAUNCHES * K,
         "clocks": clk,
         "wall_s_timed": wall,
     }
@@ -385,34 +552,73 @@ def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict, n_cand: in
 
 # ------------------------------------------------------- CPU oracle legs --
 
-def _oracle_step(xs):
+def _oracle_step(xs, search: bool = True):
     import oracle
     p, s, g = oracle.nvfp4_quantize(xs)
     pm, sm = oracle.mxfp4_quantize(xs)
     R, C = xs.shape
     oracle.nvfp4_dequantize(p, s, g, R, C)
     oracle.mxfp4_dequantize(pm, sm, R, C)
-    oracle.nvfp4_scale_search(xs)
+    if search:
+        oracle.nvfp4_scale_search(xs)
+
+
+def _oracle_layout_step(xs, kind: str):
+    """The layout and variant workloads' step on the oracle: four over six
+    and the MXFP4 ceil rule, or column-wise or row-padded quantisation in
+    both formats, then the dequantisations."""
+    import oracle
+    R, C = xs.shape
+    if kind == "variants":
+        p, s, g, _ = oracle.nvfp4_quantize_four_over_six(xs)
+        pm, sm = oracle.mxfp4_quantize_rule(xs, oracle.MX_CEIL)
+        oracle.nvfp4_dequantize(p, s, g, R, C)
+        oracle.mxfp4_dequantize(pm, sm, R, C)
+        return
+    if kind == "columns":
+        p, s, g = oracle.nvfp4_quantize_columns(xs)
+        pm, sm = oracle.mxfp4_quantize_columns(xs)
+        R, C = C, R
+    else:
+        p, s, g = oracle.nvfp4_quantize_padded(xs)
+        pm, sm = oracle.mxfp4_quantize_padded(xs)
+    oracle.nvfp4_dequantize_padded(p, s, g, R, C)
+    oracle.mxfp4_dequantize_padded(pm, sm, R, C)
+
+
+def oracle_sample_source(w: workloads.Workload):
+    """(tensor the CPU legs sample rows from, the step on a row sample, what
+    the sample is): the workload itself, or for the whole weight set its
+    first matrix (same distribution; the set is too large to draw on the
+    host)."""
+    if w.name.startswith(MODEL_WEIGHTS):
+        return (workloads.generate(workloads.model_matrix(0, 0)), lambda xs: _oracle_step(xs, False),
+                "its first matrix")
+    kind = LAYOUT_WORKLOADS.get(w.name)
+    if kind:
+        return workloads.generate(w), lambda xs: _oracle_layout_step(xs, kind), w.name
+    return workloads.generate(w), _oracle_step, w.name
 
 
 def cpu_baseline(w: workloads.Workload, budget_s: float = 15.0) -> dict:
     """The oracle as it stands (single-threaded C) on a bounded row sample of
-    the same workload, the same five steps; elements/s."""
+    the same workload, the same steps; elements/s."""
     import oracle
     oracle.build()
-    x = workloads.generate(w)
+    x, step, what = oracle_sample_source(w)
     xo = workloads.as_oracle_array(x)
-    rows = 4
+    R, C = xo.shape
+    rows = 32
     t0 = time.perf_counter()
-    _oracle_step(xo[:rows])
+    step(xo[:rows])
     t1 = time.perf_counter() - t0
-    rows = int(max(4, min(w.rows, rows * budget_s / max(t1, 1e-3) / 2)))
+    rows = int(max(4, min(R, rows * budget_s / max(t1, 1e-3) / 2)))
     t0 = time.perf_counter()
-    _oracle_step(xo[:rows])
+    step(np.ascontiguousarray(xo[:rows]))
     dt = time.perf_counter() - t0
-    return {"value": rows * w.cols / dt, "unit": "elements/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {rows} of {w.rows} rows ({rows * w.cols} elements), whole step, "
-                      f"{dt:.1f} s", "cpu": _cpu_model()}
+    return {"value": rows * C / dt, "unit": "elements/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {rows} of {R} rows ({rows * C} elements) of {what}, whole step, {dt:.1f} s",
+            "cpu": _cpu_model()}
 
 
 def _cpu_model() -> str:
@@ -433,29 +639,30 @@ def run_reference(args, rank: int, world: int):
     import oracle
     oracle.build()
     w = WORKLOADS[args.workload]
-    x = workloads.generate(w)
+    x, step, what = oracle_sample_source(w)
     xo = workloads.as_oracle_array(x)
+    R, C = xo.shape
     total_budget = 120.0
     t0 = time.perf_counter()
-    _oracle_step(xo[:2])
-    t_row = (time.perf_counter() - t0) / 2
+    step(np.ascontiguousarray(xo[:32]))
+    t_row = (time.perf_counter() - t0) / 32
     steps, warm = args.steps, max(args.warmup, 0)
-    rows = int(max(1, min(w.rows, total_budget / max(t_row, 1e-4) / (steps + warm))))
+    rows = int(max(1, min(R, total_budget / max(t_row, 1e-4) / (steps + warm))))
     for _ in range(warm):
-        _oracle_step(xo[:rows])
+        step(np.ascontiguousarray(xo[:rows]))
     t0 = time.perf_counter()
     for k in range(steps):
-        r0 = (k * rows) % max(1, w.rows - rows + 1)
-        _oracle_step(np.ascontiguousarray(xo[r0:r0 + rows]))
+        r0 = (k * rows) % max(1, R - rows + 1)
+        step(np.ascontiguousarray(xo[r0:r0 + rows]))
     dt = time.perf_counter() - t0
-    value = rows * w.cols * steps / dt
+    value = rows * C * steps / dt
     line = {
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": steps,
         "warmup": warm, "ms_per_step": dt / steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
         "config": {"workload": w.name, "description": w.description, "shape": [w.rows, w.cols]},
         "cpu_baseline": {"value": value, "unit": "elements/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{rows} rows x {w.cols} per step (bounded sample of the workload)",
+                         "sample": f"{rows} rows x {C} per step (bounded sample of {what})",
                          "cpu": _cpu_model()},
         "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

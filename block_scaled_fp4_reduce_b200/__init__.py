@@ -23,9 +23,10 @@ LIB_PATH = os.path.join(_PKG, "libfp4.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "fp4.h")
 
 # fp4_status / fp4_dtype / fp4_format values (include/fp4.h).
-OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_RANGE, ERR_WORKSPACE, ERR_CUDA = range(8)
+OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_RANGE, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(9)
 F32, BF16 = 0, 1
 NVFP4, MXFP4 = 0, 1
+MX_FLOOR, MX_CEIL = 0, 1
 
 _lib = None
 
@@ -63,6 +64,20 @@ def lib() -> ctypes.CDLL:
             "fp4_e2m1_round": (I, [P, P, I64, P]),
             "fp4_e2m1_roundtrip": (I, [P, P, I64, P]),
             "fp4_nv_encode_quotient": (I, [P, P, P, I64, P]),
+            "fp4_grouped_workspace_bytes": (SZ, [I]),
+            "fp4_nvfp4_quantize_grouped": (I, [P, I, I, P, SZ, P, P]),
+            "fp4_tensor_amax_grouped": (I, [P, I, I, P, SZ, P, P]),
+            "fp4_nvfp4_quantize_grouped_with_amax": (I, [P, I, I, P, P, P]),
+            "fp4_mxfp4_quantize_grouped": (I, [P, I, I, P, P]),
+            "fp4_mxfp4_quantize_ceil_grouped": (I, [P, I, I, P, P]),
+            "fp4_dequantize_grouped": (I, [I, P, I, I, P]),
+            "fp4_grouped_plan": (I, [P, I, I64, I, P, P, P, P, I]),
+            "fp4_set_launch_unit_limit": (I, [I64]),
+            "fp4_nvfp4_quantize_padded": (I, [P, I, I64, I64, P, P, P, P, SZ, P, P]),
+            "fp4_mxfp4_quantize_padded": (I, [P, I, I64, I64, I, P, P, P, P]),
+            "fp4_dequantize_padded": (I, [I, P, P, P, I64, I64, P, I, P]),
+            "fp4_nvfp4_quantize_columns": (I, [P, I, I64, I64, P, P, P, P, SZ, P, P]),
+            "fp4_mxfp4_quantize_columns": (I, [P, I, I64, I64, I, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -177,6 +192,99 @@ def fp4_scale_search_with_amax(x, amax, packed, scales, global_scale, block_loss
                                             _p(global_scale), _p(block_loss), _p(status), _stream(stream))
 
 
+class QuantItem(ctypes.Structure):
+    """struct fp4_quant_item (include/fp4.h)."""
+    _fields_ = [("x", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("global_scale", ctypes.c_void_p)]
+
+
+class DequantItem(ctypes.Structure):
+    """struct fp4_dequant_item (include/fp4.h)."""
+    _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("global_scale", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+def quant_items(xs, packed, scales, global_scales=None):
+    """A ctypes array of fp4_quant_item for matching lists of tensors."""
+    arr = (QuantItem * len(xs))()
+    for i, x in enumerate(xs):
+        R, C = _shape2(x)
+        arr[i] = QuantItem(_p(x), R, C, _p(packed[i]), _p(scales[i]),
+                           _p(global_scales[i]) if global_scales is not None else None)
+    return arr
+
+
+def dequant_items(qs, ys):
+    arr = (DequantItem * len(qs))()
+    for i, (q, y) in enumerate(zip(qs, ys)):
+        arr[i] = DequantItem(_p(q.packed), _p(q.scales), _p(q.global_scale), _p(y), q.rows, q.cols)
+    return arr
+
+
+def _group_dtype(xs) -> int:
+    codes = {_dtype_code(x) for x in xs}
+    if len(codes) > 1:
+        raise TypeError("all matrices of a grouped call share one dtype")
+    return codes.pop() if codes else BF16
+
+
+def fp4_nvfp4_quantize_grouped(items, dtype, workspace, status, stream=None) -> int:
+    return lib().fp4_nvfp4_quantize_grouped(ctypes.cast(items, ctypes.c_void_p), len(items), dtype,
+                                            _p(workspace), workspace.numel() * workspace.element_size(),
+                                            _p(status), _stream(stream))
+
+
+def fp4_tensor_amax_grouped(items, dtype, workspace, status, stream=None) -> int:
+    return lib().fp4_tensor_amax_grouped(ctypes.cast(items, ctypes.c_void_p), len(items), dtype,
+                                         _p(workspace), workspace.numel() * workspace.element_size(),
+                                         _p(status), _stream(stream))
+
+
+def fp4_nvfp4_quantize_grouped_with_amax(items, dtype, amax_words, status, stream=None) -> int:
+    return lib().fp4_nvfp4_quantize_grouped_with_amax(ctypes.cast(items, ctypes.c_void_p), len(items), dtype,
+                                                      _p(amax_words), _p(status), _stream(stream))
+
+
+def tensor_amax_grouped(xs, status=None, stream=None):
+    """Per-matrix amax of every matrix in xs: (fp32 [len(xs)] on the device,
+    status word)."""
+    dev = xs[0].device if xs else torch.device("cuda")
+    st = status if status is not None else new_status(dev)
+    ws = torch.empty(lib().fp4_grouped_workspace_bytes(len(xs)) // 4, dtype=torch.float32, device=dev)
+    items = quant_items(xs, [None] * len(xs), [None] * len(xs))
+    _check(fp4_tensor_amax_grouped(items, _group_dtype(xs), ws, st, stream), "fp4_tensor_amax_grouped")
+    return ws[:len(xs)], st
+
+
+def fp4_mxfp4_quantize_grouped(items, dtype, status, ceil=False, stream=None) -> int:
+    fn = lib().fp4_mxfp4_quantize_ceil_grouped if ceil else lib().fp4_mxfp4_quantize_grouped
+    return fn(ctypes.cast(items, ctypes.c_void_p), len(items), dtype, _p(status), _stream(stream))
+
+
+def fp4_dequantize_grouped(fmt, items, out_dtype, stream=None) -> int:
+    return lib().fp4_dequantize_grouped(fmt, ctypes.cast(items, ctypes.c_void_p), len(items), out_dtype,
+                                        _stream(stream))
+
+
+def grouped_plan(units, max_units, max_entries):
+    """The grouped calls' launch plan for items of `units` work units (host
+    only): a list of (launch, item, first unit, units) pieces."""
+    import numpy as np
+    n = len(units)
+    u = np.ascontiguousarray(units, dtype=np.int64)
+    cap = 2 * n + 16
+    while True:
+        lo, it = np.zeros(cap, np.int32), np.zeros(cap, np.int32)
+        fi, co = np.zeros(cap, np.int64), np.zeros(cap, np.int64)
+        k = lib().fp4_grouped_plan(u.ctypes.data if n else None, n, max_units, max_entries, lo.ctypes.data,
+                                   it.ctypes.data, fi.ctypes.data, co.ctypes.data, cap)
+        if k < 0:
+            raise ValueError("fp4_grouped_plan: invalid arguments")
+        if k <= cap:
+            return list(zip(lo[:k].tolist(), it[:k].tolist(), fi[:k].tolist(), co[:k].tolist()))
+        cap = k
+
+
 def fp4_e2m1_round(v, codes, stream=None) -> int:
     return lib().fp4_e2m1_round(_p(v), _p(codes), v.numel(), _stream(stream))
 
@@ -273,6 +381,116 @@ def dequantize(q: Quantized, out_dtype=torch.bfloat16, out=None, stream=None) ->
     _check(fp4_dequantize(q.fmt, q.packed, q.scales, q.global_scale, q.rows, q.cols, y, stream),
            "fp4_dequantize")
     return y
+
+
+def _padded(n: int, group: int) -> int:
+    return -(-n // group) * group
+
+
+def nvfp4_quantize_padded(x: torch.Tensor, workspace=None, status=None, stream=None) -> Quantized:
+    """NVFP4 of x [R, K] for any K: rows padded with +0 to whole 16-blocks
+    (packed [R, ceil(K/16)*8], scales [R, ceil(K/16)])."""
+    R, K = _shape2(x)
+    dev = x.device
+    Kp = _padded(K, 16)
+    packed = torch.empty((R, Kp // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((R, Kp // 16), dtype=torch.uint8, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else workspace_for(x)
+    st = status if status is not None else new_status(dev)
+    _check(lib().fp4_nvfp4_quantize_padded(_p(x), _dtype_code(x), R, K, _p(packed), _p(scales), _p(g), _p(ws),
+                                           ws.numel() * ws.element_size(), _p(st), _stream(stream)),
+           "fp4_nvfp4_quantize_padded")
+    return Quantized(NVFP4, packed, scales, g, st, R, K)
+
+
+def mxfp4_quantize_padded(x: torch.Tensor, rule: int = MX_FLOOR, status=None, stream=None) -> Quantized:
+    """MXFP4 of x [R, K] for any K: rows padded with +0 to whole 32-blocks."""
+    R, K = _shape2(x)
+    dev = x.device
+    Kp = _padded(K, 32)
+    packed = torch.empty((R, Kp // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((R, Kp // 32), dtype=torch.uint8, device=dev)
+    st = status if status is not None else new_status(dev)
+    _check(lib().fp4_mxfp4_quantize_padded(_p(x), _dtype_code(x), R, K, rule, _p(packed), _p(scales), _p(st),
+                                           _stream(stream)), "fp4_mxfp4_quantize_padded")
+    return Quantized(MXFP4, packed, scales, None, st, R, K)
+
+
+def dequantize_padded(q: Quantized, out_dtype=torch.bfloat16, out=None, stream=None) -> torch.Tensor:
+    """Dequantise a padded layout into the logical [q.rows, q.cols]."""
+    y = out if out is not None else torch.empty((q.rows, q.cols), dtype=out_dtype, device=q.packed.device)
+    _check(lib().fp4_dequantize_padded(q.fmt, _p(q.packed), _p(q.scales), _p(q.global_scale), q.rows, q.cols,
+                                       _p(y), _dtype_code(y), _stream(stream)), "fp4_dequantize_padded")
+    return y
+
+
+def nvfp4_quantize_columns(x: torch.Tensor, workspace=None, status=None, stream=None) -> Quantized:
+    """NVFP4 of W^T for x = W [R, C]: blocks down the columns of W; the
+    result describes the logical [C, R] transpose in the padded layout."""
+    R, C = _shape2(x)
+    dev = x.device
+    Rp = _padded(R, 16)
+    packed = torch.empty((C, Rp // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((C, Rp // 16), dtype=torch.uint8, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else workspace_for(x)
+    st = status if status is not None else new_status(dev)
+    _check(lib().fp4_nvfp4_quantize_columns(_p(x), _dtype_code(x), R, C, _p(packed), _p(scales), _p(g), _p(ws),
+                                            ws.numel() * ws.element_size(), _p(st), _stream(stream)),
+           "fp4_nvfp4_quantize_columns")
+    return Quantized(NVFP4, packed, scales, g, st, C, R)
+
+
+def mxfp4_quantize_columns(x: torch.Tensor, rule: int = MX_FLOOR, status=None, stream=None) -> Quantized:
+    """MXFP4 of W^T for x = W [R, C] (column-wise 32-blocks)."""
+    R, C = _shape2(x)
+    dev = x.device
+    Rp = _padded(R, 32)
+    packed = torch.empty((C, Rp // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((C, Rp // 32), dtype=torch.uint8, device=dev)
+    st = status if status is not None else new_status(dev)
+    _check(lib().fp4_mxfp4_quantize_columns(_p(x), _dtype_code(x), R, C, rule, _p(packed), _p(scales), _p(st),
+                                            _stream(stream)), "fp4_mxfp4_quantize_columns")
+    return Quantized(MXFP4, packed, scales, None, st, C, R)
+
+
+def nvfp4_quantize_grouped(xs, status=None, stream=None) -> list[Quantized]:
+    """NVFP4 quantisation of every matrix in xs, each with its own g, in a
+    few launches (bit-identical to nvfp4_quantize per matrix)."""
+    dev = xs[0].device if xs else torch.device("cuda")
+    outs = [(torch.empty((R, C // 2), dtype=torch.uint8, device=dev),
+             torch.empty((R, C // 16), dtype=torch.uint8, device=dev),
+             torch.empty(1, dtype=torch.float32, device=dev)) for R, C in map(_shape2, xs)]
+    st = status if status is not None else new_status(dev)
+    ws = torch.empty(lib().fp4_grouped_workspace_bytes(len(xs)), dtype=torch.uint8, device=dev)
+    items = quant_items(xs, [o[0] for o in outs], [o[1] for o in outs], [o[2] for o in outs])
+    _check(fp4_nvfp4_quantize_grouped(items, _group_dtype(xs), ws, st, stream), "fp4_nvfp4_quantize_grouped")
+    return [Quantized(NVFP4, p, s, g, st, *_shape2(x)) for x, (p, s, g) in zip(xs, outs)]
+
+
+def mxfp4_quantize_grouped(xs, ceil: bool = False, status=None, stream=None) -> list[Quantized]:
+    """MXFP4 quantisation of every matrix in xs in a few launches."""
+    dev = xs[0].device if xs else torch.device("cuda")
+    outs = [(torch.empty((R, C // 2), dtype=torch.uint8, device=dev),
+             torch.empty((R, C // 32), dtype=torch.uint8, device=dev)) for R, C in map(_shape2, xs)]
+    st = status if status is not None else new_status(dev)
+    items = quant_items(xs, [o[0] for o in outs], [o[1] for o in outs])
+    _check(fp4_mxfp4_quantize_grouped(items, _group_dtype(xs), st, ceil, stream), "fp4_mxfp4_quantize_grouped")
+    return [Quantized(MXFP4, p, s, None, st, *_shape2(x)) for x, (p, s) in zip(xs, outs)]
+
+
+def dequantize_grouped(qs, out_dtype=torch.bfloat16, outs=None, stream=None) -> list[torch.Tensor]:
+    """Dequantise every Quantized in qs (all NVFP4 or all MXFP4)."""
+    fmts = {q.fmt for q in qs}
+    if len(fmts) > 1:
+        raise ValueError("all items of a grouped dequantisation share one format")
+    ys = outs if outs is not None else [
+        torch.empty((q.rows, q.cols), dtype=out_dtype, device=q.packed.device) for q in qs]
+    code = _dtype_code(ys[0]) if ys else (F32 if out_dtype == torch.float32 else BF16)
+    _check(fp4_dequantize_grouped(fmts.pop() if fmts else NVFP4, dequant_items(qs, ys), code, stream),
+           "fp4_dequantize_grouped")
+    return ys
 
 
 def scale_search(x: torch.Tensor, with_loss: bool = True, workspace=None, status=None, stream=None) -> Quantized:

@@ -5,92 +5,23 @@
 // synchronises; every launch goes on the caller's stream.
 #include <climits>
 #include <cstdint>
+#include <type_traits>
 
 #include <cuda_runtime.h>
 
 #include "fp4.h"
 #include "fp4_kernels.cuh"
+#include "fp4_launch.cuh"
+
+namespace fp4_launch {
+int64_t g_launch_unit_limit = fp4::kMaxUnitsPerLaunch;
+}
 
 namespace {
 
+using namespace fp4_launch;
 using fp4::kMaxPartials;
 using fp4::kThreads;
-
-constexpr int kMaxDevices = 64;
-
-bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-
-// SM count of the current device (cached per device).
-int sm_count(int &dev)
-{
-    static int cache[kMaxDevices] = {0};
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
-        return -1;
-    if (dev < kMaxDevices && cache[dev] > 0)
-        return cache[dev];
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-        return -1;
-    if (dev < kMaxDevices)
-        cache[dev] = n;
-    return n;
-}
-
-// Resident CTAs per SM of `kernel` at kThreads threads (cached per device
-// and kernel instantiation).
-template <typename K> int resident_ctas(K kernel, int dev)
-{
-    static int cache[kMaxDevices] = {0};
-    if (dev < kMaxDevices && cache[dev] > 0)
-        return cache[dev];
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, 0) != cudaSuccess ||
-        n <= 0)
-        n = 1;
-    if (dev < kMaxDevices)
-        cache[dev] = n;
-    return n;
-}
-
-// Persistent grid: enough CTAs for `work` items at `per_cta` items each,
-// at most SMs x resident CTAs, at least one.
-template <typename K> int grid_for(K kernel, int64_t work, int64_t per_cta)
-{
-    int dev = 0;
-    const int sms = sm_count(dev);
-    if (sms <= 0)
-        return -1;
-    const int64_t cap = (int64_t)sms * resident_ctas(kernel, dev);
-    int64_t want = (work + per_cta - 1) / per_cta;
-    if (want < 1)
-        want = 1;
-    return (int)(want < cap ? want : cap);
-}
-
-// Launch with programmatic stream serialisation: the kernel may start while
-// the previous kernel on the stream finishes; it waits for it
-// (griddepcontrol.wait) before touching memory.
-template <typename... KArgs, typename... Args>
-fp4_status launch(void (*kernel)(KArgs...), int grid, cudaStream_t stream, Args... args)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return FP4_ERR_CUDA;
-    }
-    return FP4_OK;
-}
-
-bool valid_dtype(fp4_dtype t) { return t == FP4_F32 || t == FP4_BF16; }
 
 // rows, cols >= 0, cols % block == 0, rows * cols representable.
 fp4_status check_shape(int64_t rows, int64_t cols, int64_t block)
@@ -104,10 +35,6 @@ fp4_status check_shape(int64_t rows, int64_t cols, int64_t block)
     return FP4_OK;
 }
 
-// Workspace words: kMaxPartials per-CTA maxima, the wrapping CTA counter,
-// and the amax word the NVFP4 quantiser and the search read.
-constexpr size_t kWsAmax = kMaxPartials + 1; // kMaxPartials holds the counter
-constexpr size_t kWsWords = kMaxPartials + 8;
 
 // Tensor amax (one launch) into *amax.
 fp4_status launch_amax(const void *x, fp4_dtype dt, int64_t n, uint32_t *ws, float *amax,
@@ -132,26 +59,30 @@ fp4_status launch_amax(const void *x, fp4_dtype dt, int64_t n, uint32_t *ws, flo
                   status);
 }
 
+template <typename T>
+fp4_status launch_nv_quantize_t(const T *x, int64_t n, const float *amax, uint8_t *packed,
+                                uint8_t *scales, float *global_scale, int32_t *status,
+                                cudaStream_t stream)
+{
+    uint2 *pk = reinterpret_cast<uint2 *>(packed);
+    return for_chunks(n / 16, [&](int64_t first, int count) {
+        const int grid = grid_for(fp4::nvfp4_quantize_kernel<T>, count, (int64_t)kThreads * 2);
+        if (grid <= 0)
+            return FP4_ERR_CUDA;
+        return launch(fp4::nvfp4_quantize_kernel<T>, grid, stream, x + first * 16, count, amax,
+                      pk + first, scales + first, global_scale, status);
+    });
+}
+
 fp4_status launch_nv_quantize(const void *x, fp4_dtype dt, int64_t n, const float *amax,
                               uint8_t *packed, uint8_t *scales, float *global_scale,
                               int32_t *status, cudaStream_t stream)
 {
-    const int64_t n_blocks = n / 16;
-    const int64_t per_cta = (int64_t)kThreads * 2;
-    int grid;
     if (dt == FP4_BF16)
-        grid = grid_for(fp4::nvfp4_quantize_kernel<uint16_t>, n_blocks, per_cta);
-    else
-        grid = grid_for(fp4::nvfp4_quantize_kernel<float>, n_blocks, per_cta);
-    if (grid <= 0)
-        return FP4_ERR_CUDA;
-    uint2 *pk = reinterpret_cast<uint2 *>(packed);
-    if (dt == FP4_BF16)
-        return launch(fp4::nvfp4_quantize_kernel<uint16_t>, grid, stream,
-                      static_cast<const uint16_t *>(x), n_blocks, amax, pk, scales, global_scale,
-                      status);
-    return launch(fp4::nvfp4_quantize_kernel<float>, grid, stream, static_cast<const float *>(x),
-                  n_blocks, amax, pk, scales, global_scale, status);
+        return launch_nv_quantize_t(static_cast<const uint16_t *>(x), n, amax, packed, scales,
+                                    global_scale, status, stream);
+    return launch_nv_quantize_t(static_cast<const float *>(x), n, amax, packed, scales,
+                                global_scale, status, stream);
 }
 
 } // namespace
@@ -174,21 +105,51 @@ fp4_status mxfp4_quantize_rule(const void *x, fp4_dtype dtype, int64_t rows, int
         return FP4_ERR_INVALID_ARG;
     if (!aligned(x, 32) || !aligned(packed, 16))
         return FP4_ERR_ALIGN;
-    const int64_t n_blocks = n / 32;
-    const int64_t per_cta = (int64_t)kThreads * 2;
     uint4 *pk = reinterpret_cast<uint4 *>(packed);
-    if (dtype == FP4_BF16) {
-        const int grid = grid_for(fp4::mxfp4_quantize_kernel<uint16_t, kCeil>, n_blocks, per_cta);
+    auto run = [&](auto *xt) {
+        using T = std::remove_const_t<std::remove_pointer_t<decltype(xt)>>;
+        return for_chunks(n / 32, [&](int64_t first, int count) {
+            const int grid =
+                grid_for(fp4::mxfp4_quantize_kernel<T, kCeil>, count, (int64_t)kThreads * 2);
+            if (grid <= 0)
+                return FP4_ERR_CUDA;
+            return launch(fp4::mxfp4_quantize_kernel<T, kCeil>, grid, stream, xt + first * 32,
+                          count, pk + first, scales + first, status);
+        });
+    };
+    if (dtype == FP4_BF16)
+        return run(static_cast<const uint16_t *>(x));
+    return run(static_cast<const float *>(x));
+}
+} // namespace
+
+namespace {
+template <typename K, typename T>
+fp4_status launch_block_kernel(K kernel, const T *x, int64_t n, const float *amax,
+                               uint8_t *packed, uint8_t *scales, float *global_scale,
+                               float *block_loss, int32_t *status, cudaStream_t stream)
+{
+    uint2 *pk = reinterpret_cast<uint2 *>(packed);
+    return for_chunks(n / 16, [&](int64_t first, int count) {
+        const int grid = grid_for(kernel, count, kThreads);
         if (grid <= 0)
             return FP4_ERR_CUDA;
-        return launch(fp4::mxfp4_quantize_kernel<uint16_t, kCeil>, grid, stream,
-                      static_cast<const uint16_t *>(x), n_blocks, pk, scales, status);
-    }
-    const int grid = grid_for(fp4::mxfp4_quantize_kernel<float, kCeil>, n_blocks, per_cta);
-    if (grid <= 0)
-        return FP4_ERR_CUDA;
-    return launch(fp4::mxfp4_quantize_kernel<float, kCeil>, grid, stream,
-                  static_cast<const float *>(x), n_blocks, pk, scales, status);
+        return launch(kernel, grid, stream, x + first * 16, count, amax, pk + first,
+                      scales + first, global_scale, block_loss ? block_loss + first : block_loss,
+                      status);
+    });
+}
+
+fp4_status launch_search(const void *x, fp4_dtype dtype, int64_t n, const float *amax,
+                         uint8_t *packed, uint8_t *scales, float *global_scale,
+                         float *block_loss, int32_t *status, cudaStream_t stream)
+{
+    if (dtype == FP4_BF16)
+        return launch_block_kernel(fp4::scale_search_kernel<uint16_t>,
+                                   static_cast<const uint16_t *>(x), n, amax, packed, scales,
+                                   global_scale, block_loss, status, stream);
+    return launch_block_kernel(fp4::scale_search_kernel<float>, static_cast<const float *>(x), n,
+                               amax, packed, scales, global_scale, block_loss, status, stream);
 }
 } // namespace
 
@@ -205,11 +166,22 @@ const char *fp4_status_string(int status)
     case FP4_ERR_RANGE: return "global scale out of range";
     case FP4_ERR_WORKSPACE: return "workspace missing or too small";
     case FP4_ERR_CUDA: return "CUDA launch failure";
+    case FP4_ERR_TIMEOUT: return "a bounded device wait ran out";
     default: return "unknown status";
     }
 }
 
 int fp4_version(void) { return 100; }
+
+fp4_status fp4_set_launch_unit_limit(int64_t units)
+{
+    if (units == 0)
+        units = fp4::kMaxUnitsPerLaunch;
+    if (units < 64 || units > fp4::kMaxUnitsPerLaunch || units % 64)
+        return FP4_ERR_INVALID_ARG;
+    fp4_launch::g_launch_unit_limit = units;
+    return FP4_OK;
+}
 
 size_t fp4_workspace_bytes(fp4_format fmt, int64_t rows, int64_t cols)
 {
@@ -308,52 +280,25 @@ fp4_status fp4_dequantize(fp4_format fmt, const uint8_t *packed, const uint8_t *
         return FP4_ERR_INVALID_ARG;
     if (!aligned(packed, 16) || !aligned(y, 32) || (nv && !aligned(global_scale, 4)))
         return FP4_ERR_ALIGN;
-    const int64_t n_units = n / 16;
-    const int64_t per_cta = (int64_t)kThreads * 2;
     const uint2 *pk = reinterpret_cast<const uint2 *>(packed);
-#define FP4_DEQ_LAUNCH(NV, TOUT)                                                                \
-    do {                                                                                        \
-        const int grid = grid_for(fp4::dequantize_kernel<NV, TOUT>, n_units, per_cta);          \
-        if (grid <= 0)                                                                          \
-            return FP4_ERR_CUDA;                                                                \
-        return launch(fp4::dequantize_kernel<NV, TOUT>, grid, stream, pk, scales, global_scale, \
-                      n_units, static_cast<TOUT *>(y));                                         \
-    } while (0)
+    auto run = [&](auto kernel, auto *yt) {
+        return for_chunks(n / 16, [&](int64_t first, int count) {
+            const int grid = grid_for(kernel, count, (int64_t)kThreads * 4);
+            if (grid <= 0)
+                return FP4_ERR_CUDA;
+            return launch(kernel, grid, stream, pk + first, scales + (nv ? first : first / 2),
+                          global_scale, count, yt + first * 16);
+        });
+    };
     if (nv && out_dtype == FP4_BF16)
-        FP4_DEQ_LAUNCH(true, uint16_t);
-    else if (nv)
-        FP4_DEQ_LAUNCH(true, float);
-    else if (out_dtype == FP4_BF16)
-        FP4_DEQ_LAUNCH(false, uint16_t);
-    else
-        FP4_DEQ_LAUNCH(false, float);
-#undef FP4_DEQ_LAUNCH
+        return run(fp4::dequantize_kernel<true, uint16_t>, static_cast<uint16_t *>(y));
+    if (nv)
+        return run(fp4::dequantize_kernel<true, float>, static_cast<float *>(y));
+    if (out_dtype == FP4_BF16)
+        return run(fp4::dequantize_kernel<false, uint16_t>, static_cast<uint16_t *>(y));
+    return run(fp4::dequantize_kernel<false, float>, static_cast<float *>(y));
 }
 
-namespace {
-fp4_status launch_search(const void *x, fp4_dtype dtype, int64_t n, const float *amax,
-                         uint8_t *packed, uint8_t *scales, float *global_scale,
-                         float *block_loss, int32_t *status, cudaStream_t stream)
-{
-    const int64_t n_blocks = n / 16;
-    uint2 *pk = reinterpret_cast<uint2 *>(packed);
-    if (dtype == FP4_BF16) {
-        const int grid = grid_for(fp4::scale_search_kernel<uint16_t>, n_blocks, kThreads);
-        if (grid <= 0)
-            return FP4_ERR_CUDA;
-        return launch(fp4::scale_search_kernel<uint16_t>, grid, stream,
-                      static_cast<const uint16_t *>(x), n_blocks, amax, pk, scales, global_scale,
-                      block_loss, status);
-    } else {
-        const int grid = grid_for(fp4::scale_search_kernel<float>, n_blocks, kThreads);
-        if (grid <= 0)
-            return FP4_ERR_CUDA;
-        return launch(fp4::scale_search_kernel<float>, grid, stream,
-                      static_cast<const float *>(x), n_blocks, amax, pk, scales, global_scale,
-                      block_loss, status);
-    }
-}
-} // namespace
 
 fp4_status fp4_scale_search(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
                             uint8_t *packed, uint8_t *scales, float *global_scale,
@@ -425,22 +370,13 @@ fp4_status fp4_nvfp4_quantize_four_over_six(const void *x, fp4_dtype dtype, int6
     st = launch_amax(x, dtype, n, ws, amax, status, stream);
     if (st != FP4_OK)
         return st;
-    const int64_t n_blocks = n / 16;
-    uint2 *pk = reinterpret_cast<uint2 *>(packed);
-    if (dtype == FP4_BF16) {
-        const int grid = grid_for(fp4::nvfp4_four_over_six_kernel<uint16_t>, n_blocks, kThreads);
-        if (grid <= 0)
-            return FP4_ERR_CUDA;
-        return launch(fp4::nvfp4_four_over_six_kernel<uint16_t>, grid, stream,
-                      static_cast<const uint16_t *>(x), n_blocks, static_cast<const float *>(amax),
-                      pk, scales, global_scale, block_loss, status);
-    }
-    const int grid = grid_for(fp4::nvfp4_four_over_six_kernel<float>, n_blocks, kThreads);
-    if (grid <= 0)
-        return FP4_ERR_CUDA;
-    return launch(fp4::nvfp4_four_over_six_kernel<float>, grid, stream,
-                  static_cast<const float *>(x), n_blocks, static_cast<const float *>(amax), pk,
-                  scales, global_scale, block_loss, status);
+    if (dtype == FP4_BF16)
+        return launch_block_kernel(fp4::nvfp4_four_over_six_kernel<uint16_t>,
+                                   static_cast<const uint16_t *>(x), n, amax, packed, scales,
+                                   global_scale, block_loss, status, stream);
+    return launch_block_kernel(fp4::nvfp4_four_over_six_kernel<float>,
+                               static_cast<const float *>(x), n, amax, packed, scales,
+                               global_scale, block_loss, status, stream);
 }
 
 fp4_status fp4_e2m1_round(const float *v, uint8_t *codes, int64_t n, cudaStream_t stream)

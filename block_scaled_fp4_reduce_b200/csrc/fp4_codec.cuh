@@ -116,6 +116,37 @@ __device__ __forceinline__ void e2m1x8_qdq(const float (&v)[8], float (&p)[8])
     }
 }
 
+// Rounding error of eight fp32 values on the E2M1 grid: e[i] = p_i - v[i]
+// (p_i the grid value of v[i]), each pair rounded to codes, widened to f16
+// and subtracted from the fp32 value by the mixed-precision
+// `sub.rn.f32.f16` (sm_100) inside one asm block.  One rounding per
+// element, so |e| is the magnitude of the correctly rounded v - p.
+__device__ __forceinline__ void e2m1x8_error(const float (&v)[8], float (&e)[8])
+{
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        asm("{\n\t"
+            ".reg .b8 q;\n\t"
+            ".reg .b32 h;\n\t"
+            ".reg .b16 l, u;\n\t"
+            "cvt.rn.satfinite.e2m1x2.f32 q, %3, %2;\n\t"
+            "cvt.rn.f16x2.e2m1x2 h, q;\n\t"
+            "mov.b32 {l, u}, h;\n\t"
+            "sub.rn.f32.f16 %0, l, %2;\n\t"
+            "sub.rn.f32.f16 %1, u, %3;\n\t"
+            "}"
+            : "=f"(e[2 * j]), "=f"(e[2 * j + 1])
+            : "f"(v[2 * j]), "f"(v[2 * j + 1]));
+}
+
+// sqrt.approx.f32: relative error below 2^-21 (for bounds only).
+__device__ __forceinline__ float sqrt_approx(float x)
+{
+    float r;
+    asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // ---------------------------------------------------------------------------
 // E4M3 (FN) block scale.
 // ---------------------------------------------------------------------------
@@ -176,13 +207,45 @@ __device__ __forceinline__ uint32_t nv_scale_code(float amax_b, float inv, doubl
     return (uint32_t)(c & 0xFFu);
 }
 
-// Value of a positive E4M3 code 0..126: codes >= 8 are normal, exponent
-// field e = c / 8 and fraction f = c % 8 give the fp32 pattern
-// (e + 120) << 23 | f << 20 = (c << 20) + (120 << 23); codes below 8 are
-// the subnormals c * 2^-9.
+// Value of an E4M3 byte as f16 bits: every E4M3 value (2^-9 .. 448, NaN)
+// is exact in f16.
+__device__ __forceinline__ uint16_t e4m3_to_f16(uint32_t byte)
+{
+    uint16_t r;
+    const uint16_t b = (uint16_t)(byte & 0xFFu);
+    asm("{\n\t"
+        ".reg .b32 h;\n\t"
+        ".reg .b16 u;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h, %1;\n\t"
+        "mov.b32 {%0, u}, h;\n\t"
+        "}"
+        : "=h"(r)
+        : "h"(b));
+    return r;
+}
+
+// Value of a positive E4M3 code 0..126 as fp32 (exact): the E4M3 -> f16
+// conversion, then f16 -> fp32.
 __device__ __forceinline__ float e4m3_pos_to_f32(uint32_t c)
 {
-    return c >= 8u ? __uint_as_float((c << 20) + 0x3C000000u) : (float)c * 0x1p-9f;
+    float r;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(r) : "h"(e4m3_to_f16(c)));
+    return r;
+}
+
+// The two f16 halves of h, each times the f16 s, as fp32 with one rounding
+// (mixed-precision `fma.rn.f32.f16`, sm_100): a * s + (-0).  Adding -0 keeps
+// the sign of a zero product and changes nothing else.
+__device__ __forceinline__ void f16x2_mul_f16_to_f32(uint32_t h, uint16_t s, float &lo, float &hi)
+{
+    asm("{\n\t"
+        ".reg .b16 l, u;\n\t"
+        "mov.b32 {l, u}, %2;\n\t"
+        "fma.rn.f32.f16 %0, l, %3, 0f80000000;\n\t"
+        "fma.rn.f32.f16 %1, u, %3, 0f80000000;\n\t"
+        "}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h), "h"(s));
 }
 
 // ---------------------------------------------------------------------------
@@ -222,6 +285,15 @@ __device__ __forceinline__ uint32_t e8m0_byte_ceil(uint32_t amax_bits)
 __device__ __forceinline__ float e8m0_inverse(uint32_t byte)
 {
     return __uint_as_float((254u - byte) << 23);
+}
+
+// 2^e as f16 bits for an E8M0 byte b = e + 127 with -24 <= e <= 15:
+// normal 2^e (e >= -14) has exponent field e + 15; below that the
+// subnormal 2^e = 2^(e + 24) units of 2^-24.
+__device__ __forceinline__ uint16_t e8m0_to_f16(uint32_t byte)
+{
+    const int e = (int)byte - 127;
+    return e >= -14 ? (uint16_t)((e + 15) << 10) : (uint16_t)(1u << (e + 24));
 }
 
 // 2^e as fp32 for any E8M0 byte: 0 -> 2^-127 (subnormal), 255 -> NaN.
@@ -281,13 +353,50 @@ __device__ __forceinline__ NvRecip nv_recip(float d)
     return q;
 }
 
+// Packed fp32 pairs (sm_100): two IEEE single operations, each rounded to
+// nearest, per instruction.  pack2 / unpack2 only name a register pair.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi)
+{
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t d, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+}
+
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t nv_encode8(const float (&x)[8], const NvRecip &q)
 {
     float a[8], b[8];
+    const uint64_t rlo = pack2(q.lo, q.lo), rhi = pack2(q.hi, q.hi);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        a[i] = __fmul_rn(x[i], q.lo);
-        b[i] = __fmul_rn(x[i], q.hi);
+    for (int j = 0; j < 4; ++j) {
+        const uint64_t xp = pack2(x[2 * j], x[2 * j + 1]);
+        unpack2(mul2(xp, rlo), a[2 * j], a[2 * j + 1]);
+        unpack2(mul2(xp, rhi), b[2 * j], b[2 * j + 1]);
     }
     uint32_t ca = e2m1x8(a);
     const uint32_t cb = e2m1x8(b);

@@ -76,67 +76,47 @@ template <typename T, int N> struct Blk {
     uint32_t w[kWords];
 };
 
-template <typename T, int N>
-__device__ __forceinline__ void load_blk(const T *x, int64_t b, Blk<T, N> &k)
+template <typename T, int N, typename I>
+__device__ __forceinline__ void load_blk(const T *x, I b, Blk<T, N> &k)
 {
-    const char *p = reinterpret_cast<const char *>(x) + b * (int64_t)(N * sizeof(T));
+    const char *p = reinterpret_cast<const char *>(x) + (int64_t)b * (int64_t)(N * sizeof(T));
 #pragma unroll
     for (int j = 0; j < Blk<T, N>::kWords; j += 8)
         ldg_v8(p + 4 * j, &k.w[j]);
 }
 
-// max |x| over the block as an fp32 bit pattern.  Non-negative floats order
-// like their bit patterns; NaN / Inf patterns sort above every finite value.
+// max |x| over the block as an fp32 bit pattern, with packed
+// `max.NaN.xorsign.abs` (sm_86+): the magnitude of the result is the larger
+// magnitude, its sign is garbage and masked off at the end; a NaN operand
+// makes the result NaN.  bf16 pairs take one instruction per two elements.
+// Finite values order like their bit patterns, and NaN / Inf patterns sort
+// above every finite value.
 template <typename T, int N>
 __device__ __forceinline__ uint32_t absmax_bits(const Blk<T, N> &k)
 {
     constexpr int W = Blk<T, N>::kWords;
     uint32_t m[W];
+#pragma unroll
+    for (int j = 0; j < W; ++j)
+        m[j] = k.w[j];
     if constexpr (sizeof(T) == 2) {
 #pragma unroll
-        for (int j = 0; j < W; ++j)
-            m[j] = k.w[j] & 0x7FFF7FFFu;
-#pragma unroll
         for (int s = W / 2; s >= 1; s /= 2)
 #pragma unroll
             for (int j = 0; j < s; ++j)
-                m[j] = __vmaxu2(m[j], m[j + s]);
-        return max(m[0] & 0xFFFFu, m[0] >> 16) << 16;
-    } else {
-#pragma unroll
-        for (int j = 0; j < W; ++j)
-            m[j] = k.w[j] & 0x7FFFFFFFu;
-#pragma unroll
-        for (int s = W / 2; s >= 1; s /= 2)
-#pragma unroll
-            for (int j = 0; j < s; ++j)
-                m[j] = max(m[j], m[j + s]);
-        return m[0];
-    }
-}
-
-// max |x| over a block known to be finite, as an fp32 bit pattern: bf16
-// pairs go through packed `max.bf16x2` on absolute values (two elements per
-// instruction); fp32 through the integer path above.
-template <typename T, int N>
-__device__ __forceinline__ uint32_t absmax_bits_finite(const Blk<T, N> &k)
-{
-    if constexpr (sizeof(T) == 2) {
-        constexpr int W = Blk<T, N>::kWords;
-        uint32_t m[W];
-#pragma unroll
-        for (int j = 0; j < W; ++j)
-            m[j] = k.w[j] & 0x7FFF7FFFu;
-#pragma unroll
-        for (int s = W / 2; s >= 1; s /= 2)
-#pragma unroll
-            for (int j = 0; j < s; ++j)
-                asm("max.bf16x2 %0, %1, %2;" : "=r"(m[j]) : "r"(m[j]), "r"(m[j + s]));
+                asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m[j]) : "r"(m[j]), "r"(m[j + s]));
         uint32_t r;
-        asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(m[0]), "r"(__funnelshift_l(m[0], m[0], 16)));
-        return r << 16;
+        asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;"
+            : "=r"(r)
+            : "r"(m[0]), "r"(__funnelshift_l(m[0], m[0], 16)));
+        return r & 0x7FFF0000u;
     } else {
-        return absmax_bits(k);
+#pragma unroll
+        for (int s = W / 2; s >= 1; s /= 2)
+#pragma unroll
+            for (int j = 0; j < s; ++j)
+                asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=r"(m[j]) : "r"(m[j]), "r"(m[j + s]));
+        return m[0] & 0x7FFFFFFFu;
     }
 }
 
@@ -157,6 +137,65 @@ __device__ __forceinline__ void elems8(const Blk<T, N> &k, int first, float (&x)
     for (int i = 0; i < 8; ++i)
         x[i] = elem(k, first + i);
 }
+
+// Grid-stride loop over n units with U units in flight per thread: `load(u,
+// i)` for all U units first, then `work(u, i)`, so that U loads are
+// outstanding together.  The main loop runs unguarded over whole groups of
+// U; the remaining units go one at a time.  Indices are 32-bit (the host
+// splits larger problems into chunks below 2^30 units), so every address is
+// one wide multiply-add.
+template <int U, typename Load, typename Work>
+__device__ __forceinline__ void stream_units(int n, Load &&load, Work &&work)
+{
+    const int stride = (int)(gridDim.x * blockDim.x);
+    int i = (int)(blockIdx.x * blockDim.x + threadIdx.x);
+    for (; i + (U - 1) * stride < n; i += U * stride) {
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            load(u, i + u * stride);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            work(u, i + u * stride);
+    }
+    for (; i < n; i += stride) {
+        load(0, i);
+        work(0, i);
+    }
+}
+
+// The same with a blocked distribution: CTA c takes one contiguous range of
+// units (whole tiles of blockDim * U consecutive units), and within a tile
+// consecutive threads take consecutive units.  A thread's units then lie in
+// one short stretch of the unit space (used where per-stretch state, such as
+// the matrix of a grouped launch, is costly to switch).
+template <int U, typename Load, typename Work>
+__device__ __forceinline__ void stream_units_blocked(int n, Load &&load, Work &&work)
+{
+    const int tile = (int)blockDim.x * U;
+    const int tiles = (n + tile - 1) / tile;
+    const int per_cta = (tiles + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int t0 = (int)blockIdx.x * per_cta;
+    const int t1 = min(t0 + per_cta, tiles);
+    for (int t = t0; t < t1; ++t) {
+        const int base = t * tile + (int)threadIdx.x;
+        if (base + (U - 1) * (int)blockDim.x < n) {
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                load(u, base + u * (int)blockDim.x);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                work(u, base + u * (int)blockDim.x);
+        } else {
+            for (int i = base; i < n; i += (int)blockDim.x) {
+                load(0, i);
+                work(0, i);
+            }
+        }
+    }
+}
+
+// Largest unit count one launch of a stream_units kernel takes.
+constexpr int64_t kMaxUnitsPerLaunch = (int64_t)1 << 30;
 
 __device__ __forceinline__ void pdl_begin()
 {
@@ -302,9 +341,21 @@ __device__ __forceinline__ uint2 nv_block_codes(const Blk<T, 16> &b, uint32_t c,
 // NVFP4 quantise + pack.  One thread per 16-element block: one 32-byte load
 // (bf16) or two (fp32), one 8-byte packed store, one scale byte.
 // ---------------------------------------------------------------------------
+// NVFP4 codes and scale byte of one loaded 16-block under the global scale
+// g (constants sc): written to *packed / *scale.
+template <typename T>
+__device__ __forceinline__ void nv_quantize_block(const Blk<T, 16> &blk, const NvScaleConsts &sc,
+                                                  uint2 *packed, uint8_t *scale)
+{
+    const float amax_b = __uint_as_float(absmax_bits(blk));
+    const uint32_t code = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
+    *packed = nv_block_codes(blk, code, sc.g);
+    *scale = (uint8_t)code;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-    nvfp4_quantize_kernel(const T *__restrict__ x, int64_t n_blocks, const float *amax,
+    nvfp4_quantize_kernel(const T *__restrict__ x, int n_blocks, const float *amax,
                           uint2 *__restrict__ packed, uint8_t *__restrict__ scales,
                           float *global_scale, int32_t *status)
 {
@@ -313,135 +364,160 @@ __global__ void __launch_bounds__(kThreads)
     if (!nv_prologue(amax, global_scale, status, g))
         return;
     const NvScaleConsts sc = nv_scale_consts(g);
-    constexpr int kUnroll = 2;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b0 < n_blocks;
-         b0 += kUnroll * stride) {
-        Blk<T, 16> blk[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-            if (b0 + u * stride < n_blocks)
-                load_blk(x, b0 + u * stride, blk[u]);
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t b = b0 + u * stride;
-            if (b < n_blocks) {
-                const float amax_b = __uint_as_float(absmax_bits_finite(blk[u]));
-                const uint32_t code = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
-                packed[b] = nv_block_codes(blk[u], code, g);
-                scales[b] = (uint8_t)code;
-            }
-        }
-    }
+    Blk<T, 16> blk[4];
+    stream_units<4>(
+        n_blocks, [&](int u, int b) { load_blk(x, b, blk[u]); },
+        [&](int u, int b) { nv_quantize_block(blk[u], sc, packed + b, scales + b); });
 }
 
 // ---------------------------------------------------------------------------
 // MXFP4 quantise + pack.  One thread per 32-element block: two 32-byte loads
 // (bf16) or four (fp32), one 16-byte packed store, one scale byte.  kCeil
-// selects the ceil scale rule instead of the OCP rounding-down one.
+// selects the ceil scale rule instead of the OCP rounding-down one.  The
+// scaling x 2^-e is exact, so it runs as packed pair multiplies.  A block
+// with a NaN or Inf sets *bad.
 // ---------------------------------------------------------------------------
+template <bool kCeil, typename T>
+__device__ __forceinline__ void mx_quantize_block(const Blk<T, 32> &blk, uint4 *packed,
+                                                  uint8_t *scale, bool &bad)
+{
+    const uint32_t ab = absmax_bits(blk);
+    bad |= ab >= kNonFiniteBits;
+    const uint32_t byte = kCeil ? e8m0_byte_ceil(ab) : e8m0_byte_floor(ab);
+    const float inv = e8m0_inverse(byte);
+    const uint64_t inv2 = pack2(inv, inv);
+    uint32_t pk[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            unpack2(mul2(pack2(elem(blk, 8 * j + 2 * i), elem(blk, 8 * j + 2 * i + 1)), inv2),
+                    v[2 * i], v[2 * i + 1]);
+        pk[j] = e2m1x8(v);
+    }
+    *packed = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *scale = (uint8_t)byte;
+}
+
 template <typename T, bool kCeil = false>
 __global__ void __launch_bounds__(kThreads)
-    mxfp4_quantize_kernel(const T *__restrict__ x, int64_t n_blocks,
-                          uint4 *__restrict__ packed, uint8_t *__restrict__ scales,
-                          int32_t *status)
+    mxfp4_quantize_kernel(const T *__restrict__ x, int n_blocks, uint4 *__restrict__ packed,
+                          uint8_t *__restrict__ scales, int32_t *status)
 {
     pdl_begin();
-    constexpr int kUnroll = 2;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     bool bad = false;
-    for (int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b0 < n_blocks;
-         b0 += kUnroll * stride) {
-        Blk<T, 32> blk[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-            if (b0 + u * stride < n_blocks)
-                load_blk(x, b0 + u * stride, blk[u]);
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t b = b0 + u * stride;
-            if (b < n_blocks) {
-                const uint32_t ab = absmax_bits(blk[u]);
-                bad |= ab >= kNonFiniteBits;
-                const uint32_t byte = kCeil ? e8m0_byte_ceil(ab) : e8m0_byte_floor(ab);
-                const float inv = e8m0_inverse(byte);
-                uint32_t pk[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float v[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        v[i] = __fmul_rn(elem(blk[u], 8 * j + i), inv); // exact: 2^-e
-                    pk[j] = e2m1x8(v);
-                }
-                packed[b] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                scales[b] = (uint8_t)byte;
-            }
-        }
-    }
+    Blk<T, 32> blk[2];
+    stream_units<2>(
+        n_blocks, [&](int u, int b) { load_blk(x, b, blk[u]); },
+        [&](int u, int b) { mx_quantize_block<kCeil>(blk[u], packed + b, scales + b, bad); });
     if (bad)
         raise_status(status, kStatusNonFinite);
 }
 
 // ---------------------------------------------------------------------------
 // Dequantise.  One thread per 16 codes (8 packed bytes) -> 16 outputs (one
-// 32-byte bf16 store or two fp32 ones).
+// 32-byte bf16 store or two fp32 ones), four units in flight per thread.
+// NVFP4: p * s_b is exact in any format with 6 significant bits and the
+// range 2^-10 .. 2688, so it is formed by the mixed-precision
+// `fma.rn.f32.f16` (f16 code value x f16 scale + -0, the -0 keeping the
+// sign of a zero product), then multiplied by g as fp32 pairs.  MXFP4:
+// p * 2^e, exact, as fp32 pairs.  y points at the unit's 16 outputs.
 // ---------------------------------------------------------------------------
+template <bool kNv>
+__device__ __forceinline__ void dequant_floats(uint2 pk, uint32_t sbyte, uint64_t g2, float (&y16)[16])
+{
+    if constexpr (kNv) {
+        const uint16_t sh = e4m3_to_f16(sbyte);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t ph[4];
+            e2m1x8_to_f16x2(h ? pk.y : pk.x, ph);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float a, b;
+                f16x2_mul_f16_to_f32(ph[j], sh, a, b);
+                unpack2(mul2(pack2(a, b), g2), y16[8 * h + 2 * j], y16[8 * h + 2 * j + 1]);
+            }
+        }
+    } else if (sbyte - 103u <= 39u) {
+        // 2^e with -24 <= e <= 15 is exact in f16: p * 2^e (exact) by the
+        // mixed-precision fma, one instruction per element
+        const uint16_t sh = e8m0_to_f16(sbyte);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t ph[4];
+            e2m1x8_to_f16x2(h ? pk.y : pk.x, ph);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                f16x2_mul_f16_to_f32(ph[j], sh, y16[8 * h + 2 * j], y16[8 * h + 2 * j + 1]);
+        }
+    } else {
+        const float s = e8m0_to_f32(sbyte);
+        const uint64_t s2 = pack2(s, s);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float p[8];
+            e2m1x8_decode(h ? pk.y : pk.x, p);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                unpack2(mul2(pack2(p[2 * j], p[2 * j + 1]), s2), y16[8 * h + 2 * j],
+                        y16[8 * h + 2 * j + 1]);
+        }
+    }
+}
+
+// fp32 -> output element: bf16 bits (round to nearest even) or fp32.
+template <typename TOut> __device__ __forceinline__ TOut to_out(float v)
+{
+    if constexpr (sizeof(TOut) == 2) {
+        uint16_t h;
+        asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(v));
+        return h;
+    } else {
+        return v;
+    }
+}
+
+template <bool kNv, typename TOut>
+__device__ __forceinline__ void dequant_unit(uint2 pk, uint32_t sbyte, uint64_t g2, TOut *y)
+{
+    float y16[16];
+    dequant_floats<kNv>(pk, sbyte, g2, y16);
+    uint32_t o[8];
+    if constexpr (sizeof(TOut) == 2) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(y16[2 * j + 1]), "f"(y16[2 * j]));
+        stg_v8(y, o);
+    } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                o[j] = __float_as_uint(y16[8 * h + j]);
+            stg_v8(y + 8 * h, o);
+        }
+    }
+}
+
 template <bool kNv, typename TOut>
 __global__ void __launch_bounds__(kThreads)
     dequantize_kernel(const uint2 *__restrict__ packed, const uint8_t *__restrict__ scales,
-                      const float *__restrict__ global_scale, int64_t n_units,
-                      TOut *__restrict__ y)
+                      const float *__restrict__ global_scale, int n_units, TOut *__restrict__ y)
 {
     pdl_begin();
-    constexpr int kUnroll = 2;
     const float g = kNv ? __ldcg(global_scale) : 1.0f;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n_units;
-         i0 += kUnroll * stride) {
-        uint2 pk[kUnroll];
-        uint32_t sbyte[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t unit = i0 + u * stride;
-            if (unit < n_units) {
-                pk[u] = __ldcg(packed + unit);
-                sbyte[u] = __ldcg(scales + (kNv ? unit : (unit >> 1)));
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t unit = i0 + u * stride;
-            if (unit >= n_units)
-                continue;
-            const float s = kNv ? e4m3_to_f32(sbyte[u]) : e8m0_to_f32(sbyte[u]);
-            float y16[16];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float p[8];
-                e2m1x8_decode(h ? pk[u].y : pk[u].x, p);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    y16[8 * h + k] = kNv ? nv_dequant(p[k], s, g) : __fmul_rn(p[k], s);
-            }
-            if constexpr (sizeof(TOut) == 2) {
-                uint32_t o[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[j]) : "f"(y16[2 * j + 1]), "f"(y16[2 * j]));
-                stg_v8(reinterpret_cast<char *>(y) + unit * 32, o);
-            } else {
-                uint32_t o[8];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        o[j] = __float_as_uint(y16[8 * h + j]);
-                    stg_v8(reinterpret_cast<char *>(y) + unit * 64 + 32 * h, o);
-                }
-            }
-        }
-    }
+    const uint64_t g2 = pack2(g, g);
+    uint2 pk[4];
+    uint32_t sbyte[4];
+    stream_units<4>(
+        n_units,
+        [&](int u, int i) {
+            pk[u] = __ldcg(packed + i);
+            sbyte[u] = __ldcg(scales + (kNv ? i : (i >> 1)));
+        },
+        [&](int u, int i) { dequant_unit<kNv>(pk[u], sbyte[u], g2, y + (int64_t)i * 16); });
 }
 
 // ---------------------------------------------------------------------------
@@ -478,9 +554,9 @@ __global__ void __launch_bounds__(kThreads)
 // ---------------------------------------------------------------------------
 // Eight consecutive elements (half a block) reloaded from memory as fp32.
 template <typename T>
-__device__ __forceinline__ void load_half(const T *x, int64_t blk, int h, float (&v)[8])
+__device__ __forceinline__ void load_half(const T *x, int blk, int h, float (&v)[8])
 {
-    const char *p = reinterpret_cast<const char *>(x) + (blk * 16 + 8 * h) * (int64_t)sizeof(T);
+    const char *p = reinterpret_cast<const char *>(x) + ((int64_t)blk * 16 + 8 * h) * (int64_t)sizeof(T);
     uint32_t w[8];
     if constexpr (sizeof(T) == 2) {
         asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -501,7 +577,7 @@ __device__ __forceinline__ void load_half(const T *x, int64_t blk, int h, float 
 
 // Exact codes of one half-block at scale code c (zero scale -> zero codes).
 template <typename T>
-__device__ __forceinline__ uint32_t exact_half_codes(const T *x, int64_t blk, int h, uint32_t c,
+__device__ __forceinline__ uint32_t exact_half_codes(const T *x, int blk, int h, uint32_t c,
                                                      float g, float (&v)[8])
 {
     load_half(x, blk, h, v);
@@ -516,7 +592,7 @@ __device__ __forceinline__ uint32_t exact_half_codes(const T *x, int64_t blk, in
 // at a time to stay light on registers (inlined: it is small, and ptxas
 // 12.9 crashed on an out-of-line version called from two kernels).
 template <typename T>
-__device__ __forceinline__ double exact_loss_of(const T *x, int64_t blk, uint32_t c, float g)
+__device__ __forceinline__ double exact_loss_of(const T *x, int blk, uint32_t c, float g)
 {
     const float sb = e4m3_pos_to_f32(c);
     double acc = 0.0;
@@ -536,7 +612,7 @@ __device__ __forceinline__ double exact_loss_of(const T *x, int64_t blk, uint32_
 // Exact codes of a whole block at scale code c (used when g is so small that
 // the scaled encode could see subnormal reconstructions).
 template <typename T>
-__device__ __forceinline__ uint2 exact_codes_of(const T *x, int64_t blk, uint32_t c, float g)
+__device__ __forceinline__ uint2 exact_codes_of(const T *x, int blk, uint32_t c, float g)
 {
     float v[8];
     uint2 pk;
@@ -565,23 +641,31 @@ __device__ __forceinline__ Screen screen(const float (&xk)[16], uint32_t c, floa
     const float dk = __fmul_rn(__fmul_rn(e4m3_pos_to_f32(c), g), k);
     const float r0 = rcp_approx(dk);
     const float rc = fmaf(r0, fmaf(-dk, r0, 1.0f), r0);
-    float acc = 0.0f;
+    // four interleaved fp32 sums (two packed pairs, two short dependency
+    // chains); summation error < 7u S
+    const uint64_t rc2 = pack2(rc, rc);
+    uint64_t acc2[2] = {pack2(0.0f, 0.0f), pack2(0.0f, 0.0f)};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        float v[8], p[8];
+        float v[8], e[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            v[i] = __fmul_rn(xk[8 * h + i], rc);
-        e2m1x8_qdq(v, p);
+        for (int j = 0; j < 4; ++j)
+            unpack2(mul2(pack2(xk[8 * h + 2 * j], xk[8 * h + 2 * j + 1]), rc2), v[2 * j], v[2 * j + 1]);
+        e2m1x8_error(v, e);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float e = __fsub_rn(v[i], p[i]);
-            acc = fmaf(e, e, acc);
+        for (int j = 0; j < 4; ++j) {
+            const uint64_t e2 = pack2(e[2 * j], e[2 * j + 1]);
+            acc2[j & 1] = fma2(e2, e2, acc2[j & 1]);
         }
     }
+    float a0, a1, a2, a3;
+    unpack2(acc2[0], a0, a1);
+    unpack2(acc2[1], a2, a3);
+    const float acc = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
     const float d2 = __fmul_rn(dk, dk);
     r.s = __fmul_rn(acc, d2);
-    r.bound = fmaf(r.s, 1e-6f, fmaf(sqrtf(r.s), 6e-6f, fmaf(d2, 7e-5f, 1e-11f)));
+    // sqrt.approx is within 2^-21 of sqrt(S): the 6.001e-6 covers it
+    r.bound = fmaf(r.s, 1e-6f, fmaf(sqrt_approx(r.s), 6.001e-6f, fmaf(d2, 7e-5f, 1e-11f)));
     return r;
 }
 
@@ -592,7 +676,7 @@ __device__ __forceinline__ Screen screen(const float (&xk)[16], uint32_t c, floa
 // optional loss output reload the block.
 template <typename T> struct BlockSearch {
     const T *x;
-    int64_t blk;
+    int blk;
     float xk[16];
     float g, k, ak, gk;
     uint32_t c_lo, best_c, next_c;
@@ -600,7 +684,7 @@ template <typename T> struct BlockSearch {
     bool exact_always;
 
     // Loads the block; returns max |x| over it.
-    __device__ __forceinline__ float setup(const T *x_, int64_t blk_, float g_, bool exact_always_)
+    __device__ __forceinline__ float setup(const T *x_, int blk_, float g_, bool exact_always_)
     {
         x = x_;
         blk = blk_;
@@ -608,13 +692,14 @@ template <typename T> struct BlockSearch {
         exact_always = exact_always_;
         Blk<T, 16> b;
         load_blk(x, blk, b);
-        const uint32_t ab = absmax_bits_finite(b);
+        const uint32_t ab = absmax_bits(b);
         k = __uint_as_float((254u - min(ab >> 23, 253u)) << 23);
         gk = __fmul_rn(g, k);
         ak = __fmul_rn(__uint_as_float(ab), k);
+        const uint64_t k2 = pack2(k, k);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            xk[i] = __fmul_rn(elem(b, i), k);
+        for (int i = 0; i < 8; ++i)
+            unpack2(mul2(pack2(elem(b, 2 * i), elem(b, 2 * i + 1)), k2), xk[2 * i], xk[2 * i + 1]);
         return __uint_as_float(ab);
     }
 
@@ -685,8 +770,8 @@ template <typename T> struct BlockSearch {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
-    scale_search_kernel(const T *__restrict__ x, int64_t n_blocks, const float *amax,
+__global__ void __launch_bounds__(kThreads, 4)
+    scale_search_kernel(const T *__restrict__ x, int n_blocks, const float *amax,
                         uint2 *__restrict__ packed, uint8_t *__restrict__ scales,
                         float *global_scale, float *__restrict__ block_loss, int32_t *status)
 {
@@ -698,9 +783,8 @@ __global__ void __launch_bounds__(kThreads)
     const double g1260 = 1260.0 * (double)g;      // exact: 9 + 24 significant bits
     const float inv_lo = (float)(147.0 / g1260);  // RN32(0.7 / (6g))
     const bool exact_always = !(g >= 0x1p-116f);
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < n_blocks;
-         blk += stride) {
+    const int stride = (int)(gridDim.x * blockDim.x);
+    for (int blk = (int)(blockIdx.x * blockDim.x + threadIdx.x); blk < n_blocks; blk += stride) {
         BlockSearch<T> bs;
         const float amax_b = bs.setup(x, blk, g, exact_always);
         const uint32_t c_hi = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
@@ -725,7 +809,7 @@ __global__ void __launch_bounds__(kThreads)
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-    nvfp4_four_over_six_kernel(const T *__restrict__ x, int64_t n_blocks, const float *amax,
+    nvfp4_four_over_six_kernel(const T *__restrict__ x, int n_blocks, const float *amax,
                                uint2 *__restrict__ packed, uint8_t *__restrict__ scales,
                                float *global_scale, float *__restrict__ block_loss,
                                int32_t *status)
@@ -738,9 +822,8 @@ __global__ void __launch_bounds__(kThreads)
     const double four_g = 4.0 * (double)g;    // exact
     const float inv4g = (float)(1.0 / four_g); // RN32(1 / (4g))
     const bool exact_always = !(g >= 0x1p-116f);
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < n_blocks;
-         blk += stride) {
+    const int stride = (int)(gridDim.x * blockDim.x);
+    for (int blk = (int)(blockIdx.x * blockDim.x + threadIdx.x); blk < n_blocks; blk += stride) {
         BlockSearch<T> bs;
         const float amax_b = bs.setup(x, blk, g, exact_always);
         const uint32_t c6 = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);

@@ -1,0 +1,158 @@
+// fp4_launch.cuh -- host-side launch helpers shared by the C-ABI translation
+// units: SM count, persistent grid size, launch with programmatic stream
+// serialisation, and the split of a problem into launches of at most
+// fp4::kMaxUnitsPerLaunch units.  Internal linkage (each translation unit
+// keeps its own caches).
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "fp4.h"
+#include "fp4_kernels.cuh"
+
+namespace fp4_launch {
+
+// Units per launch of the chunked calls: fp4::kMaxUnitsPerLaunch, or a
+// smaller multiple of 64 set by fp4_set_launch_unit_limit (tests only).
+// One definition, in fp4_capi.cu.
+extern int64_t g_launch_unit_limit;
+
+namespace {
+
+using fp4::kThreads;
+
+constexpr int kMaxDevices = 64;
+
+// Workspace words of the single-tensor calls: fp4::kMaxPartials per-CTA
+// maxima, the wrapping CTA counter, and the amax word the NVFP4 quantiser
+// and the search read.
+constexpr size_t kWsAmax = fp4::kMaxPartials + 1; // word kMaxPartials is the counter
+constexpr size_t kWsWords = fp4::kMaxPartials + 8;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// SM count of the current device (cached per device).
+int sm_count(int &dev)
+{
+    static int cache[kMaxDevices] = {0};
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
+        return -1;
+    if (dev < kMaxDevices && cache[dev] > 0)
+        return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return -1;
+    if (dev < kMaxDevices)
+        cache[dev] = n;
+    return n;
+}
+
+// Resident CTAs per SM of `kernel` at `block` threads and `smem` bytes of
+// dynamic shared memory (cached per device and kernel instantiation; a
+// kernel is always queried with the same block and smem).
+template <typename K> int resident_ctas(K kernel, int dev, int block = kThreads, size_t smem = 0)
+{
+    static int cache[kMaxDevices] = {0};
+    if (dev < kMaxDevices && cache[dev] > 0)
+        return cache[dev];
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, smem) != cudaSuccess ||
+        n <= 0)
+        n = 1;
+    if (dev < kMaxDevices)
+        cache[dev] = n;
+    return n;
+}
+
+// Persistent grid: enough CTAs for `work` items at `per_cta` items each,
+// at most SMs x resident CTAs, at least one.
+template <typename K>
+int grid_for(K kernel, int64_t work, int64_t per_cta, int block = kThreads, size_t smem = 0)
+{
+    int dev = 0;
+    const int sms = sm_count(dev);
+    if (sms <= 0)
+        return -1;
+    const int64_t cap = (int64_t)sms * resident_ctas(kernel, dev, block, smem);
+    int64_t want = (work + per_cta - 1) / per_cta;
+    if (want < 1)
+        want = 1;
+    return (int)(want < cap ? want : cap);
+}
+
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel on the stream finishes; it waits for it
+// (griddepcontrol.wait) before touching memory.
+template <typename... KArgs, typename... Args>
+fp4_status launch_cfg(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                      cudaStream_t stream, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return FP4_ERR_CUDA;
+    }
+    return FP4_OK;
+}
+
+template <typename... KArgs, typename... Args>
+fp4_status launch(void (*kernel)(KArgs...), int grid, cudaStream_t stream, Args... args)
+{
+    return launch_cfg(kernel, grid, kThreads, 0, stream, args...);
+}
+
+// Runs one(first, count) over units [0, n) in chunks of at most
+// g_launch_unit_limit (the kernels index units with 32-bit integers).
+// At least one call is made, with count 0 for an empty problem, so that
+// kernels with a prologue (the NVFP4 global scale) still run once.
+template <typename F> fp4_status for_chunks(int64_t n, F &&one)
+{
+    int64_t first = 0;
+    do {
+        const int64_t left = n - first;
+        const int64_t lim = g_launch_unit_limit;
+        const int count = (int)(left < lim ? left : lim);
+        const fp4_status st = one(first, count);
+        if (st != FP4_OK)
+            return st;
+        first += count;
+    } while (first < n);
+    return FP4_OK;
+}
+
+// Runs one(first_row, count) over rows [0, rows) in chunks whose
+// units (rows x units_per_row) stay within g_launch_unit_limit (a row larger
+// than that is FP4_ERR_SHAPE); at least one call, as for_chunks.
+// units_per_row >= 1.
+template <typename F> fp4_status for_row_chunks(int64_t rows, int64_t units_per_row, F &&one)
+{
+    const int64_t per = g_launch_unit_limit / units_per_row;
+    if (per < 1)
+        return FP4_ERR_SHAPE;
+    int64_t first = 0;
+    do {
+        const int64_t left = rows - first;
+        const int64_t count = left < per ? left : per;
+        const fp4_status st = one(first, count);
+        if (st != FP4_OK)
+            return st;
+        first += count;
+    } while (first < rows);
+    return FP4_OK;
+}
+
+bool valid_dtype(fp4_dtype t) { return t == FP4_F32 || t == FP4_BF16; }
+
+} // namespace
+} // namespace fp4_launch

@@ -1,0 +1,329 @@
+// fp4_layouts.cu -- entry points of include/fp4.h for ragged rows (padded
+// to whole blocks) and column-wise grouping.  Argument checks, the TMA
+// tensor map of the column-wise pass, and the launches.
+#include <climits>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fp4.h"
+#include "fp4_launch.cuh"
+#include "fp4_layouts.cuh"
+
+namespace {
+
+using namespace fp4_launch;
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+fp4_status check_rows_cols(int64_t rows, int64_t cols)
+{
+    if (rows < 0 || cols < 0)
+        return FP4_ERR_INVALID_ARG;
+    if (cols > 0 && rows > INT64_MAX / cols / 4)
+        return FP4_ERR_SHAPE;
+    return FP4_OK;
+}
+
+// ---------------------------------------------------------------- padded --
+
+template <typename T>
+fp4_status nv_padded(const T *x, int64_t rows, int64_t cols, const float *amax, uint8_t *packed,
+                     uint8_t *scales, float *global_scale, int32_t *status, cudaStream_t stream)
+{
+    const int64_t nbp = ceil_div(cols, 16);
+    constexpr size_t kSmem = fp4::pad_smem_bytes<T>(16);
+    return for_row_chunks(rows, nbp, [&](int64_t r0, int64_t nr) {
+        const int n = (int)(nr * nbp);
+        const int grid = grid_for(fp4::nvfp4_quantize_padded_kernel<T>, n, fp4::kPadTile, fp4::kPadTile, kSmem);
+        if (grid <= 0)
+            return FP4_ERR_CUDA;
+        return launch_cfg(fp4::nvfp4_quantize_padded_kernel<T>, grid, fp4::kPadTile, kSmem, stream,
+                          x + r0 * cols, cols, fp4::fast_div_for((uint32_t)nbp), n, amax,
+                          reinterpret_cast<uint2 *>(packed) + r0 * nbp, scales + r0 * nbp, global_scale,
+                          status);
+    });
+}
+
+template <typename T, bool kCeil>
+fp4_status mx_padded(const T *x, int64_t rows, int64_t cols, uint8_t *packed, uint8_t *scales,
+                     int32_t *status, cudaStream_t stream)
+{
+    const int64_t nbp = ceil_div(cols, 32);
+    constexpr size_t kSmem = fp4::pad_smem_bytes<T>(32);
+    return for_row_chunks(rows, nbp, [&](int64_t r0, int64_t nr) {
+        const int n = (int)(nr * nbp);
+        const int grid = grid_for(fp4::mxfp4_quantize_padded_kernel<T, kCeil>, n, fp4::kPadTile,
+                                  fp4::kPadTile, kSmem);
+        if (grid <= 0)
+            return FP4_ERR_CUDA;
+        return launch_cfg(fp4::mxfp4_quantize_padded_kernel<T, kCeil>, grid, fp4::kPadTile, kSmem, stream,
+                          x + r0 * cols, cols, fp4::fast_div_for((uint32_t)nbp), n,
+                          reinterpret_cast<uint4 *>(packed) + r0 * nbp, scales + r0 * nbp, status);
+    });
+}
+
+template <bool kNv, typename TOut>
+fp4_status dq_padded(const uint8_t *packed, const uint8_t *scales, const float *global_scale,
+                     int64_t rows, int64_t cols, TOut *y, cudaStream_t stream)
+{
+    const int64_t nup = ceil_div(cols, kNv ? 16 : 32) * (kNv ? 1 : 2); // 16-code units per row
+    constexpr size_t kSmem = fp4::pad_smem_bytes<TOut>(16);
+    return for_row_chunks(rows, nup, [&](int64_t r0, int64_t nr) {
+        const int n = (int)(nr * nup);
+        const int grid = grid_for(fp4::dequantize_padded_kernel<kNv, TOut>, n, fp4::kPadTile, fp4::kPadTile,
+                                  kSmem);
+        if (grid <= 0)
+            return FP4_ERR_CUDA;
+        return launch_cfg(fp4::dequantize_padded_kernel<kNv, TOut>, grid, fp4::kPadTile, kSmem, stream,
+                          reinterpret_cast<const uint2 *>(packed) + r0 * nup,
+                          scales + (kNv ? r0 * nup : r0 * nup / 2), global_scale, cols,
+                          fp4::fast_div_for((uint32_t)nup), n, y + r0 * cols);
+    });
+}
+
+// ----------------------------------------------------------- column-wise --
+
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                 const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                 const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+EncodeTiled encode_tiled()
+{
+    static std::once_flag once;
+    static EncodeTiled fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+        else
+            (void)cudaGetLastError();
+    });
+    return fn;
+}
+
+// Tensor map of W [rows, cols] (innermost: cols), box 512 bytes x 64 rows,
+// no swizzle, zero fill out of bounds.
+template <typename T> fp4_status column_map(const T *x, int64_t rows, int64_t cols, CUtensorMap *map)
+{
+    EncodeTiled enc = encode_tiled();
+    if (!enc)
+        return FP4_ERR_CUDA;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(T)};
+    const cuuint32_t box[2] = {512u / (cuuint32_t)sizeof(T), (cuuint32_t)fp4::kColTileRows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                           2, const_cast<T *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
+}
+
+template <typename T, bool kNv, bool kCeil>
+fp4_status columns(const T *x, int64_t rows, int64_t cols, const float *amax, uint8_t *packed,
+                   uint8_t *scales, float *global_scale, int32_t *status, cudaStream_t stream)
+{
+    auto kernel = fp4::quantize_columns_kernel<T, kNv, kCeil>;
+    constexpr size_t kSmem = (size_t)fp4::kColStages * fp4::kColTileBytes;
+    static bool attr_set[kMaxDevices] = {false};
+    int dev = 0;
+    if (sm_count(dev) <= 0 || dev >= kMaxDevices)
+        return FP4_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem) !=
+            cudaSuccess) {
+            (void)cudaGetLastError();
+            return FP4_ERR_CUDA;
+        }
+        attr_set[dev] = true;
+    }
+    CUtensorMap map;
+    memset(&map, 0, sizeof(map));
+    const int64_t tile_cols = 512 / (int64_t)sizeof(T);
+    const int64_t n_tiles = (rows > 0 && cols > 0) ? ceil_div(rows, fp4::kColTileRows) * ceil_div(cols, tile_cols) : 0;
+    if (n_tiles > 0) {
+        const fp4_status st = column_map(x, rows, cols, &map);
+        if (st != FP4_OK)
+            return st;
+    }
+    constexpr int kBlock = fp4::col_threads<kNv>();
+    const int grid = grid_for(kernel, n_tiles, 1, kBlock, kSmem);
+    if (grid <= 0)
+        return FP4_ERR_CUDA;
+    return launch_cfg(kernel, grid, kBlock, kSmem, stream, map, (int)rows, (int)cols,
+                      (int)n_tiles, amax, packed, scales, global_scale, status);
+}
+
+// Common checks of the quantisers here; NV also needs a workspace.
+fp4_status check_quant(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                       const uint8_t *packed, const uint8_t *scales, const int32_t *status)
+{
+    if (!status || !valid_dtype(dtype))
+        return FP4_ERR_INVALID_ARG;
+    const fp4_status st = check_rows_cols(rows, cols);
+    if (st != FP4_OK)
+        return st;
+    if (rows * cols > 0 && (!x || !packed || !scales))
+        return FP4_ERR_INVALID_ARG;
+    if (!aligned(x, 32) || !aligned(packed, 16))
+        return FP4_ERR_ALIGN;
+    return FP4_OK;
+}
+
+fp4_status check_ws(const void *workspace, size_t bytes)
+{
+    if (!workspace || bytes < kWsWords * sizeof(uint32_t) || !aligned(workspace, 4))
+        return FP4_ERR_WORKSPACE;
+    return FP4_OK;
+}
+
+// The column-wise pass reads W through a TMA tensor map: 32-bit sizes and
+// a row pitch that is a multiple of 16 bytes.
+fp4_status check_columns(fp4_dtype dtype, int64_t rows, int64_t cols)
+{
+    if (rows > INT_MAX || cols > INT_MAX)
+        return FP4_ERR_SHAPE;
+    if ((cols * (dtype == FP4_BF16 ? 2 : 4)) % 16)
+        return FP4_ERR_ALIGN;
+    return FP4_OK;
+}
+
+} // namespace
+
+extern "C" {
+
+fp4_status fp4_nvfp4_quantize_padded(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                     uint8_t *packed, uint8_t *scales, float *global_scale,
+                                     void *workspace, size_t workspace_bytes, int32_t *status,
+                                     cudaStream_t stream)
+{
+    fp4_status st = check_quant(x, dtype, rows, cols, packed, scales, status);
+    if (st != FP4_OK)
+        return st;
+    if (!global_scale)
+        return FP4_ERR_INVALID_ARG;
+    if ((st = check_ws(workspace, workspace_bytes)) != FP4_OK)
+        return st;
+    if (cols % 16 == 0)
+        return fp4_nvfp4_quantize(x, dtype, rows, cols, packed, scales, global_scale, workspace,
+                                  workspace_bytes, status, stream);
+    float *amax = reinterpret_cast<float *>(static_cast<uint32_t *>(workspace) + kWsAmax);
+    st = fp4_tensor_amax(x, dtype, rows * cols, amax, workspace, workspace_bytes, status, stream);
+    if (st != FP4_OK)
+        return st;
+    if (dtype == FP4_BF16)
+        return nv_padded(static_cast<const uint16_t *>(x), rows, cols, amax, packed, scales,
+                         global_scale, status, stream);
+    return nv_padded(static_cast<const float *>(x), rows, cols, amax, packed, scales, global_scale,
+                     status, stream);
+}
+
+fp4_status fp4_mxfp4_quantize_padded(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                     fp4_mx_rule rule, uint8_t *packed, uint8_t *scales,
+                                     int32_t *status, cudaStream_t stream)
+{
+    fp4_status st = check_quant(x, dtype, rows, cols, packed, scales, status);
+    if (st != FP4_OK)
+        return st;
+    if (rule != FP4_MX_FLOOR && rule != FP4_MX_CEIL)
+        return FP4_ERR_INVALID_ARG;
+    if (cols % 32 == 0)
+        return rule == FP4_MX_CEIL
+                   ? fp4_mxfp4_quantize_ceil(x, dtype, rows, cols, packed, scales, status, stream)
+                   : fp4_mxfp4_quantize(x, dtype, rows, cols, packed, scales, status, stream);
+    const bool bf = dtype == FP4_BF16, ceil = rule == FP4_MX_CEIL;
+    if (bf && ceil)
+        return mx_padded<uint16_t, true>(static_cast<const uint16_t *>(x), rows, cols, packed, scales, status, stream);
+    if (bf)
+        return mx_padded<uint16_t, false>(static_cast<const uint16_t *>(x), rows, cols, packed, scales, status, stream);
+    if (ceil)
+        return mx_padded<float, true>(static_cast<const float *>(x), rows, cols, packed, scales, status, stream);
+    return mx_padded<float, false>(static_cast<const float *>(x), rows, cols, packed, scales, status, stream);
+}
+
+fp4_status fp4_dequantize_padded(fp4_format fmt, const uint8_t *packed, const uint8_t *scales,
+                                 const float *global_scale, int64_t rows, int64_t cols, void *y,
+                                 fp4_dtype out_dtype, cudaStream_t stream)
+{
+    if ((fmt != FP4_NVFP4 && fmt != FP4_MXFP4) || !valid_dtype(out_dtype))
+        return FP4_ERR_INVALID_ARG;
+    const bool nv = fmt == FP4_NVFP4;
+    fp4_status st = check_rows_cols(rows, cols);
+    if (st != FP4_OK)
+        return st;
+    if (rows * cols == 0)
+        return FP4_OK;
+    if (!packed || !scales || !y || (nv && !global_scale))
+        return FP4_ERR_INVALID_ARG;
+    const size_t esz = out_dtype == FP4_BF16 ? 2 : 4;
+    if (!aligned(packed, 16) || !aligned(y, esz) || (nv && !aligned(global_scale, 4)))
+        return FP4_ERR_ALIGN;
+    if (cols % (nv ? 16 : 32) == 0 && aligned(y, 32))
+        return fp4_dequantize(fmt, packed, scales, global_scale, rows, cols, y, out_dtype, stream);
+    if (nv && out_dtype == FP4_BF16)
+        return dq_padded<true>(packed, scales, global_scale, rows, cols, static_cast<uint16_t *>(y), stream);
+    if (nv)
+        return dq_padded<true>(packed, scales, global_scale, rows, cols, static_cast<float *>(y), stream);
+    if (out_dtype == FP4_BF16)
+        return dq_padded<false>(packed, scales, global_scale, rows, cols, static_cast<uint16_t *>(y), stream);
+    return dq_padded<false>(packed, scales, global_scale, rows, cols, static_cast<float *>(y), stream);
+}
+
+fp4_status fp4_nvfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                      uint8_t *packed, uint8_t *scales, float *global_scale,
+                                      void *workspace, size_t workspace_bytes, int32_t *status,
+                                      cudaStream_t stream)
+{
+    fp4_status st = check_quant(x, dtype, rows, cols, packed, scales, status);
+    if (st != FP4_OK)
+        return st;
+    if (!global_scale)
+        return FP4_ERR_INVALID_ARG;
+    if ((st = check_columns(dtype, rows, cols)) != FP4_OK)
+        return st;
+    if ((st = check_ws(workspace, workspace_bytes)) != FP4_OK)
+        return st;
+    float *amax = reinterpret_cast<float *>(static_cast<uint32_t *>(workspace) + kWsAmax);
+    st = fp4_tensor_amax(x, dtype, rows * cols, amax, workspace, workspace_bytes, status, stream);
+    if (st != FP4_OK)
+        return st;
+    if (dtype == FP4_BF16)
+        return columns<uint16_t, true, false>(static_cast<const uint16_t *>(x), rows, cols, amax, packed,
+                                              scales, global_scale, status, stream);
+    return columns<float, true, false>(static_cast<const float *>(x), rows, cols, amax, packed, scales,
+                                       global_scale, status, stream);
+}
+
+fp4_status fp4_mxfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                      fp4_mx_rule rule, uint8_t *packed, uint8_t *scales,
+                                      int32_t *status, cudaStream_t stream)
+{
+    fp4_status st = check_quant(x, dtype, rows, cols, packed, scales, status);
+    if (st != FP4_OK)
+        return st;
+    if (rule != FP4_MX_FLOOR && rule != FP4_MX_CEIL)
+        return FP4_ERR_INVALID_ARG;
+    if ((st = check_columns(dtype, rows, cols)) != FP4_OK)
+        return st;
+    const bool bf = dtype == FP4_BF16, ceil = rule == FP4_MX_CEIL;
+    const uint16_t *xb = static_cast<const uint16_t *>(x);
+    const float *xf = static_cast<const float *>(x);
+    if (bf && ceil)
+        return columns<uint16_t, false, true>(xb, rows, cols, nullptr, packed, scales, nullptr, status, stream);
+    if (bf)
+        return columns<uint16_t, false, false>(xb, rows, cols, nullptr, packed, scales, nullptr, status, stream);
+    if (ceil)
+        return columns<float, false, true>(xf, rows, cols, nullptr, packed, scales, nullptr, status, stream);
+    return columns<float, false, false>(xf, rows, cols, nullptr, packed, scales, nullptr, status, stream);
+}
+
+} // extern "C"

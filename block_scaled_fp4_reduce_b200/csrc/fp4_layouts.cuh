@@ -1,0 +1,535 @@
+// fp4_layouts.cuh -- the other block layouts of "NVFP4 与 MXFP4 格式":
+//
+//   ragged rows (section 8: padding each row to whole blocks, R*ceil(K/G)
+//     blocks; section 7: the padded layout is decoded as padded and then cut
+//     back to the logical shape).  Rows of K elements, K not a multiple of
+//     the block size G, are quantised as if padded with +0 to
+//     Kp = ceil(K/G)*G; the outputs are the plain layout of the padded
+//     [R, Kp] matrix.  Dequantisation writes only the K logical columns.
+//   column-wise grouping (section 6: grouping along the other axis changes
+//     which elements share a block, Q(W)^T != Q(W^T)).  The blocks of
+//     Q(W^T) run down the columns of W [R, C]; the output is the plain
+//     row-padded layout of the [C, R] transpose, produced from W directly.
+//
+// The column-wise quantiser stages 64-row x 512-byte tiles of W in shared
+// memory with 2-D TMA loads (cp.async.bulk.tensor, no multicast), two
+// stages deep: each stage has a "full" mbarrier (the TMA bytes landed) and
+// an "empty" one (every warp released the tile), and thread 0 refills a
+// stage as soon as it is empty, so no CTA-wide barrier sits in the loop.
+// Each thread then quantises whole 16- or 32-element blocks down one (fp32)
+// or two (bf16) tile columns.  Rows past R read as zeros (TMA out-of-bounds
+// fill), which is the +0 padding.  Every mbarrier wait is bounded: a thread
+// that runs out records FP4_ERR_TIMEOUT and leaves the loop, the waits that
+// depended on it run out in turn, and thread 0 waits (bounded again) for
+// every copy it started before the CTA ends.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda.h>
+
+#include "fp4_kernels.cuh"
+
+namespace fp4 {
+
+constexpr int32_t kStatusTimeout = 8;
+
+// ---------------------------------------------------------------------------
+// Ragged rows.  Block b of the row-padded [R, Kp] matrix is row b / nbp,
+// block b % nbp of that row; it covers the elements [f, f + cnt) of the flat
+// input, f = (b / nbp) K + (b % nbp) G, cnt = min(G, K - (b % nbp) G), and
+// reads +0 past them.  Consecutive blocks cover consecutive flat elements,
+// so a tile of kPadTile blocks is one contiguous span of x.  The kernels
+// stage that span (rounded out to 32-byte vectors) in shared memory with
+// aligned 256-bit loads, or, for dequantisation, assemble it there and
+// write its interior back with 256-bit stores.  In shared memory each
+// 32-byte vector takes 36 bytes (one pad word per eight): a block that
+// starts 32 bytes after its neighbour's then starts in another bank, so the
+// word accesses of a warp are conflict-free.
+// ---------------------------------------------------------------------------
+constexpr int kPadTile = 256; // blocks (quantise) or 16-code units (dequantise) per tile
+
+// Word w of the staged span lives at word w + w / 8.
+__device__ __forceinline__ int pad_word(int w) { return w + (w >> 3); }
+
+template <typename T> constexpr int pad_smem_bytes(int G)
+{
+    // span of kPadTile blocks of G elements, one vector of slack at each end,
+    // and room for the last block's reads past its real elements
+    return (kPadTile * G * (int)sizeof(T) / 32 + 4) * 36;
+}
+
+// First element of the span of [f0, ...) that starts a 32-byte vector at
+// the absolute address (p: the array, element-aligned; the result may lie a
+// few elements before f0 when p itself is not 32-byte aligned).
+template <typename T> __device__ __forceinline__ int64_t span_base(const T *p, int64_t f0)
+{
+    constexpr int kPerVec = 32 / (int)sizeof(T);
+    const int64_t mis = (int64_t)((reinterpret_cast<uintptr_t>(p) / sizeof(T)) % kPerVec);
+    return f0 - (f0 + mis) % kPerVec;
+}
+
+// Division of a 31-bit unsigned n by a launch-invariant d >= 1 (the round-up
+// method of Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994): l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1,
+// q = (mulhi(m, n) + n) >> l; mulhi(m, n) <= n < 2^31, so the sum does not
+// overflow.  The host builds it (fast_div_for).
+struct FastDiv {
+    uint32_t d, m, l;
+    __device__ __forceinline__ int div(int n) const
+    {
+        return (int)((__umulhi(m, (uint32_t)n) + (uint32_t)n) >> l);
+    }
+};
+
+inline FastDiv fast_div_for(uint32_t d)
+{
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < d)
+        ++l;
+    const uint64_t m = ((1ull << 32) * ((1ull << l) - d)) / d + 1;
+    return FastDiv{d, (uint32_t)m, l};
+}
+
+// First flat element of block b and its element count.
+__device__ __forceinline__ int64_t pad_block_start(int b, const FastDiv &nbp, int64_t K, int G, int &cnt)
+{
+    const int r = nbp.div(b);
+    const int j = b - r * (int)nbp.d;
+    const int64_t c0 = (int64_t)j * G;
+    cnt = (int)min((int64_t)G, K - c0);
+    return (int64_t)r * K + c0;
+}
+
+// Stages the flat elements [base, base + nvec * per_vec) of x into smem
+// (36-byte slots); elements at or past n read as +0.  base is 32-byte
+// aligned in memory; it precedes the tile's first element by less than one
+// vector, and lies before x only when x is a later row chunk of the caller's
+// tensor (memory of the same tensor; those words are never used).
+template <typename T>
+__device__ __forceinline__ void stage_span(const T *x, int64_t n, int64_t base, int nvec, uint32_t *sw)
+{
+    constexpr int kPerVec = 32 / (int)sizeof(T);
+    for (int v = (int)threadIdx.x; v < nvec; v += (int)blockDim.x) {
+        const int64_t e = base + (int64_t)v * kPerVec;
+        uint32_t w[8];
+        if (e + kPerVec <= n) {
+            ldg_v8(x + e, w);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if constexpr (sizeof(T) == 2) {
+                    const uint32_t lo = e + 2 * i < n ? (uint32_t)__ldcg(reinterpret_cast<const unsigned short *>(x + e + 2 * i)) : 0u;
+                    const uint32_t hi = e + 2 * i + 1 < n ? (uint32_t)__ldcg(reinterpret_cast<const unsigned short *>(x + e + 2 * i + 1)) : 0u;
+                    w[i] = lo | (hi << 16);
+                } else {
+                    w[i] = e + i < n ? __float_as_uint(__ldcg(x + e + i)) : 0u;
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            sw[v * 9 + i] = w[i];
+    }
+}
+
+// Block of N elements starting at staged element q (cnt of them real, the
+// rest +0) as a Blk.
+template <typename T, int N>
+__device__ __forceinline__ void staged_block(const uint32_t *sw, int q, int cnt, Blk<T, N> &k)
+{
+    if constexpr (sizeof(T) == 2) {
+        const int w0 = q >> 1;
+        const uint32_t sh = (uint32_t)(q & 1) * 16u;
+        uint32_t prev = sw[pad_word(w0)];
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) {
+            const uint32_t next = sw[pad_word(w0 + i + 1)];
+            k.w[i] = __funnelshift_r(prev, next, sh);
+            prev = next;
+        }
+        if (cnt < N) {
+#pragma unroll
+            for (int i = 0; i < N / 2; ++i) {
+                if (2 * i >= cnt)
+                    k.w[i] = 0u;
+                else if (2 * i + 1 >= cnt)
+                    k.w[i] &= 0xFFFFu;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            k.w[i] = i < cnt ? sw[pad_word(q + i)] : 0u;
+    }
+}
+
+// Tile loop shared by the padded quantisers: stage each tile's span, then
+// hand every thread its block (kPadTile threads).
+template <typename T, int G, typename Body>
+__device__ __forceinline__ void padded_tiles(const T *x, int64_t K, const FastDiv &nbp, int n_blocks,
+                                             Body &&body)
+{
+    constexpr int kPerVec = 32 / (int)sizeof(T);
+    extern __shared__ __align__(16) uint32_t sw[];
+    const int64_t n = (int64_t)nbp.div(n_blocks) * K; // whole rows in this launch
+    for (int b0 = (int)blockIdx.x * kPadTile; b0 < n_blocks; b0 += (int)gridDim.x * kPadTile) {
+        const int nb = min(kPadTile, n_blocks - b0);
+        int cnt0, cnt1;
+        const int64_t f0 = pad_block_start(b0, nbp, K, G, cnt0);
+        const int64_t f1 = pad_block_start(b0 + nb - 1, nbp, K, G, cnt1) + cnt1;
+        const int64_t base = span_base(x, f0);
+        const int nvec = (int)((f1 - base + kPerVec - 1) / kPerVec);
+        stage_span(x, n, base, nvec, sw);
+        __syncthreads();
+        if ((int)threadIdx.x < nb) {
+            const int b = b0 + (int)threadIdx.x;
+            int cnt;
+            const int64_t f = pad_block_start(b, nbp, K, G, cnt);
+            Blk<T, G> blk;
+            staged_block(sw, (int)(f - base), cnt, blk);
+            body(b, blk);
+        }
+        __syncthreads();
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPadTile)
+    nvfp4_quantize_padded_kernel(const T *__restrict__ x, int64_t K, FastDiv nbp, int n_blocks,
+                                 const float *amax, uint2 *__restrict__ packed,
+                                 uint8_t *__restrict__ scales, float *global_scale, int32_t *status)
+{
+    pdl_begin();
+    float g;
+    if (!nv_prologue(amax, global_scale, status, g))
+        return;
+    const NvScaleConsts sc = nv_scale_consts(g);
+    padded_tiles<T, 16>(x, K, nbp, n_blocks, [&](int b, const Blk<T, 16> &blk) {
+        nv_quantize_block(blk, sc, packed + b, scales + b);
+    });
+}
+
+template <typename T, bool kCeil>
+__global__ void __launch_bounds__(kPadTile)
+    mxfp4_quantize_padded_kernel(const T *__restrict__ x, int64_t K, FastDiv nbp, int n_blocks,
+                                 uint4 *__restrict__ packed, uint8_t *__restrict__ scales,
+                                 int32_t *status)
+{
+    pdl_begin();
+    bool bad = false;
+    padded_tiles<T, 32>(x, K, nbp, n_blocks, [&](int b, const Blk<T, 32> &blk) {
+        mx_quantize_block<kCeil>(blk, packed + b, scales + b, bad);
+    });
+    if (bad)
+        raise_status(status, kStatusNonFinite);
+}
+
+// Dequantise a row-padded layout into the logical [R, K] output.  Unit i is
+// 16 codes of the padded matrix (row i / nup, columns (i % nup) * 16 ..);
+// each thread writes its unit's logical outputs (columns below K) into the
+// staged span, then the CTA stores the span: whole 32-byte vectors with
+// 256-bit stores (the span starts on a 32-byte boundary of y), the two edge
+// vectors, shared with the neighbouring tiles, element by element.
+template <bool kNv, typename TOut>
+__global__ void __launch_bounds__(kPadTile)
+    dequantize_padded_kernel(const uint2 *__restrict__ packed, const uint8_t *__restrict__ scales,
+                             const float *__restrict__ global_scale, int64_t K, FastDiv nup,
+                             int n_units, TOut *__restrict__ y)
+{
+    constexpr int kPerVec = 32 / (int)sizeof(TOut);
+    extern __shared__ __align__(16) uint32_t sw[];
+    uint16_t *sh = reinterpret_cast<uint16_t *>(sw);
+    pdl_begin();
+    const float g = kNv ? __ldcg(global_scale) : 1.0f;
+    const uint64_t g2 = pack2(g, g);
+    for (int i0 = (int)blockIdx.x * kPadTile; i0 < n_units; i0 += (int)gridDim.x * kPadTile) {
+        const int nu = min(kPadTile, n_units - i0);
+        int cnt0, cnt1;
+        const int64_t f0 = pad_block_start(i0, nup, K, 16, cnt0);
+        const int64_t f1 = pad_block_start(i0 + nu - 1, nup, K, 16, cnt1) + cnt1;
+        const int64_t base = span_base(y, f0);
+        const int lo = (int)(f0 - base), hi = (int)(f1 - base); // the span, relative to base
+        if ((int)threadIdx.x < nu) {
+            const int i = i0 + (int)threadIdx.x;
+            int cnt;
+            const int q = (int)(pad_block_start(i, nup, K, 16, cnt) - base);
+            float y16[16];
+            dequant_floats<kNv>(__ldcg(packed + i), __ldcg(scales + (kNv ? i : (i >> 1))), g2, y16);
+            if constexpr (sizeof(TOut) == 2) {
+                uint32_t pr[8]; // bf16 pairs (y[2k], y[2k+1]), low half first
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(pr[k]) : "f"(y16[2 * k + 1]), "f"(y16[2 * k]));
+                const int w0 = q >> 1;
+                if (cnt == 16 && !(q & 1)) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        sw[pad_word(w0 + k)] = pr[k];
+                } else if (cnt == 16) {
+                    // odd start: y[0] is the high half of word w0, y[15] the
+                    // low half of word w0 + 8 (the other halves belong to the
+                    // neighbouring units); words in between hold (y[2k-1], y[2k])
+                    sh[2 * pad_word(w0) + 1] = (uint16_t)pr[0];
+#pragma unroll
+                    for (int k = 1; k < 8; ++k)
+                        sw[pad_word(w0 + k)] = __byte_perm(pr[k - 1], pr[k], 0x5432);
+                    sh[2 * pad_word(w0 + 8)] = (uint16_t)(pr[7] >> 16);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        if (j >= cnt)
+                            break;
+                        const int e = q + j;
+                        sh[2 * pad_word(e >> 1) + (e & 1)] = (uint16_t)(pr[j >> 1] >> (16 * (j & 1)));
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    if (j >= cnt)
+                        break;
+                    sw[pad_word(q + j)] = __float_as_uint(y16[j]);
+                }
+            }
+        }
+        __syncthreads();
+        const int nvec = (hi + kPerVec - 1) / kPerVec;
+        for (int v = (int)threadIdx.x; v < nvec; v += (int)blockDim.x) {
+            const int e = v * kPerVec;
+            if (e >= lo && e + kPerVec <= hi) {
+                uint32_t w[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    w[k] = sw[v * 9 + k];
+                stg_v8(y + base + e, w);
+            } else {
+                for (int k = max(lo - e, 0); k < min(kPerVec, hi - e); ++k) {
+                    const int ei = e + k;
+                    if constexpr (sizeof(TOut) == 2)
+                        y[base + ei] = sh[2 * pad_word(ei >> 1) + (ei & 1)];
+                    else
+                        y[base + ei] = __uint_as_float(sw[pad_word(ei)]);
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Column-wise quantisation.  Tiles of kColTileRows rows x 512 bytes of W
+// (256 bf16 or 128 fp32 columns).  A tile row is 128 four-byte words; the
+// CTA has 128 threads per block row of the tile (64 / G block rows: 512
+// threads for NVFP4, 256 for MXFP4), and thread (j, w) quantises the
+// block(s) of block row j in word column w: one fp32 column, or the two bf16
+// columns that share the word.
+// ---------------------------------------------------------------------------
+constexpr int kColWords = 128;
+constexpr int kColTileRows = 64;
+constexpr int kColTileBytes = kColTileRows * 512;
+constexpr int kColStages = 2;
+template <bool kNv> constexpr int col_threads() { return kColWords * (kColTileRows / (kNv ? 16 : 32)); }
+constexpr uint32_t kWaitTries = 1u << 22;
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Bounded wait for phase `parity` of the barrier; false when the tries run out.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    for (uint32_t t = 0; t < kWaitTries; ++t) {
+        uint32_t done;
+        asm volatile("{\n\t"
+                     ".reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t"
+                     "}"
+                     : "=r"(done)
+                     : "r"(smem_addr(bar)), "r"(parity)
+                     : "memory");
+        if (done)
+            return true;
+    }
+    return false;
+}
+
+// 2-D TMA tile load of box (x = column, y = row) into shared memory,
+// completing on `bar`.  x is a multiple of 512 bytes' worth of elements.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+// Tile t of the column-wise pass: column tile t % n_tc, row tile t / n_tc
+// (consecutive CTAs sweep across the columns of one row band together).
+struct ColTile {
+    int r0, c0;
+};
+
+__device__ __forceinline__ ColTile col_tile(int t, int n_tc, int tile_cols)
+{
+    const int tr = t / n_tc;
+    return {tr * kColTileRows, (t - tr * n_tc) * tile_cols};
+}
+
+// Quantises the G-element blocks of the tile rows [j*G, j*G + G) in this
+// thread's columns and stores them into the output rows (= columns of W).
+template <typename T, bool kNv, bool kCeil, int G>
+__device__ __forceinline__ void column_blocks(const uint8_t *tile, int j, int w, int c_first, int C,
+                                              int blk, const NvScaleConsts &sc, uint8_t *packed,
+                                              uint8_t *scales, int64_t prow, int nbo, bool &bad)
+{
+    constexpr int kPerThread = 4 / (int)sizeof(T); // columns per word: 2 (bf16) or 1 (fp32)
+    const uint32_t *tw = reinterpret_cast<const uint32_t *>(tile) + j * G * kColWords + w;
+    uint32_t rowv[G]; // row i of this thread's word column
+#pragma unroll
+    for (int i = 0; i < G; ++i)
+        rowv[i] = tw[i * kColWords];
+#pragma unroll
+    for (int p = 0; p < kPerThread; ++p) {
+        const int c = c_first + p;
+        if (c >= C)
+            continue;
+        Blk<T, G> b;
+        if constexpr (sizeof(T) == 2) {
+            // bf16: a word holds columns 2t (low half) and 2t+1 (high half);
+            // gather one column's halves of rows 2i, 2i+1 into word i.
+#pragma unroll
+            for (int i = 0; i < G / 2; ++i)
+                b.w[i] = __byte_perm(rowv[2 * i], rowv[2 * i + 1], p ? 0x7632 : 0x5410);
+        } else {
+#pragma unroll
+            for (int i = 0; i < G; ++i)
+                b.w[i] = rowv[i];
+        }
+        uint8_t *orow = packed + (int64_t)c * prow;
+        if constexpr (kNv)
+            nv_quantize_block(b, sc, reinterpret_cast<uint2 *>(orow) + blk, scales + (int64_t)c * nbo + blk);
+        else
+            mx_quantize_block<kCeil>(b, reinterpret_cast<uint4 *>(orow) + blk,
+                                     scales + (int64_t)c * nbo + blk, bad);
+    }
+}
+
+template <typename T, bool kNv, bool kCeil>
+__global__ void __launch_bounds__(col_threads<kNv>())
+    quantize_columns_kernel(const __grid_constant__ CUtensorMap map, int R, int C, int n_tiles,
+                            const float *amax, uint8_t *__restrict__ packed,
+                            uint8_t *__restrict__ scales, float *global_scale, int32_t *status)
+{
+    constexpr int G = kNv ? 16 : 32;
+    constexpr int kCols = 512 / (int)sizeof(T);          // tile columns
+    constexpr int kPerWord = 4 / (int)sizeof(T);         // columns per 4-byte word
+    constexpr int kWarps = col_threads<kNv>() / 32;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ __align__(8) uint64_t full[kColStages];  // tile landed (TMA bytes)
+    __shared__ __align__(8) uint64_t empty[kColStages]; // every warp is done with the tile
+
+    pdl_begin();
+    float g = 1.0f;
+    if constexpr (kNv) {
+        if (!nv_prologue(amax, global_scale, status, g))
+            return;
+    }
+    const NvScaleConsts sc = nv_scale_consts(g);
+    const int n_tc = (C + kCols - 1) / kCols;
+    const int Rp = (R + G - 1) / G * G;                  // padded column length
+    const int64_t prow = Rp / 2;                         // packed bytes per output row
+    const int nbo = Rp / G;                              // blocks (scale bytes) per output row
+    const int first_tile = blockIdx.x;
+    const int stride = gridDim.x;
+    const int w = (int)threadIdx.x % kColWords;          // word column of the tile
+    const int jb = (int)threadIdx.x / kColWords;         // block row of the tile
+    const bool producer = threadIdx.x == 0;
+
+    if (producer) {
+        for (int s = 0; s < kColStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kWarps);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    int issued = 0; // tiles of this CTA whose copy thread 0 has started
+    if (producer) {
+        for (int s = 0; s < kColStages; ++s) {
+            const int t = first_tile + s * stride;
+            if (t < n_tiles) {
+                const ColTile ct = col_tile(t, n_tc, kCols);
+                mbar_expect_tx(&full[s], kColTileBytes);
+                tma_load_2d(smem + s * kColTileBytes, &map, ct.c0, ct.r0, &full[s]);
+                ++issued;
+            }
+        }
+    }
+    // Each warp waits for its tiles on full[s], releases them on empty[s];
+    // thread 0 refills a stage once every warp has released it.  All waits
+    // are bounded; a thread that gives up leaves the loop, and every wait
+    // that depended on it then runs out in turn.
+    bool bad = false, timed_out = false;
+    int k = 0;
+    for (int t = first_tile; t < n_tiles; t += stride, ++k) {
+        const int s = k % kColStages;
+        const uint32_t phase = (uint32_t)(k / kColStages) & 1u;
+        if (!mbar_wait(&full[s], phase)) {
+            timed_out = true;
+            break;
+        }
+        const ColTile ct = col_tile(t, n_tc, kCols);
+        const int blk_row = ct.r0 + jb * G;
+        if (blk_row < R)
+            column_blocks<T, kNv, kCeil, G>(smem + s * kColTileBytes, jb, w, ct.c0 + w * kPerWord, C,
+                                            blk_row / G, sc, packed, scales, prow, nbo, bad);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0)
+            mbar_arrive(&empty[s]);
+        if (producer) {
+            const int tn = t + kColStages * stride;
+            if (tn < n_tiles) {
+                if (!mbar_wait(&empty[s], phase)) {
+                    timed_out = true;
+                    break;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                const ColTile cn = col_tile(tn, n_tc, kCols);
+                mbar_expect_tx(&full[s], kColTileBytes);
+                tma_load_2d(smem + s * kColTileBytes, &map, cn.c0, cn.r0, &full[s]);
+                ++issued;
+            }
+        }
+    }
+    if (timed_out)
+        raise_status(status, kStatusTimeout);
+    if (producer) {
+        // Before the CTA can end, every copy thread 0 started must have
+        // landed: wait (bounded) for those not consumed above.
+        for (int j = k; j < issued; ++j)
+            (void)mbar_wait(&full[j % kColStages], (uint32_t)(j / kColStages) & 1u);
+    }
+    if (bad)
+        raise_status(status, kStatusNonFinite);
+}
+
+} // namespace fp4

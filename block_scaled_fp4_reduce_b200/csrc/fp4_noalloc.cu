@@ -127,13 +127,25 @@ fp4_status quantize_with_static_scratch(const T *x, int64_t rows, int64_t cols, 
     fp4_status st = launch_chained(fp4::amax_kernel<T>, grid, stream, x, n, ws, amax, status);
     if (st != FP4_OK)
         return st;
+    // 32-bit block indices in the kernel: chunks of at most 2^30 blocks, and
+    // one launch even for an empty tensor (it publishes g).
     const int64_t n_blocks = n / 16;
-    grid = persistent_grid(fp4::nvfp4_quantize_kernel<T>, n_blocks, (int64_t)fp4::kThreads * 2);
-    if (grid <= 0)
-        return FP4_ERR_CUDA;
-    return launch_chained(fp4::nvfp4_quantize_kernel<T>, grid, stream, x, n_blocks,
-                          static_cast<const float *>(amax), reinterpret_cast<uint2 *>(packed),
-                          scales, global_scale, status);
+    int64_t first = 0;
+    do {
+        const int64_t left = n_blocks - first;
+        const int count = (int)(left < fp4::kMaxUnitsPerLaunch ? left : fp4::kMaxUnitsPerLaunch);
+        grid = persistent_grid(fp4::nvfp4_quantize_kernel<T>, count, (int64_t)fp4::kThreads * 2);
+        if (grid <= 0)
+            return FP4_ERR_CUDA;
+        st = launch_chained(fp4::nvfp4_quantize_kernel<T>, grid, stream, x + first * 16, count,
+                            static_cast<const float *>(amax),
+                            reinterpret_cast<uint2 *>(packed) + first, scales + first,
+                            global_scale, status);
+        if (st != FP4_OK)
+            return st;
+        first += count;
+    } while (first < n_blocks);
+    return FP4_OK;
 }
 
 } // namespace

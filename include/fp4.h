@@ -71,11 +71,16 @@ typedef enum fp4_status {
     FP4_ERR_NONFINITE = 4,   /* (device status) NaN or Inf in the input */
     FP4_ERR_RANGE = 5,       /* (device status) NVFP4 global scale out of range */
     FP4_ERR_WORKSPACE = 6,   /* workspace NULL or smaller than required */
-    FP4_ERR_CUDA = 7         /* a CUDA launch or query failed */
+    FP4_ERR_CUDA = 7,        /* a CUDA launch or query failed */
+    FP4_ERR_TIMEOUT = 8      /* (device status) a bounded wait on a copy ran out */
 } fp4_status;
 
 typedef enum fp4_dtype { FP4_F32 = 0, FP4_BF16 = 1 } fp4_dtype;
 typedef enum fp4_format { FP4_NVFP4 = 0, FP4_MXFP4 = 1 } fp4_format;
+
+/* MXFP4 scale rule: the OCP rounding-down rule e = floor(log2 A_b) - 2, or
+ * the ceil rule 2^ceil(log2(A_b / 6)) ("NVFP4 与 MXFP4 格式" section 5). */
+typedef enum fp4_mx_rule { FP4_MX_FLOOR = 0, FP4_MX_CEIL = 1 } fp4_mx_rule;
 
 /* Human-readable name of a status value (static string). */
 const char *fp4_status_string(int status);
@@ -219,6 +224,166 @@ fp4_status fp4_scale_search_with_amax(const void *x, fp4_dtype dtype, int64_t ro
 fp4_status fp4_nvfp4_quantize_noalloc(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
                                       uint8_t *packed, uint8_t *scales, float *global_scale,
                                       int32_t *status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Ragged rows and column-wise grouping ("NVFP4 与 MXFP4 格式" sections 6-8).
+ *
+ * Padded layout.  A [rows, cols] matrix whose cols is not a multiple of the
+ * block size G (16 NVFP4, 32 MXFP4) is quantised as if every row were
+ * padded with +0 to Kp = ceil(cols / G) * G elements (section 8: rows *
+ * ceil(cols/G) blocks, not ceil(rows*cols/G); the pad value is not given on
+ * the page, and +0 changes no block maximum).  The outputs are the plain
+ * layout of the padded [rows, Kp] matrix: packed uint8 [rows, Kp/2], scales
+ * uint8 [rows, Kp/G]; NVFP4 g is that of the logical elements.  For cols a
+ * multiple of G the padded layout is the plain one, and the calls below are
+ * the plain calls.  Dequantisation of a padded layout (section 7: decode as
+ * padded, then cut each row back) writes only the logical [rows, cols].
+ * x must be 32-byte aligned as everywhere; y of fp4_dequantize_padded needs
+ * only its element alignment.
+ *
+ * Column-wise grouping.  Section 6: blocks taken down the columns of W are
+ * other blocks than those along its rows (Q(W)^T != Q(W^T)).  The
+ * _columns calls quantise W^T, the [cols, rows] transpose of the row-major
+ * x [rows, cols], without materialising it: the outputs are the padded
+ * layout of W^T (packed [cols, ceil(rows/G)*G/2], scales [cols,
+ * ceil(rows/G)]); decode them with fp4_dequantize_padded(rows = cols of x,
+ * cols = rows of x).  x is read through a TMA tensor map: rows, cols below
+ * 2^31 (else FP4_ERR_SHAPE) and a row pitch (cols * element size) that is a
+ * multiple of 16 bytes (else FP4_ERR_ALIGN).  A copy that never completes
+ * ends the kernel with FP4_ERR_TIMEOUT in *status instead of a hang.
+ * ------------------------------------------------------------------------ */
+
+/* NVFP4 quantise + pack of x [rows, cols], any cols >= 0, padded layout.
+ * Workspace, outputs and errors as fp4_nvfp4_quantize. */
+fp4_status fp4_nvfp4_quantize_padded(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                     uint8_t *packed, uint8_t *scales, float *global_scale,
+                                     void *workspace, size_t workspace_bytes, int32_t *status,
+                                     cudaStream_t stream);
+
+/* MXFP4 quantise + pack of x [rows, cols], any cols >= 0, padded layout,
+ * with scale rule `rule`.  Errors as fp4_mxfp4_quantize. */
+fp4_status fp4_mxfp4_quantize_padded(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                     fp4_mx_rule rule, uint8_t *packed, uint8_t *scales,
+                                     int32_t *status, cudaStream_t stream);
+
+/* Dequantise a padded layout of the logical [rows, cols] matrix into y
+ * [rows, cols] (fp32 or bf16), as fp4_dequantize on the padded matrix
+ * followed by cutting every row to cols. */
+fp4_status fp4_dequantize_padded(fp4_format fmt, const uint8_t *packed, const uint8_t *scales,
+                                 const float *global_scale, int64_t rows, int64_t cols, void *y,
+                                 fp4_dtype out_dtype, cudaStream_t stream);
+
+/* NVFP4 quantise + pack of W^T for x = W [rows, cols] (column-wise blocks),
+ * padded layout of the [cols, rows] transpose; g from the amax of W.
+ * Workspace as fp4_nvfp4_quantize.  Data errors NONFINITE, RANGE, TIMEOUT. */
+fp4_status fp4_nvfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                      uint8_t *packed, uint8_t *scales, float *global_scale,
+                                      void *workspace, size_t workspace_bytes, int32_t *status,
+                                      cudaStream_t stream);
+
+/* MXFP4 quantise + pack of W^T for x = W [rows, cols], padded layout of the
+ * transpose, scale rule `rule`.  Data errors NONFINITE, TIMEOUT. */
+fp4_status fp4_mxfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                      fp4_mx_rule rule, uint8_t *packed, uint8_t *scales,
+                                      int32_t *status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped calls: many matrices per call, each with its own scales.
+ *
+ * The global scale is a per-tensor quantity ("NVFP4 与 MXFP4 格式" section 3:
+ * A is the absolute maximum of the tensor being quantised), so a weight set
+ * of many matrices is quantised matrix by matrix, each with its own A and g.
+ * The grouped entry points do exactly what one single-matrix call per item
+ * would do -- bit for bit the same packed codes, scale bytes, g and
+ * dequantised values -- in a few launches for the whole set instead of one
+ * or two per matrix.  `items` is a HOST array read during the call only;
+ * every pointer inside it is a device pointer with the alignment and layout
+ * rules above.  Items may be empty (rows * cols == 0).  All argument checks
+ * run on every item before anything is queued.
+ * ------------------------------------------------------------------------ */
+
+/* One matrix of a grouped quantisation. */
+typedef struct fp4_quant_item {
+    const void *x;       /* input [rows, cols], fp32 or bf16 (the call's dtype) */
+    int64_t rows, cols;  /* cols % 16 == 0 (NVFP4) or % 32 == 0 (MXFP4) */
+    uint8_t *packed;     /* uint8 [rows, cols/2] */
+    uint8_t *scales;     /* uint8 [rows, cols/16] E4M3 or [rows, cols/32] E8M0 */
+    float *global_scale; /* NVFP4: receives this matrix's g; MXFP4: unused */
+} fp4_quant_item;
+
+/* One matrix of a grouped dequantisation. */
+typedef struct fp4_dequant_item {
+    const uint8_t *packed;     /* uint8 [rows, cols/2] */
+    const uint8_t *scales;     /* as produced by the quantisers */
+    const float *global_scale; /* NVFP4: this matrix's g; MXFP4: unused */
+    void *y;                   /* output [rows, cols], fp32 or bf16 (out_dtype) */
+    int64_t rows, cols;
+} fp4_dequant_item;
+
+/* Workspace of fp4_nvfp4_quantize_grouped: one 32-bit word per item,
+ * rounded up to 256 bytes.  Any contents on entry (the call clears it on
+ * `stream` first); after the call, in stream order, word i holds the fp32
+ * bit pattern of max|x| of item i. */
+size_t fp4_grouped_workspace_bytes(int n_items);
+
+/* Tensor amax of every item: after the call, in stream order, workspace
+ * word i holds max|x_i| as an fp32 (bit pattern), as fp4_tensor_amax gives
+ * for item i (NVFP4 item rules: cols % 16 == 0; global_scale unused).  The
+ * call clears the words on `stream` first.  A NaN or Inf in any item sets
+ * NONFINITE.  One clear and one kernel per 256 items or 2^30 x 64 KB. */
+fp4_status fp4_tensor_amax_grouped(const fp4_quant_item *items, int n_items, fp4_dtype dtype,
+                                   void *workspace, size_t workspace_bytes, int32_t *status,
+                                   cudaStream_t stream);
+
+/* NVFP4 quantise + pack of every item given the amax words of
+ * fp4_tensor_amax_grouped (`amax_words`, device, word i = item i), as
+ * fp4_nvfp4_quantize_with_amax per item.  One kernel per 256 items or 2^30
+ * blocks. */
+fp4_status fp4_nvfp4_quantize_grouped_with_amax(const fp4_quant_item *items, int n_items,
+                                                fp4_dtype dtype, const void *amax_words,
+                                                int32_t *status, cudaStream_t stream);
+
+/* NVFP4 quantise + pack of every item, each with its own tensor amax and
+ * global scale g_i = fl32(A_i / 2688), exactly as fp4_nvfp4_quantize per
+ * item.  A NaN or Inf in any item sets NONFINITE; an item whose g underflows
+ * sets RANGE; the outputs of such an item are unspecified, the others are
+ * still correct.  fp4_tensor_amax_grouped followed by
+ * fp4_nvfp4_quantize_grouped_with_amax on the workspace. */
+fp4_status fp4_nvfp4_quantize_grouped(const fp4_quant_item *items, int n_items, fp4_dtype dtype,
+                                      void *workspace, size_t workspace_bytes, int32_t *status,
+                                      cudaStream_t stream);
+
+/* MXFP4 quantise + pack of every item, as fp4_mxfp4_quantize per item
+ * (OCP rounding-down scale rule); _ceil: as fp4_mxfp4_quantize_ceil.  One
+ * kernel per 256 items or 2^30 blocks. */
+fp4_status fp4_mxfp4_quantize_grouped(const fp4_quant_item *items, int n_items, fp4_dtype dtype,
+                                      int32_t *status, cudaStream_t stream);
+fp4_status fp4_mxfp4_quantize_ceil_grouped(const fp4_quant_item *items, int n_items,
+                                           fp4_dtype dtype, int32_t *status, cudaStream_t stream);
+
+/* Dequantise every item, as fp4_dequantize per item.  One kernel per 256
+ * items or 2^30 units of 16 codes. */
+fp4_status fp4_dequantize_grouped(fp4_format fmt, const fp4_dequant_item *items, int n_items,
+                                  fp4_dtype out_dtype, cudaStream_t stream);
+
+/* Tests only: the largest number of work units one launch takes (default
+ * 2^30, restored by units = 0; else a multiple of 64 from 64 up).  Every
+ * call above splits larger problems into several launches at this limit;
+ * lowering it makes small tensors cross those split points.  Process-wide,
+ * not thread-safe; set it only while no other call is being made.
+ * FP4_ERR_INVALID_ARG for other values. */
+fp4_status fp4_set_launch_unit_limit(int64_t units);
+
+/* Launch planner of the grouped calls alone, for tests (host only, no GPU
+ * work).  Splits items of units[i] work units into launches of at most
+ * max_units units (64 .. 2^30) and max_entries entries (1 .. 256), as the
+ * grouped calls do with the largest limits: piece k covers units
+ * [first_of[k], first_of[k] + count_of[k]) of item item_of[k] in launch
+ * launch_of[k].  Returns the number of pieces (the arrays hold the first
+ * max_pieces of them), or -1 for invalid arguments. */
+int fp4_grouped_plan(const int64_t *units, int n_items, int64_t max_units, int max_entries,
+                     int32_t *launch_of, int32_t *item_of, int64_t *first_of, int64_t *count_of,
+                     int max_pieces);
 
 /* Element encoder alone, for tests: codes[i] = E2M1 code of the fp32 value
  * v[i] (nearest, ties to even code, saturating, sign bit kept).  A NaN or

@@ -1,0 +1,173 @@
+"""GPU parity of the ragged-row (padded) and column-wise layouts against the
+oracle, bit for bit ("NVFP4 与 MXFP4 格式" section 6: grouping along the
+other axis; section 7: decode padded, then cut each row back; section 8:
+R * ceil(K/G) blocks)."""
+import numpy as np
+import pytest
+import torch
+
+import block_scaled_fp4_reduce_b200 as fp4
+import oracle
+import workloads
+from conftest import golden
+from test_gpu_parity import assert_same, assert_same_bits, odata
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def rand(R, K, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(R, K, generator=g) * 0.05
+    if R * K:
+        x.view(-1)[torch.randint(0, R * K, (max(1, R * K // 300),), generator=g)] *= 30
+    return x.to(dtype)
+
+
+def check_padded(x):
+    R, K = x.shape
+    xo = odata(x)
+    xd = x.to(DEV)
+    nv = fp4.nvfp4_quantize_padded(xd)
+    mxf = fp4.mxfp4_quantize_padded(xd, fp4.MX_FLOOR)
+    mxc = fp4.mxfp4_quantize_padded(xd, fp4.MX_CEIL)
+    ynv = fp4.dequantize_padded(nv, torch.float32)
+    ynvb = fp4.dequantize_padded(nv, torch.bfloat16)
+    ymx = fp4.dequantize_padded(mxf, torch.bfloat16)
+    torch.cuda.synchronize()
+    for q in (nv, mxf, mxc):
+        q.check()
+    p, s, g = oracle.nvfp4_quantize_padded(xo)
+    assert nv.global_scale.item() == g
+    assert_same(nv.packed, p, f"NV padded packed {R}x{K}")
+    assert_same(nv.scales, s, f"NV padded scales {R}x{K}")
+    want = oracle.nvfp4_dequantize_padded(p, s, g, R, K)
+    assert ynv.shape == (R, K)
+    assert_same_bits(ynv, want, f"NV padded dequant fp32 {R}x{K}")
+    assert_same_bits(ynvb, want, f"NV padded dequant bf16 {R}x{K}")
+    for q, rule in ((mxf, oracle.MX_FLOOR), (mxc, oracle.MX_CEIL)):
+        p, s = oracle.mxfp4_quantize_padded(xo, rule)
+        assert_same(q.packed, p, f"MX padded packed rule {rule} {R}x{K}")
+        assert_same(q.scales, s, f"MX padded scales rule {rule} {R}x{K}")
+    p, s = oracle.mxfp4_quantize_padded(xo, oracle.MX_FLOOR)
+    assert_same_bits(ymx, oracle.mxfp4_dequantize_padded(p, s, R, K), f"MX padded dequant {R}x{K}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", [(1, 1), (2, 17), (3, 15), (5, 33), (7, 100), (64, 1000), (129, 4099), (4, 64)])
+def test_padded_rows_parity(dtype, shape):
+    check_padded(rand(*shape, dtype, seed=shape[0] * 7 + shape[1]))
+
+
+def test_padded_layout_bytes_of_the_page():
+    gd = golden("padded_layout.json")
+    x = torch.linspace(-1, 1, gd["rows"] * gd["cols"]).reshape(gd["rows"], gd["cols"]).to(DEV)
+    q = fp4.nvfp4_quantize_padded(x)
+    torch.cuda.synchronize()
+    q.check()
+    assert q.packed.numel() + q.scales.numel() + 4 == gd["nv_bytes"]
+    assert q.scales.numel() == gd["blocks_padded"]
+    check_padded(x.cpu())
+
+
+def test_padded_equals_plain_for_complete_rows():
+    x = rand(33, 256, torch.bfloat16, seed=2).to(DEV)
+    a, b = fp4.nvfp4_quantize(x), fp4.nvfp4_quantize_padded(x)
+    c, d = fp4.mxfp4_quantize(x), fp4.mxfp4_quantize_padded(x)
+    torch.cuda.synchronize()
+    assert torch.equal(a.packed, b.packed) and torch.equal(a.scales, b.scales)
+    assert a.global_scale.item() == b.global_scale.item()
+    assert torch.equal(c.packed, d.packed) and torch.equal(c.scales, d.scales)
+
+
+def check_columns(x):
+    R, C = x.shape
+    xo = odata(x)
+    xd = x.to(DEV)
+    nv = fp4.nvfp4_quantize_columns(xd)
+    mxf = fp4.mxfp4_quantize_columns(xd, fp4.MX_FLOOR)
+    mxc = fp4.mxfp4_quantize_columns(xd, fp4.MX_CEIL)
+    torch.cuda.synchronize()
+    for q in (nv, mxf, mxc):
+        q.check()
+    p, s, g = oracle.nvfp4_quantize_columns(xo)
+    assert nv.global_scale.item() == g
+    assert_same(nv.packed, p, f"NV columns packed {R}x{C}")
+    assert_same(nv.scales, s, f"NV columns scales {R}x{C}")
+    y = fp4.dequantize_padded(nv, torch.float32)
+    torch.cuda.synchronize()
+    assert y.shape == (C, R)
+    assert_same_bits(y, oracle.nvfp4_dequantize_padded(p, s, g, C, R), f"NV columns dequant {R}x{C}")
+    for q, rule in ((mxf, oracle.MX_FLOOR), (mxc, oracle.MX_CEIL)):
+        p, s = oracle.mxfp4_quantize_columns(xo, rule)
+        assert_same(q.packed, p, f"MX columns packed rule {rule} {R}x{C}")
+        assert_same(q.scales, s, f"MX columns scales rule {rule} {R}x{C}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", [(16, 8), (20, 8), (64, 256), (100, 264), (129, 520), (300, 1032), (65, 4)])
+def test_columns_parity(dtype, shape):
+    R, C = shape
+    if dtype == torch.bfloat16 and C % 8:
+        pytest.skip("bf16 rows need a 16-byte pitch")
+    check_columns(rand(R, C, dtype, seed=R * 5 + C))
+
+
+def test_columns_transpose_counterexample_of_the_page():
+    gd = golden("transpose_floor_rule.json")
+    n = gd["size"]
+    w = torch.full((n, n), gd["rest"])
+    w[0, 0] = gd["corner"]
+    wd = w.to(DEV)
+    col = fp4.mxfp4_quantize_columns(wd)
+    row = fp4.mxfp4_quantize(wd)
+    yc = fp4.dequantize_padded(col, torch.float32)
+    yr = fp4.dequantize(row, torch.float32)
+    torch.cuda.synchronize()
+    assert yc[0, 1].item() == gd["column_wise_0_1"]
+    assert yr.T[0, 1].item() == gd["row_wise_then_transpose_0_1"]
+    check_columns(w)
+
+
+def test_columns_argument_errors():
+    x = torch.randn(16, 12, device=DEV).bfloat16()  # 24-byte pitch
+    with pytest.raises(fp4.FP4Error) as e:
+        fp4.nvfp4_quantize_columns(x)
+    assert e.value.status == fp4.ERR_ALIGN
+    for R, C in ((0, 64), (64, 0)):
+        q = fp4.nvfp4_quantize_columns(torch.zeros(R, C, device=DEV))
+        torch.cuda.synchronize()
+        assert q.status.item() == 0 and q.global_scale.item() == 1.0
+
+
+def test_nonfinite_in_layouts():
+    x = torch.randn(40, 72)
+    x[13, 5] = float("inf")
+    xd = x.to(DEV)
+    for q in (fp4.nvfp4_quantize_padded(xd[:, :70].contiguous()), fp4.mxfp4_quantize_padded(xd[:, :70].contiguous()),
+              fp4.nvfp4_quantize_columns(xd), fp4.mxfp4_quantize_columns(xd)):
+        torch.cuda.synchronize()
+        assert q.status.item() == fp4.ERR_NONFINITE
+
+
+def test_columns_full_size_weight_sampled_columns():
+    """4096 x 4096 bf16 weight: column-wise blocks checked against the
+    oracle on sampled columns (each is one output row)."""
+    w = workloads.WEIGHT_4K
+    x = workloads.generate(w)
+    xd = x.to(DEV)
+    nv = fp4.nvfp4_quantize_columns(xd)
+    mx = fp4.mxfp4_quantize_columns(xd)
+    torch.cuda.synchronize()
+    nv.check()
+    mx.check()
+    g = oracle.nv_global_scale(x.abs().amax().float().item())
+    assert nv.global_scale.item() == g
+    cols = workloads.sample_rows(w.cols, 12, seed=3)
+    sub = odata(x[:, cols].T.contiguous())  # [k, R]: the sampled columns as rows
+    p, s = oracle.nvfp4_quantize_with_g(sub, g)
+    assert_same(nv.packed[cols], p, "NV columns packed (sampled)")
+    assert_same(nv.scales[cols], s, "NV columns scales (sampled)")
+    p, s = oracle.mxfp4_quantize(sub)
+    assert_same(mx.packed[cols], p, "MX columns packed (sampled)")
+    assert_same(mx.scales[cols], s, "MX columns scales (sampled)")

@@ -390,6 +390,22 @@ def test_tensor_amax_and_with_amax_variant():
     a, st = fp4.tensor_amax(x)
     torch.cuda.synchronize()
     assert st.item() == 0 and a.item() == x.abs().amax().float().item()
+    # subnormal and normal magnitudes mixed, both signs: the packed
+    # sign-agnostic max must order subnormals like their magnitudes
+    g = torch.Generator().manual_seed(11)
+    for dt, lo, hi in ((torch.bfloat16, -133, -120), (torch.float32, -149, -120)):
+        e = torch.randint(lo, hi, (4096,), generator=g).double()
+        s = torch.where(torch.rand(4096, generator=g) < 0.5, -1.0, 1.0).double()
+        y = (s * torch.exp2(e) * (1 + torch.rand(4096, generator=g).double() * 0.9)).to(dt)
+        y[torch.randperm(4096, generator=g)[:9]] = 0.0
+        a, st = fp4.tensor_amax(y.to(DEV))
+        torch.cuda.synchronize()
+        assert st.item() == 0 and a.item() == y.abs().amax().float().item()
+        m = fp4.mxfp4_quantize(y.reshape(128, 32).to(DEV))
+        torch.cuda.synchronize()
+        p, sc = oracle.mxfp4_quantize(odata(y.reshape(128, 32)))
+        assert_same(m.scales, sc, "MX scales on subnormals")
+        assert_same(m.packed, p, "MX codes on subnormals")
     # odd element counts take the scalar tail
     for n in (1, 7, 8, 9, 1001):
         y = torch.randn(n, device=DEV).to(torch.bfloat16)

@@ -53,6 +53,23 @@ ACT_8K = Workload("act-8192x14336-bf16", 8192, 14336, torch.bfloat16, 2, "studen
 SEARCH_4K = Workload("search-4096x14336-bf16", 4096, 14336, torch.bfloat16, 4, "laplace",
                      std=0.02, description="bf16 4096x14336 Laplace(0,0.02), seed 4")
 
+# The other block layouts: a weight grouped along its columns (Q(W^T) of a
+# 4096x14336 matrix, the down-projection shape of the weight set) and an
+# activation whose rows are one element short of whole blocks (14335 =
+# 895 x 16 + 15: every row ends in a 15-element block padded with +0).
+COLUMNS_4K = Workload("columns-4096x14336-bf16", 4096, 14336, torch.bfloat16, 5, "normal-outliers",
+                      std=0.02, out_frac=0.001, out_mult=50.0,
+                      description="bf16 4096x14336 N(0,0.02), 0.1% x50, seed 5; blocks down the columns")
+RAGGED_8K = Workload("ragged-8192x14335-bf16", 8192, 14335, torch.bfloat16, 6, "student-t",
+                     std=0.5, description="bf16 8192x14335 Student-t(nu=3) x0.5, seed 6; rows padded to "
+                                          "whole blocks")
+
+# The scale-rule variants on the activation distribution (Student-t rows of
+# 14336 elements, a fresh seed).
+VARIANTS_8K = Workload("variants-8192x14336-bf16", 8192, 14336, torch.bfloat16, 7, "student-t",
+                       std=0.5, description="bf16 8192x14336 Student-t(nu=3) x0.5, seed 7; MXFP4 ceil rule "
+                                            "and NVFP4 four over six")
+
 # The 7B-class weight set: per layer 4 square 4096x4096 and 3 4096x14336.
 MODEL_LAYERS = 32
 MODEL_MATRICES = [(4096, 4096)] * 4 + [(4096, 14336)] * 3
@@ -68,6 +85,16 @@ def model_matrix(layer: int, idx: int) -> Workload:
 
 def model_numel() -> int:
     return MODEL_LAYERS * sum(r * c for r, c in MODEL_MATRICES)
+
+
+# The whole weight set as one workload (processed with grouped calls, each
+# matrix drawn from its own model_matrix seed): rows x cols is only the
+# element count, 7,784,628,224 = 1,900,544 x 4096; the real shapes are
+# MODEL_MATRICES per layer.
+MODEL_WEIGHTS = Workload("model-7b-weights-bf16", model_numel() // 4096, 4096, torch.bfloat16, 3,
+                         "normal-outliers", std=0.02, out_frac=0.0005, out_mult=30.0,
+                         description="7B-class weight set: 32 layers x (4 x 4096x4096 + 3 x 4096x14336) "
+                                     "bf16, N(0,0.02), 0.05% x30 per matrix, seed 3 (per-matrix seeds)")
 
 
 def with_shape(w: Workload, rows: int, cols: int, seed_offset: int = 0) -> Workload:
