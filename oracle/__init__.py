@@ -95,6 +95,8 @@ def lib() -> ctypes.CDLL:
             "oracle_pad_rows": (I, [P, I, I64, I64, I64, P]),
             "oracle_crop_rows": (I, [P, I64, I64, I64, P]),
             "oracle_transpose": (I, [P, I, I64, I64, P]),
+            "oracle_nvfp4_gemm": (I, [P, P, F, P, P, F, I64, I64, I64, P, P]),
+            "oracle_scales_mma_layout": (I, [P, I64, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -461,3 +463,28 @@ def nvfp4_quantize_columns(x: np.ndarray):
 
 def mxfp4_quantize_columns(x: np.ndarray, rule: int = 0):
     return mxfp4_quantize_padded(transpose(x), rule)
+
+
+# --------------------------------------------------------------------------
+# The consumer: block-scaled matrix product ("NVFP4 与 MXFP4 格式" section 6)
+# --------------------------------------------------------------------------
+
+def nvfp4_gemm(pa, sa, ga, pb, sb, gb, M: int, N: int, K: int):
+    """D = A B^T of two NVFP4 operands blocked along K (A [M, K], B [N, K]),
+    exact in double; returns (D float64 [M, N], sum of |terms| [M, N])."""
+    pa, sa, pb, sb = (np.ascontiguousarray(a, dtype=np.uint8) for a in (pa, sa, pb, sb))
+    d = np.zeros((M, N), np.float64)
+    mag = np.zeros((M, N), np.float64)
+    _check(lib().oracle_nvfp4_gemm(_ptr(pa), _ptr(sa), float(ga), _ptr(pb), _ptr(sb), float(gb), M, N, K,
+                                   _ptr(d), _ptr(mag)))
+    return d, mag
+
+
+def scales_mma_layout(scales: np.ndarray) -> np.ndarray:
+    """Scale bytes [rows, nb] in the 128-row x 4-block tiled layout of the
+    block-scaled tensor-core MMA (flat uint8, zero padded)."""
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, nb = s.shape
+    out = np.zeros((-(-rows // 128)) * 128 * (-(-nb // 4)) * 4, np.uint8)
+    _check(lib().oracle_scales_mma_layout(_ptr(s), rows, nb, _ptr(out)))
+    return out

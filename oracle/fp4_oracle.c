@@ -743,3 +743,70 @@ int oracle_transpose(const void *x, int dtype, int64_t rows, int64_t cols, void 
         }
     return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* The consumer of the quantised operands: a block-scaled matrix       */
+/* product ([NVMX] S6: Y = X W with both operands blocked along K; the */
+/* block scales can only be taken out of the dot product of one block).*/
+/* ------------------------------------------------------------------ */
+
+/* D[m][n] = g_a g_b sum over 16-blocks kb of s_a[m][kb] s_b[n][kb]
+ * sum_{k in kb} p_a[m][k] p_b[n][k], for A = (packed_a [M, K/2], scales_a
+ * [M, K/16] E4M3, g_a) and B = (packed_b [N, K/2], scales_b [N, K/16], g_b),
+ * both blocked along K (B is stored N x K, the weight's K-grouping of
+ * [NVMX] S6).  Every product p s p s is exact in double, and the block sums
+ * are exact; the total is summed in double in k order.  Also returns, per
+ * output, the sum of the magnitudes of the terms (for error bounds). */
+int oracle_nvfp4_gemm(const uint8_t *packed_a, const uint8_t *scales_a, float g_a,
+                      const uint8_t *packed_b, const uint8_t *scales_b, float g_b, int64_t M,
+                      int64_t N, int64_t K, double *d, double *mag)
+{
+    if (M < 0 || N < 0 || K < 0 || K % 16)
+        return ORACLE_ERR_SHAPE;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, abs_acc = 0.0;
+            for (int64_t kb = 0; kb < K / 16; ++kb) {
+                double sa = oracle_e4m3_decode_byte(scales_a[m * (K / 16) + kb]);
+                double sb = oracle_e4m3_decode_byte(scales_b[n * (K / 16) + kb]);
+                double dot = 0.0, dot_abs = 0.0;
+                for (int64_t k = kb * 16; k < kb * 16 + 16; ++k) {
+                    int64_t ia = m * K + k, ib = n * K + k;
+                    int ca = (ia & 1) ? packed_a[ia / 2] >> 4 : packed_a[ia / 2] & 15;
+                    int cb = (ib & 1) ? packed_b[ib / 2] >> 4 : packed_b[ib / 2] & 15;
+                    double t = oracle_e2m1_decode(ca) * oracle_e2m1_decode(cb);
+                    dot += t;
+                    dot_abs += fabs(t);
+                }
+                acc += sa * sb * dot;
+                abs_acc += fabs(sa * sb) * dot_abs;
+            }
+            d[m * N + n] = acc * (double)g_a * (double)g_b;
+            if (mag)
+                mag[m * N + n] = abs_acc * fabs((double)g_a * (double)g_b);
+        }
+    return ORACLE_OK;
+}
+
+/* Scale bytes [rows, nb] (one per 16-block, row-major) in the blocked
+ * layout the block-scaled tensor-core MMA reads (not on the pages; it is
+ * the layout of the sm100 block-scaled MMA's scale factors): rows grouped
+ * in tiles of 128, blocks in tiles of 4, tiles in row-tile-major order with
+ * the block tiles contiguous; inside a 512-byte tile, row r = r0 + 32 r1
+ * (r0 < 32, r1 < 4) and block j (< 4) sit at byte 16 r0 + 4 r1 + j.  Rows
+ * and blocks past the matrix hold 0.  out has ceil(rows/128) * 128 *
+ * ceil(nb/4) * 4 bytes. */
+int oracle_scales_mma_layout(const uint8_t *scales, int64_t rows, int64_t nb, uint8_t *out)
+{
+    if (rows < 0 || nb < 0)
+        return ORACLE_ERR_ARG;
+    int64_t rt = (rows + 127) / 128, kt = (nb + 3) / 4;
+    memset(out, 0, (size_t)(rt * kt * 512));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < nb; ++j) {
+            int64_t tile = (r / 128) * kt + j / 4;
+            int64_t rr = r % 128;
+            out[tile * 512 + (rr % 32) * 16 + (rr / 32) * 4 + j % 4] = scales[r * nb + j];
+        }
+    return ORACLE_OK;
+}
