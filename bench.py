@@ -49,7 +49,9 @@ WORKLOADS = {
     "columns-4096x14336-bf16": workloads.COLUMNS_4K,
     "ragged-8192x14335-bf16": workloads.RAGGED_8K,
     "variants-8192x14336-bf16": workloads.VARIANTS_8K,
+    "gemm-8192x4096x14336-nvfp4": workloads.GEMM_ACT,
 }
+GEMM_WORKLOAD = "gemm-8192x4096x14336-nvfp4"
 LAYOUT_WORKLOADS = {"columns-4096x14336-bf16": "columns", "ragged-8192x14335-bf16": "padded",
                     "variants-8192x14336-bf16": "variants"}
 MODEL_WEIGHTS = "model-7b-weights-bf16"  # the whole weight set, grouped calls
@@ -66,8 +68,8 @@ def peaks() -> dict:
         with open(p) as f:
             d = json.load(f)
         return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
-                "source": "measured"}
-    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+                "bf16_tflops": float(d.get("bf16_tflops", 1590.0)), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
 def kernel_source_hash() -> str:
@@ -91,6 +93,7 @@ def algorithmic_bytes(w: workloads.Workload) -> dict:
         "nvfp4_dequantize": n // 2 + n // 16 + 2 * n,
         "mxfp4_dequantize": n // 2 + n // 32 + 2 * n,
         "scale_search": n * e + n // 2 + n // 16,
+        "scales_to_mma": 2 * (n // 16),
     }
 
 
@@ -350,6 +353,52 @@ class LayoutPath:
     check_status = Path.check_status
 
 
+class GemmPath:
+    """The consumer: per step the activation x [M, K] is quantised (tensor
+    amax, NVFP4 quantise, scales to the MMA layout) and multiplied on the
+    tensor cores by the weight W [N, K], quantised once before timing:
+    D [M, N] fp32 = g_x g_w x_hat W_hat^T."""
+    OPS = ["amax", "nvfp4_quantize", "scales_to_mma", "nvfp4_gemm"]
+    LAUNCHES = 4
+
+    def __init__(self, x: torch.Tensor, w: torch.Tensor):
+        import block_scaled_fp4_reduce_b200 as fp4
+        self.fp4 = fp4
+        L = fp4.lib()
+        dev = x.device
+        M, K = x.shape
+        N = w.shape[0]
+        self.x, self.n, self.M, self.N, self.K = x, x.numel(), M, N, K
+        u8 = torch.uint8
+        qw = fp4.nvfp4_quantize(w)
+        self.w_sf = fp4.scales_to_mma(qw.scales)
+        torch.cuda.synchronize()
+        qw.check()
+        self.qw = qw
+        self.amax = torch.empty(1, dtype=torch.float32, device=dev)
+        self.ws = fp4.workspace_for(x)
+        self.status = fp4.new_status(dev)
+        self.p = torch.empty((M, K // 2), dtype=u8, device=dev)
+        self.s = torch.empty((M, K // 16), dtype=u8, device=dev)
+        self.g = torch.empty(1, dtype=torch.float32, device=dev)
+        self.sf = torch.empty(L.fp4_mma_scales_bytes(M, K // 16), dtype=u8, device=dev)
+        self.d = torch.empty((M, N), dtype=torch.float32, device=dev)
+        st = torch.cuda.current_stream().cuda_stream
+        P = lambda t: t.data_ptr()  # noqa: E731
+        self.calls = [
+            (L.fp4_tensor_amax, (P(x), fp4.BF16, self.n, P(self.amax), P(self.ws), self.ws.numel(), P(self.status), st)),
+            (L.fp4_nvfp4_quantize_with_amax, (P(x), fp4.BF16, M, K, P(self.amax), P(self.p), P(self.s), P(self.g),
+                                              P(self.status), st)),
+            (L.fp4_scales_to_mma_layout, (P(self.s), M, K // 16, P(self.sf), st)),
+            (L.fp4_nvfp4_gemm, (P(self.p), P(self.sf), P(self.g), P(qw.packed), P(self.w_sf), P(qw.global_scale),
+                                M, N, K, P(self.d), P(self.status), st)),
+        ]
+        self.results = [self.d, self.status]
+
+    step = Path.step
+    check_status = Path.check_status
+
+
 def max_over_ranks(values: list[float], device, world: int) -> list[float]:
     """Element-wise max of per-rank timings (one all-reduce; identity at N=1)."""
     if world == 1:
@@ -390,7 +439,10 @@ def run_ours(args, rank: int, world: int, local: int):
         x_host = workloads.generate(w).pin_memory()
         x = x_host.to(dev, non_blocking=False)
         kind = LAYOUT_WORKLOADS.get(args.workload)
-        path = LayoutPath(x, kind) if kind else Path(x)
+        if args.workload == GEMM_WORKLOAD:
+            path = GemmPath(x, workloads.generate(workloads.for_rank(workloads.GEMM_W, rank), device=dev))
+        else:
+            path = LayoutPath(x, kind) if kind else Path(x)
     flush_l2 = L2Flush(args.flush_mib, dev)
     nops = len(path.calls)
 
@@ -458,6 +510,9 @@ def run_ours(args, rank: int, world: int, local: int):
     value = n_all * K / (total_ms / 1e3)
     pk = peaks()
     ab = algorithmic_bytes(w)
+    if args.workload == GEMM_WORKLOAD:  # operands, their scales and the fp32 output
+        M_, N_, K_ = path.M, path.N, path.K
+        ab["nvfp4_gemm"] = (M_ + N_) * (K_ // 2 + K_ // 16) + 4 * M_ * N_
     kernels = {}
     for name, ms in zip(path.OPS, per_op_ms):
         us = ms / K * 1e3
@@ -476,10 +531,16 @@ def run_ours(args, rank: int, world: int, local: int):
                      "variants": "amax, nvfp4 four-over-six quantize (its own amax + the two-candidate kernel), "
                                  "mxfp4 quantize with the ceil scale rule, nvfp4 and mxfp4 dequantize (bf16)"
                      }[LAYOUT_WORKLOADS[args.workload]]
+    if args.workload == GEMM_WORKLOAD:
+        step_desc = ("activation amax, nvfp4 quantize, scales to the MMA layout, tcgen05 block-scaled NVFP4 GEMM "
+                     "D [8192, 4096] fp32 with the weight [4096, 14336] quantised once before timing")
     if args.workload == MODEL_WEIGHTS:
         step_desc = ("grouped over all 224 matrices (one kernel per pass): per-matrix amax, nvfp4 quantize "
                      "(per-matrix g), mxfp4 quantize, nvfp4 dequantize (bf16), mxfp4 dequantize (bf16)")
-    roof = roofline_for(dom, kernels[dom], w, pk, n_cand)
+    gemm_mnk = (path.M, path.N, path.K) if args.workload == GEMM_WORKLOAD else None
+    if gemm_mnk:
+        dom = "nvfp4_gemm"  # the tensor-core kernel is the one this workload is about
+    roof = roofline_for(dom, kernels[dom], w, pk, n_cand, gemm_mnk)
     line = {
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": K,
         "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
@@ -527,7 +588,8 @@ def search_candidate_count(x: torch.Tensor, g: float) -> int:
 SEARCH_OPS_PER_EVAL = 7
 
 
-def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict, n_cand: int | None = None) -> dict:
+def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict, n_cand: int | None = None,
+                 gemm_mnk=None) -> dict:
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
@@ -536,6 +598,17 @@ def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict, n_cand: in
         ent = t.get("kernels", {}).get(name)
         if ent and ent.get("source_hash") == kernel_source_hash() and ent.get("workload") == w.name:
             traffic = ent.get("bytes_per_launch")
+    if name == "nvfp4_gemm" and gemm_mnk:
+        # tensor-bound: 2 M N K flops per launch against the FP4 dense peak,
+        # taken as the measured bf16 GEMM peak times the nominal FP4 / bf16
+        # ratio (9 / 2.25 PFLOP/s dense)
+        M, N, K = gemm_mnk
+        peak = pk["bf16_tflops"] * 4.0
+        achieved = 2.0 * M * N * K / (k["us"] * 1e-6) / 1e12
+        return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": name,
+                "work": f"2 x {M} x {N} x {K} flops",
+                "peak_source": f"measured bf16 {pk['bf16_tflops']:.1f} TFLOP/s x 4 (nominal FP4 / bf16 ratio)"}
     if name == "scale_search" and n_cand:
         # ALU-bound: fp32 lane operations of the distinct candidate
         # evaluations per second, against SMs x 128 FP32 lanes x max SM clock.
@@ -586,6 +659,24 @@ def _oracle_layout_step(xs, kind: str):
     oracle.mxfp4_dequantize_padded(pm, sm, R, C)
 
 
+_GEMM_W_SLICE = 256  # weight rows the oracle multiplies by (of 4096)
+
+
+def _oracle_gemm_step_factory():
+    """The GEMM workload on the oracle: quantise the sample rows of the
+    activation and multiply them by the first 256 rows of the quantised
+    weight (the weight is quantised once, before timing, as in the GPU
+    arm)."""
+    import oracle
+    wsl = workloads.as_oracle_array(workloads.generate(workloads.GEMM_W))[:_GEMM_W_SLICE]
+    wp, wsc, wg = oracle.nvfp4_quantize(np.ascontiguousarray(wsl))
+
+    def step(xs):
+        p, s, g = oracle.nvfp4_quantize(xs)
+        oracle.nvfp4_gemm(p, s, g, wp, wsc, wg, xs.shape[0], _GEMM_W_SLICE, xs.shape[1])
+    return step
+
+
 def oracle_sample_source(w: workloads.Workload):
     """(tensor the CPU legs sample rows from, the step on a row sample, what
     the sample is): the workload itself, or for the whole weight set its
@@ -597,6 +688,9 @@ def oracle_sample_source(w: workloads.Workload):
     kind = LAYOUT_WORKLOADS.get(w.name)
     if kind:
         return workloads.generate(w), lambda xs: _oracle_layout_step(xs, kind), w.name
+    if w.name == GEMM_WORKLOAD:
+        return (workloads.generate(w), _oracle_gemm_step_factory(),
+                f"{w.name}, times the first {_GEMM_W_SLICE} of the 4096 weight rows")
     return workloads.generate(w), _oracle_step, w.name
 
 

@@ -73,6 +73,9 @@ def lib() -> ctypes.CDLL:
             "fp4_dequantize_grouped": (I, [I, P, I, I, P]),
             "fp4_grouped_plan": (I, [P, I, I64, I, P, P, P, P, I]),
             "fp4_set_launch_unit_limit": (I, [I64]),
+            "fp4_mma_scales_bytes": (SZ, [I64, I64]),
+            "fp4_scales_to_mma_layout": (I, [P, I64, I64, P, P]),
+            "fp4_nvfp4_gemm": (I, [P, P, P, P, P, P, I64, I64, I64, P, P, P]),
             "fp4_nvfp4_quantize_padded": (I, [P, I, I64, I64, P, P, P, P, SZ, P, P]),
             "fp4_mxfp4_quantize_padded": (I, [P, I, I64, I64, I, P, P, P, P]),
             "fp4_dequantize_padded": (I, [I, P, P, P, I64, I64, P, I, P]),
@@ -453,6 +456,30 @@ def mxfp4_quantize_columns(x: torch.Tensor, rule: int = MX_FLOOR, status=None, s
     _check(lib().fp4_mxfp4_quantize_columns(_p(x), _dtype_code(x), R, C, rule, _p(packed), _p(scales), _p(st),
                                             _stream(stream)), "fp4_mxfp4_quantize_columns")
     return Quantized(MXFP4, packed, scales, None, st, C, R)
+
+
+def scales_to_mma(scales: torch.Tensor, stream=None) -> torch.Tensor:
+    """Block scales [rows, blocks] -> the tiled layout of the tensor-core MMA
+    (flat uint8, fp4_mma_scales_bytes long)."""
+    rows, nb = scales.shape
+    out = torch.empty(lib().fp4_mma_scales_bytes(rows, nb), dtype=torch.uint8, device=scales.device)
+    _check(lib().fp4_scales_to_mma_layout(_p(scales), rows, nb, _p(out), _stream(stream)), "fp4_scales_to_mma_layout")
+    return out
+
+
+def nvfp4_gemm(qa: Quantized, qb: Quantized, out=None, status=None, stream=None) -> torch.Tensor:
+    """D [M, N] fp32 = g_a g_b A B^T on the tensor cores for NVFP4 A [M, K]
+    and B [N, K] (M, N multiples of 128, K of 256)."""
+    if qa.fmt != NVFP4 or qb.fmt != NVFP4 or qa.cols != qb.cols:
+        raise ValueError("two NVFP4 operands with the same K required")
+    M, N, K = qa.rows, qb.rows, qa.cols
+    dev = qa.packed.device
+    d = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=dev)
+    st = status if status is not None else new_status(dev)
+    sa, sb = scales_to_mma(qa.scales, stream), scales_to_mma(qb.scales, stream)
+    _check(lib().fp4_nvfp4_gemm(_p(qa.packed), _p(sa), _p(qa.global_scale), _p(qb.packed), _p(sb),
+                                _p(qb.global_scale), M, N, K, _p(d), _p(st), _stream(stream)), "fp4_nvfp4_gemm")
+    return d
 
 
 def nvfp4_quantize_grouped(xs, status=None, stream=None) -> list[Quantized]:

@@ -1,0 +1,314 @@
+// fp4_gemm.cuh -- the consumer of the quantised operands on the tensor cores.
+//
+// "NVFP4 与 MXFP4 格式" section 6: for Y = X W with X [M, K] and W [K, N]
+// both blocked along K, an output element is g_X g_W sum over blocks of
+// s_X s_W (sum of the block's payload products): the block scales can only
+// be taken out of one block's dot product.  The sm100 block-scaled MMA
+// (tcgen05.mma kind::mxf4nvf4, block16) computes exactly that sum with the
+// E2M1 payloads and the E4M3 block scales as operands and an fp32
+// accumulator in tensor memory; the global scales multiply the result.
+//
+//   scales_to_mma_kernel  block scales [rows, K/16] (plain, as the quantisers
+//                         write them) -> the tiled layout the MMA reads:
+//                         128-row x 4-block tiles of 512 bytes, row r = r0 +
+//                         32 r1 and block j of a tile at byte 16 r0 + 4 r1 + j,
+//                         tiles row-tile-major with the block tiles
+//                         contiguous; padding 0 (the sm100 block-scaled
+//                         layout; it is not on the pages)
+//   nvfp4_gemm_kernel     D [M, N] fp32 = g_a g_b A B^T for NVFP4 A [M, K]
+//                         and B [N, K] (both K-major, i.e. blocked along K)
+//
+// GEMM structure: one CTA per 128 x 128 tile of D, 128 threads.  Warp 0
+// lane 0 is the producer: per K step of 256 elements it loads the A and B
+// tiles (128 rows x 128 bytes each, 2-D TMA with 128-byte swizzle) and the
+// four 512-byte scale tiles of each operand (1-D bulk copies) into one of
+// three shared-memory stages, completing on the stage's "full" mbarrier.
+// Warp 1 lane 0 is the MMA issuer: it copies the scale tiles to tensor
+// memory (tcgen05.cp 32x128b.warpx4), issues four K=64 MMAs and commits
+// them to the stage's "empty" mbarrier, which frees the stage for the
+// producer.  After the last K step a commit to the "done" mbarrier releases
+// all four warps into the epilogue: tcgen05.ld of their 32 accumulator
+// lanes, times g_a g_b, fp32 stores.  Tensor memory: 128 accumulator
+// columns and 32 scale columns per stage (256 allocated; at most two CTAs
+// fit on an SM by shared memory, so allocation never waits).  All mbarrier
+// waits are bounded: on running out the thread records FP4_ERR_TIMEOUT,
+// the waits that depend on it run out in turn, the producer waits (bounded)
+// for its copies, and the tensor memory is freed before the CTA ends.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda.h>
+
+#include "fp4_kernels.cuh"
+#include "fp4_layouts.cuh"
+
+namespace fp4 {
+
+// ---------------------------------------------------------------------------
+// Scale layout for the MMA.  One thread per output 32-bit word: word
+// 4 r0 + r1 of tile t holds blocks 4 (t % kt) .. + 3 of row
+// (t / kt) * 128 + 32 r1 + r0 (kt = ceil(nb / 4) block tiles per row band).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads)
+    scales_to_mma_kernel(const uint8_t *__restrict__ s, int rows, int nb, int kt, int n_words,
+                         uint32_t *__restrict__ out)
+{
+    pdl_begin();
+    const int stride = (int)(gridDim.x * blockDim.x);
+    for (int wi = (int)(blockIdx.x * blockDim.x + threadIdx.x); wi < n_words; wi += stride) {
+        const int tile = wi >> 7;    // 128 words per 512-byte tile
+        const int within = wi & 127; // word 4 r0 + r1 of the tile
+        const int r0 = within >> 2, r1 = within & 3;
+        const int row = (tile / kt) * 128 + r1 * 32 + r0;
+        const int j0 = (tile % kt) * 4;
+        uint32_t v = 0;
+        if (row < rows) {
+            const uint8_t *src = s + (int64_t)row * nb;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (j0 + j < nb)
+                    v |= (uint32_t)__ldcg(src + j0 + j) << (8 * j);
+        }
+        out[wi] = v;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 primitives (sm_100a).
+// ---------------------------------------------------------------------------
+constexpr int kGemmTile = 128;            // M and N of a CTA tile
+constexpr int kGemmKStep = 256;           // elements of K per stage (128 bytes)
+constexpr int kGemmStages = 3;
+constexpr int kGemmOpBytes = kGemmTile * 128;          // one operand tile: 16 KB
+constexpr int kGemmSfBytes = 4 * 512;                  // scale tiles of one operand per K step
+constexpr int kGemmStageBytes = 2 * kGemmOpBytes + 2 * kGemmSfBytes; // 36 KB
+constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + 1024;     // + alignment slack
+constexpr uint32_t kGemmTmemCols = 256;
+
+// Instruction descriptor of tcgen05.mma kind::mxf4nvf4 block16: A and B
+// E2M1 (format 1 in this kind), K-major, UE4M3 scales (format 0), M = 128
+// (bits 24..28 = M / 16), N = 128 (bits 17..22 = N / 8), dense, K = 64.
+constexpr uint32_t kGemmIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kGemmTile / 8) << 17) |
+                                ((uint32_t)(kGemmTile / 16) << 24);
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: rows of 128
+// bytes, 8-row groups 1024 bytes apart (SBO 64 x 16 B), LBO 1, descriptor
+// version 1, layout type 2.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr)
+{
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
+// Shared-memory descriptor of a 512-byte scale tile for tcgen05.cp (32 rows
+// of 16 bytes, K-major without swizzle: 8-row core matrices of 128 bytes,
+// SBO 8 x 16 B), version 1, layout type 0.
+__device__ __forceinline__ uint64_t smem_desc_sf(uint32_t addr)
+{
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | (8ull << 32) | (1ull << 46);
+}
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t cols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)),
+                 "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_copy_sf(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_nvfp4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile("{\n\t"
+                 ".reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+                 "}" ::"r"(d_tmem),
+                 "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+// 32 consecutive accumulator columns of this warp's 32 lanes.
+__device__ __forceinline__ void tc_load_32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+                   "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+                   "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+    // the registers are operands of the wait, so no use moves above it
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
+                   "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+                   "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------
+// The GEMM.  Grid (N / 128, M / 128); map_a / map_b: 2-D uint8 tensor maps of
+// the packed operands ([rows, K/2] bytes, box 128 bytes x 128 rows, 128-byte
+// swizzle); sfa / sfb: the scale tiles of the whole operands in the MMA
+// layout (K/64 tiles per 128-row band).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128, 1)
+    nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                      const uint8_t *__restrict__ sfa, const uint8_t *__restrict__ sfb,
+                      const float *g_a, const float *g_b, int M, int N, int K, float *__restrict__ d,
+                      int32_t *status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kGemmStages], empty[kGemmStages], done;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int consumed_steps; // K steps the MMA issuer waited for
+    // 1024-byte aligned stages (128-byte swizzle atoms)
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+
+    pdl_begin();
+    const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
+    const int bn = (int)blockIdx.x, bm = (int)blockIdx.y;
+    const int kt_steps = K / kGemmKStep;
+    const int sf_tiles_per_band = K / 64; // 4-block scale tiles per 128-row band
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGemmStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&done, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        consumed_steps = 0;
+    }
+    __syncwarp();
+    if (warp == 0)
+        tmem_alloc(&tmem_slot, kGemmTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;      // lane 0, first allocated column
+    const uint32_t tmem_acc = tmem;       // columns [0, 128): the accumulator
+    const uint32_t tmem_sf = tmem + 128;  // 32 columns per stage: 16 for A, 16 for B
+
+    bool timed_out = false;
+    int issued = 0;
+    if (warp == 0 && lane == 0) {
+        // producer
+        for (int k = 0; k < kt_steps; ++k) {
+            const int s = k % kGemmStages;
+            if (k >= kGemmStages && !mbar_wait(&empty[s], (uint32_t)((k / kGemmStages) - 1) & 1u)) {
+                timed_out = true;
+                break;
+            }
+            uint8_t *st = smem + s * kGemmStageBytes;
+            mbar_expect_tx(&full[s], kGemmStageBytes);
+            tma_load_2d(st, &map_a, k * 128, bm * kGemmTile, &full[s]);
+            tma_load_2d(st + kGemmOpBytes, &map_b, k * 128, bn * kGemmTile, &full[s]);
+            const int64_t sf_off = ((int64_t)bm * sf_tiles_per_band + 4 * k) * 512;
+            const int64_t sfb_off = ((int64_t)bn * sf_tiles_per_band + 4 * k) * 512;
+            bulk_load(st + 2 * kGemmOpBytes, sfa + sf_off, kGemmSfBytes, &full[s]);
+            bulk_load(st + 2 * kGemmOpBytes + kGemmSfBytes, sfb + sfb_off, kGemmSfBytes, &full[s]);
+            ++issued;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer
+        for (int k = 0; k < kt_steps; ++k) {
+            const int s = k % kGemmStages;
+            if (!mbar_wait(&full[s], (uint32_t)(k / kGemmStages) & 1u)) {
+                timed_out = true;
+                break;
+            }
+            tc_fence_after();
+            const uint8_t *st = smem + s * kGemmStageBytes;
+            const uint32_t a_addr = smem_addr(st), b_addr = smem_addr(st + kGemmOpBytes);
+            const uint32_t sa_addr = smem_addr(st + 2 * kGemmOpBytes);
+            const uint32_t sb_addr = sa_addr + kGemmSfBytes;
+            const uint32_t sf_cols = tmem_sf + (uint32_t)s * 32;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                tc_copy_sf(sf_cols + 4 * i, smem_desc_sf(sa_addr + 512 * i));
+                tc_copy_sf(sf_cols + 16 + 4 * i, smem_desc_sf(sb_addr + 512 * i));
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) // four MMAs of K = 64 (32 bytes of each 128-byte row)
+                tc_mma_nvfp4(tmem_acc, smem_desc_sw128(a_addr + 32 * i), smem_desc_sw128(b_addr + 32 * i),
+                             kGemmIdesc, sf_cols + 4 * i, sf_cols + 16 + 4 * i, (k | i) != 0);
+            tc_commit(&empty[s]); // frees the stage once these MMAs have read it
+            consumed_steps = k + 1;
+        }
+        tc_commit(&done);
+    }
+    // Everyone: wait for the accumulator (bounded), then the epilogue.
+    const bool ok = mbar_wait(&done, 0);
+    if (!ok || timed_out)
+        raise_status(status, kStatusTimeout);
+    __syncthreads();
+    if (warp == 0 && lane == 0) {
+        // Copies started that the issuer never waited for (only after a
+        // timeout; at most one per stage) must land before the CTA ends.
+        for (int j = consumed_steps; j < issued; ++j)
+            (void)mbar_wait(&full[j % kGemmStages], (uint32_t)(j / kGemmStages) & 1u);
+    }
+    __syncwarp();
+    if (ok) {
+        tc_fence_after();
+        const float gg = __fmul_rn(__ldcg(g_a), __ldcg(g_b));
+        const int row = bm * kGemmTile + warp * 32 + lane;
+        float *drow = d + (int64_t)row * N + (int64_t)bn * kGemmTile;
+#pragma unroll 1
+        for (int c = 0; c < kGemmTile / 32; ++c) {
+            float v[32];
+            tc_load_32(tmem_acc + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 32), v);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                float4 o = make_float4(__fmul_rn(v[4 * q], gg), __fmul_rn(v[4 * q + 1], gg),
+                                       __fmul_rn(v[4 * q + 2], gg), __fmul_rn(v[4 * q + 3], gg));
+                *reinterpret_cast<float4 *>(drow + c * 32 + 4 * q) = o;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0)
+        tmem_dealloc(tmem, kGemmTmemCols);
+}
+
+} // namespace fp4

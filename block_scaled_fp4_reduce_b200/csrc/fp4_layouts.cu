@@ -3,7 +3,6 @@
 // tensor map of the column-wise pass, and the launches.
 #include <climits>
 #include <cstdint>
-#include <mutex>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -85,30 +84,6 @@ fp4_status dq_padded(const uint8_t *packed, const uint8_t *scales, const float *
 }
 
 // ----------------------------------------------------------- column-wise --
-
-using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                 const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                 const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
-// against the driver library).
-EncodeTiled encode_tiled()
-{
-    static std::once_flag once;
-    static EncodeTiled fn = nullptr;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiled>(p);
-        else
-            (void)cudaGetLastError();
-    });
-    return fn;
-}
 
 // Tensor map of W [rows, cols] (innermost: cols), box 512 bytes x 64 rows,
 // no swizzle, zero fill out of bounds.

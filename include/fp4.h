@@ -288,6 +288,41 @@ fp4_status fp4_mxfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t ro
                                       int32_t *status, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The consumer on the tensor cores ("NVFP4 与 MXFP4 格式" section 6: with
+ * both operands of Y = X W blocked along K, an output is g_X g_W times the
+ * sum over blocks of s_X s_W times the block's payload dot product).
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of the MMA scale layout of a [rows, blocks] scale matrix:
+ * ceil(rows/128) * 128 * ceil(blocks/4) * 4. */
+size_t fp4_mma_scales_bytes(int64_t rows, int64_t blocks);
+
+/* Block scales [rows, blocks] (one byte per 16-block, row-major, as the
+ * quantisers write them) -> the tiled layout the sm100 block-scaled MMA
+ * reads (not on the pages): 128-row x 4-block tiles of 512 bytes, row-band
+ * major with the block tiles of a band contiguous; inside a tile row r = r0
+ * + 32 r1 (r0 < 32) and block j (< 4) at byte 16 r0 + 4 r1 + j; rows and
+ * blocks past the matrix are 0.  out: fp4_mma_scales_bytes bytes, 4-byte
+ * aligned.  One kernel. */
+fp4_status fp4_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t blocks, uint8_t *out,
+                                    cudaStream_t stream);
+
+/* D [M, N] fp32 row-major = g_a g_b A B^T on the tensor cores (tcgen05.mma
+ * kind::mxf4nvf4, 16-element blocks, E4M3 scales, fp32 accumulation in
+ * tensor memory).  A: packed [M, K/2] with scales_a_mma = the MMA layout of
+ * its [M, K/16] scales; B: packed [N, K/2] (the K-grouping of a K x N
+ * weight stored N x K) with scales_b_mma; global scales as the quantisers
+ * write them.  M and N multiples of 128, K a multiple of 256 (else
+ * FP4_ERR_SHAPE); packed, scales and d 16-byte aligned.  One kernel, one
+ * CTA per 128 x 128 tile of D; a copy that never completes ends the kernel
+ * with FP4_ERR_TIMEOUT in *status.  The accumulation order inside the
+ * tensor core is the hardware's: D agrees with the exact product to fp32
+ * accumulation accuracy, not bit for bit. */
+fp4_status fp4_nvfp4_gemm(const uint8_t *packed_a, const uint8_t *scales_a_mma, const float *global_scale_a,
+                          const uint8_t *packed_b, const uint8_t *scales_b_mma, const float *global_scale_b,
+                          int64_t M, int64_t N, int64_t K, float *d, int32_t *status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Grouped calls: many matrices per call, each with its own scales.
  *
  * The global scale is a per-tensor quantity ("NVFP4 与 MXFP4 格式" section 3:

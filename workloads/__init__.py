@@ -70,6 +70,16 @@ VARIANTS_8K = Workload("variants-8192x14336-bf16", 8192, 14336, torch.bfloat16, 
                        std=0.5, description="bf16 8192x14336 Student-t(nu=3) x0.5, seed 7; MXFP4 ceil rule "
                                             "and NVFP4 four over six")
 
+# The consumer: an activation of 8192 tokens x 14336 features (as the
+# activation workload) times the 4096 x 14336 down-projection weight of the
+# weight set, both NVFP4 along K = 14336.
+GEMM_ACT = Workload("gemm-8192x4096x14336-nvfp4", 8192, 14336, torch.bfloat16, 8, "student-t",
+                    std=0.5, description="D [8192, 4096] = A [8192, 14336] x W^T, W [4096, 14336]: A bf16 "
+                                         "Student-t(nu=3) x0.5 seed 8 quantised each step, W N(0,0.02) 0.05% x30 "
+                                         "seed 9 quantised once")
+GEMM_W = Workload("gemm-weight-4096x14336", 4096, 14336, torch.bfloat16, 9, "normal-outliers",
+                  std=0.02, out_frac=0.0005, out_mult=30.0)
+
 # The 7B-class weight set: per layer 4 square 4096x4096 and 3 4096x14336.
 MODEL_LAYERS = 32
 MODEL_MATRICES = [(4096, 4096)] * 4 + [(4096, 14336)] * 3
