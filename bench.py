@@ -23,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -227,11 +228,11 @@ class GroupedPath:
     OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize"]
     LAUNCHES = 5
 
-    def __init__(self, device, rank: int = 0):
+    def __init__(self, device, rank: int = 0, layers: int = workloads.MODEL_LAYERS):
         import block_scaled_fp4_reduce_b200 as fp4
         self.fp4 = fp4
         L = fp4.lib()
-        self.ws_list = [workloads.model_matrix(l, i) for l in range(workloads.MODEL_LAYERS)
+        self.ws_list = [workloads.model_matrix(l, i) for l in range(layers)
                         for i in range(len(workloads.MODEL_MATRICES))]
         if rank:
             self.ws_list = [workloads.for_rank(w, rank) for w in self.ws_list]
@@ -431,7 +432,10 @@ def run_ours(args, rank: int, world: int, local: int):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     w = workloads.for_rank(WORKLOADS[args.workload], rank)
     if args.workload == MODEL_WEIGHTS:
-        path = GroupedPath(dev, rank)
+        path = GroupedPath(dev, rank, args.model_layers)
+        if args.model_layers != workloads.MODEL_LAYERS:  # a profiling-sized subset of the set
+            w = dataclasses.replace(w, rows=path.n // w.cols,
+                                    name=f"{w.name}@{args.model_layers}-layers")
         x = path.x
         x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
         x_host.copy_(x)
@@ -540,7 +544,14 @@ def run_ours(args, rank: int, world: int, local: int):
     gemm_mnk = (path.M, path.N, path.K) if args.workload == GEMM_WORKLOAD else None
     if gemm_mnk:
         dom = "nvfp4_gemm"  # the tensor-core kernel is the one this workload is about
-    roof = roofline_for(dom, kernels[dom], w, pk, n_cand, gemm_mnk)
+    if LAYOUT_WORKLOADS.get(args.workload) == "variants" and dom == "nvfp4_quantize":
+        # four over six: two screened candidates per block, ALU-bound like the search
+        n_cand = 2 * (w.numel // 16)
+        roof = roofline_for("scale_search", kernels[dom], w, pk, n_cand)
+        roof["kernel"] = "nvfp4_quantize_four_over_six"
+        roof["work"] = roof["work"].replace("distinct candidates", "candidates (2 per block)")
+    else:
+        roof = roofline_for(dom, kernels[dom], w, pk, n_cand, gemm_mnk)
     line = {
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": K,
         "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
@@ -776,6 +787,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--model-layers", type=int, default=workloads.MODEL_LAYERS,
+                    help="layers of the 7B weight set in model-7b-weights-bf16 (fewer only for profiler runs)")
     ap.add_argument("--flush-mib", type=int, default=512,
                     help="L2 flush size between steps (0 = no flush, for profiler runs only)")
     args = ap.parse_args()
