@@ -27,6 +27,8 @@ OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_RANGE, ERR_WORKSPA
 F32, BF16 = 0, 1
 NVFP4, MXFP4 = 0, 1
 MX_FLOOR, MX_CEIL = 0, 1
+# fp4_gemm_kernel
+GEMM_AUTO, GEMM_CTA, GEMM_CTA_PAIR = 0, 1, 2
 
 _lib = None
 
@@ -76,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "fp4_mma_scales_bytes": (SZ, [I64, I64]),
             "fp4_scales_to_mma_layout": (I, [P, I64, I64, P, P]),
             "fp4_nvfp4_gemm": (I, [P, P, P, P, P, P, I64, I64, I64, P, P, P]),
+            "fp4_nvfp4_gemm_ex": (I, [P, P, P, P, P, P, I64, I64, I64, P, I, P, P]),
             "fp4_nvfp4_quantize_padded": (I, [P, I, I64, I64, P, P, P, P, SZ, P, P]),
             "fp4_mxfp4_quantize_padded": (I, [P, I, I64, I64, I, P, P, P, P]),
             "fp4_dequantize_padded": (I, [I, P, P, P, I64, I64, P, I, P]),
@@ -467,9 +470,11 @@ def scales_to_mma(scales: torch.Tensor, stream=None) -> torch.Tensor:
     return out
 
 
-def nvfp4_gemm(qa: Quantized, qb: Quantized, out=None, status=None, stream=None) -> torch.Tensor:
+def nvfp4_gemm(qa: Quantized, qb: Quantized, out=None, status=None, stream=None,
+               kernel: int = GEMM_AUTO) -> torch.Tensor:
     """D [M, N] fp32 = g_a g_b A B^T on the tensor cores for NVFP4 A [M, K]
-    and B [N, K] (M, N multiples of 128, K of 256)."""
+    and B [N, K] (M, N multiples of 128, K of 256; GEMM_CTA_PAIR needs M, N
+    multiples of 256)."""
     if qa.fmt != NVFP4 or qb.fmt != NVFP4 or qa.cols != qb.cols:
         raise ValueError("two NVFP4 operands with the same K required")
     M, N, K = qa.rows, qb.rows, qa.cols
@@ -477,8 +482,9 @@ def nvfp4_gemm(qa: Quantized, qb: Quantized, out=None, status=None, stream=None)
     d = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=dev)
     st = status if status is not None else new_status(dev)
     sa, sb = scales_to_mma(qa.scales, stream), scales_to_mma(qb.scales, stream)
-    _check(lib().fp4_nvfp4_gemm(_p(qa.packed), _p(sa), _p(qa.global_scale), _p(qb.packed), _p(sb),
-                                _p(qb.global_scale), M, N, K, _p(d), _p(st), _stream(stream)), "fp4_nvfp4_gemm")
+    _check(lib().fp4_nvfp4_gemm_ex(_p(qa.packed), _p(sa), _p(qa.global_scale), _p(qb.packed), _p(sb),
+                                   _p(qb.global_scale), M, N, K, _p(d), kernel, _p(st), _stream(stream)),
+           "fp4_nvfp4_gemm_ex")
     return d
 
 

@@ -36,6 +36,124 @@ fp4_status operand_map(const uint8_t *p, int64_t rows, int64_t K, CUtensorMap *m
     return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
 }
 
+// 2-D tensor map of an MMA scale layout viewed as uint32 [tiles, 128] (one
+// 512-byte tile per row; rows / 128 bands of K / 64 tiles): box 128 x 4, the
+// four tiles of one 256-element K step of one band.
+fp4_status scale_map(const uint8_t *sf, int64_t rows, int64_t K, CUtensorMap *map)
+{
+    EncodeTiled enc = encode_tiled();
+    if (!enc)
+        return FP4_ERR_CUDA;
+    const cuuint64_t dims[2] = {128u, (cuuint64_t)((rows / 128) * (K / 64))};
+    const cuuint64_t strides[1] = {512u};
+    const cuuint32_t box[2] = {128u, 4u};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t *>(sf), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
+}
+
+bool set_smem_attr(const void *kernel, int bytes, bool (&done)[kMaxDevices], int dev)
+{
+    if (done[dev])
+        return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    done[dev] = true;
+    return true;
+}
+
+// 2-D tensor map of D [M, N] fp32: box 32 x 32 with 128-byte swizzle (the
+// pair kernel's epilogue staging tiles).
+fp4_status out_map(float *d, int64_t M, int64_t N, CUtensorMap *map)
+{
+    EncodeTiled enc = encode_tiled();
+    if (!enc)
+        return FP4_ERR_CUDA;
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)N * 4u};
+    const cuuint32_t box[2] = {32u, 32u};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, d, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
+}
+
+// Clusters of two CTAs of the pair kernel that fit on the device at once.
+int pair_clusters(int dev)
+{
+    static int cached[kMaxDevices] = {0};
+    if (cached[dev] > 0)
+        return cached[dev];
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * 74);
+    cfg.blockDim = dim3(fp4::kPairThreads);
+    cfg.dynamicSmemBytes = fp4::kPairSmem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fp4::nvfp4_gemm_pair_kernel, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    cached[dev] = n;
+    return n;
+}
+
+fp4_status launch_pair(const uint8_t *packed_a, const uint8_t *sfa, const float *g_a, const uint8_t *packed_b,
+                       const uint8_t *sfb, const float *g_b, int64_t M, int64_t N, int64_t K, float *d,
+                       int32_t *status, cudaStream_t stream, int dev)
+{
+    static bool attr_set[kMaxDevices] = {false};
+    if (!set_smem_attr((const void *)fp4::nvfp4_gemm_pair_kernel, fp4::kPairSmem, attr_set, dev))
+        return FP4_ERR_CUDA;
+    const int clusters = pair_clusters(dev);
+    if (clusters <= 0)
+        return FP4_ERR_CUDA;
+    CUtensorMap map_a, map_b, map_sfa, map_sfb, map_d;
+    std::memset(&map_a, 0, sizeof(map_a));
+    std::memset(&map_b, 0, sizeof(map_b));
+    std::memset(&map_sfa, 0, sizeof(map_sfa));
+    std::memset(&map_sfb, 0, sizeof(map_sfb));
+    std::memset(&map_d, 0, sizeof(map_d));
+    fp4_status st;
+    if ((st = operand_map(packed_a, M, K, &map_a)) != FP4_OK || (st = operand_map(packed_b, N, K, &map_b)) != FP4_OK ||
+        (st = scale_map(sfa, M, K, &map_sfa)) != FP4_OK || (st = scale_map(sfb, N, K, &map_sfb)) != FP4_OK ||
+        (st = out_map(d, M, N, &map_d)) != FP4_OK)
+        return st;
+    const int64_t tiles = (M / fp4::kPairTileM) * (N / fp4::kPairTileN);
+    const int64_t pairs = tiles < clusters ? tiles : clusters;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(fp4::kPairThreads);
+    cfg.dynamicSmemBytes = fp4::kPairSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, fp4::nvfp4_gemm_pair_kernel, map_a, map_b, map_sfa, map_sfb, map_d, g_a, g_b,
+                           (int)M, (int)N, (int)K, status) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return FP4_ERR_CUDA;
+    }
+    return FP4_OK;
+}
+
 } // namespace
 
 extern "C" {
@@ -72,10 +190,24 @@ fp4_status fp4_nvfp4_gemm(const uint8_t *packed_a, const uint8_t *scales_a_mma, 
                           const uint8_t *packed_b, const uint8_t *scales_b_mma, const float *global_scale_b,
                           int64_t M, int64_t N, int64_t K, float *d, int32_t *status, cudaStream_t stream)
 {
-    if (M < 0 || N < 0 || K < 0 || !status)
+    return fp4_nvfp4_gemm_ex(packed_a, scales_a_mma, global_scale_a, packed_b, scales_b_mma, global_scale_b, M, N, K,
+                             d, FP4_GEMM_AUTO, status, stream);
+}
+
+fp4_status fp4_nvfp4_gemm_ex(const uint8_t *packed_a, const uint8_t *scales_a_mma, const float *global_scale_a,
+                             const uint8_t *packed_b, const uint8_t *scales_b_mma, const float *global_scale_b,
+                             int64_t M, int64_t N, int64_t K, float *d, fp4_gemm_kernel kernel, int32_t *status,
+                             cudaStream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || !status ||
+        (kernel != FP4_GEMM_AUTO && kernel != FP4_GEMM_CTA && kernel != FP4_GEMM_CTA_PAIR))
         return FP4_ERR_INVALID_ARG;
     if (M % fp4::kGemmTile || N % fp4::kGemmTile || K % fp4::kGemmKStep || M > INT_MAX || N > INT_MAX ||
         K > INT_MAX)
+        return FP4_ERR_SHAPE;
+    const bool pair_shape = M % fp4::kPairTileM == 0 && N % fp4::kPairTileN == 0 && (M / 128) * (K / 64) <= INT_MAX &&
+                            (N / 128) * (K / 64) <= INT_MAX;
+    if (kernel == FP4_GEMM_CTA_PAIR && !pair_shape)
         return FP4_ERR_SHAPE;
     if (M == 0 || N == 0)
         return FP4_OK;
@@ -92,18 +224,23 @@ fp4_status fp4_nvfp4_gemm(const uint8_t *packed_a, const uint8_t *scales_a_mma, 
         }
         return FP4_OK;
     }
-    static bool attr_set[kMaxDevices] = {false};
     int dev = 0;
-    if (sm_count(dev) <= 0 || dev >= kMaxDevices)
+    const int sms = sm_count(dev);
+    if (sms <= 0 || dev >= kMaxDevices)
         return FP4_ERR_CUDA;
-    if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(fp4::nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 fp4::kGemmSmem) != cudaSuccess) {
-            (void)cudaGetLastError();
-            return FP4_ERR_CUDA;
-        }
-        attr_set[dev] = true;
-    }
+    // The pair kernel once its 256 x 256 tiles give every SM pair work and K
+    // is short enough that its persistent epilogue overlap pays; for long K
+    // the one-CTA kernel's deeper copy pipeline per SM (two CTAs x three
+    // stages) wins (measured on B200: 8192^3 3.08 against 2.86 PFLOP/s,
+    // 8192 x 4096 x 14336 3.15 against 3.23).
+    if (kernel == FP4_GEMM_CTA_PAIR ||
+        (kernel == FP4_GEMM_AUTO && pair_shape && K <= 8192 &&
+         (M / fp4::kPairTileM) * (N / fp4::kPairTileN) >= sms / 2))
+        return launch_pair(packed_a, scales_a_mma, global_scale_a, packed_b, scales_b_mma, global_scale_b, M, N, K, d,
+                           status, stream, dev);
+    static bool attr_set[kMaxDevices] = {false};
+    if (!set_smem_attr((const void *)fp4::nvfp4_gemm_kernel, fp4::kGemmSmem, attr_set, dev))
+        return FP4_ERR_CUDA;
     CUtensorMap map_a, map_b;
     std::memset(&map_a, 0, sizeof(map_a));
     std::memset(&map_b, 0, sizeof(map_b));

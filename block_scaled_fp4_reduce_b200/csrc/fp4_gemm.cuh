@@ -355,4 +355,370 @@ __global__ void __launch_bounds__(128, 1)
         tmem_dealloc(tmem, kGemmTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// The GEMM on CTA pairs: tcgen05 cta_group::2, persistent.
+//
+// A 128 x 128 tile per SM reads 32 KB of operands from shared memory per
+// 8.4 MFLOP.  Two SMs of a cluster pair computing one 256 x 256 tile of D
+// with one MMA stream (M = 256, N = 256) read the same bytes per SM for
+// twice the flops: each SM holds 128 rows of A and 128 rows of B, the
+// pair's tensor cores read both halves.
+//
+// Roles (320 threads per CTA): warp 0 of both CTAs loads (2-D TMA, 128-byte
+// swizzle) this CTA's 128 rows of A and of B and the scale tiles (its own
+// 128 rows of A's, all 256 rows of B's) into a five-stage ring; every copy
+// completes on the leader CTA's "full" barrier, so the leader sees the
+// stage of both CTAs arrive.  Warp 1 of the leader issues: scale tiles to
+// tensor memory (tcgen05.cp, which reaches the same columns of both CTAs),
+// four K = 64 MMAs per stage, and a commit that arrives on the "empty"
+// barrier of the stage in both CTAs.  After a tile's last stage a commit
+// arrives on "acc_full" in both CTAs.  Warps 2..9 of both CTAs drain the
+// accumulator: each reads its 32 lanes (warp % 4) and one 128-column half
+// into registers, releases the accumulator (an arrival on the leader's
+// "acc_empty", 16 per tile), and only then scales and stores -- through a
+// swizzled 32 x 32 staging tile and a TMA store -- so the next tile's MMAs
+// run while the stores drain.  The grid is persistent: cluster p takes
+// tiles p, p + P, ... (M-tile fastest).  Tensor memory (512 columns,
+// allocated by the pair): the accumulator in columns 0..255, then a ring of
+// four scale column sets (16 for A, 32 for B).  All waits are bounded; on
+// running out a warp records FP4_ERR_TIMEOUT and leaves its loop, the waits
+// that depend on it run out in turn, the leader waits (bounded) for copies
+// nobody consumed and for its MMAs, and both CTAs free the tensor memory
+// together.
+// ---------------------------------------------------------------------------
+constexpr int kPairTileM = 256;
+constexpr int kPairTileN = 256;
+constexpr int kPairStages = 5;
+constexpr int kPairSfaBytes = 4 * 512; // this CTA's 128 rows of A: four 4-block scale tiles
+constexpr int kPairSfbBytes = 8 * 512; // both 128-row bands of the B tile
+constexpr int kPairStageBytes = 2 * kGemmOpBytes + kPairSfaBytes + kPairSfbBytes; // 38 KB
+constexpr int kPairOutBytes = 32 * 32 * 4; // one epilogue staging tile
+constexpr int kPairEpiWarps = 8;
+constexpr int kPairThreads = 320;
+constexpr int kPairOutOffset = kPairStages * kPairStageBytes;
+constexpr int kPairSmem = kPairOutOffset + kPairEpiWarps * kPairOutBytes + 1024;
+constexpr uint32_t kPairSfCols = 16 + 32; // A: 4 columns per MMA; B (256 rows): 8
+constexpr uint32_t kPairSfRing = 4;
+constexpr uint32_t kPairTmemCols = 512;
+static_assert(kPairTileN + kPairSfRing * kPairSfCols <= kPairTmemCols, "tensor memory");
+static_assert(kPairStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
+static_assert(kPairSmem <= 232448 - 512, "shared memory");
+// M = 256 (bits 24..28 = M / 16), N = 256 (bits 17..22 = N / 8), E2M1 x E2M1,
+// UE4M3 scales, K-major, dense.
+constexpr uint32_t kPairIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kPairTileN / 8) << 17) |
+                                ((uint32_t)(kPairTileM / 16) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank)
+{
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_addr(p)), "r"(rank));
+    return a;
+}
+
+// Every thread of both CTAs (release / acquire).
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+
+__device__ __forceinline__ int ld_cluster_s32(uint32_t cl_addr)
+{
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cl_addr) : "memory");
+    return v;
+}
+
+// 2-D TMA load into this CTA's shared memory, completing on a barrier of
+// either CTA of the pair (bar_cl: a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, int x, int y, uint32_t bar_cl)
+{
+    asm volatile("cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cl)
+                 : "memory");
+}
+
+// 2-D TMA store of a shared-memory box to (x = column, y = row); bulk group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_addr(src))
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// This thread's bulk stores have read their shared memory / have finished.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot, uint32_t cols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)),
+                 "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t cols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
+// Scale tile of each CTA's shared memory into the same columns of each
+// CTA's tensor memory.
+__device__ __forceinline__ void tc_copy_sf_pair(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_nvfp4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile("{\n\t"
+                 ".reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+                 "}" ::"r"(d_tmem),
+                 "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+                 : "memory");
+}
+
+// Arrive on the barrier at this offset in both CTAs once the issued
+// tcgen05 operations are done.
+__device__ __forceinline__ void tc_commit_both(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                     smem_addr(bar)),
+                 "h"((uint16_t)0x3)
+                 : "memory");
+}
+
+// Arrive on this CTA's barrier only.
+__device__ __forceinline__ void tc_commit_own(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// map_a / map_b: the packed operands as in nvfp4_gemm_kernel.  map_sfa /
+// map_sfb: the MMA scale layouts viewed as uint32 [tiles, 128] (one 512-byte
+// tile per row, K/64 tiles per 128-row band), box 128 x 4: one K step of
+// one band.  map_d: D fp32, box 32 x 32, 128-byte swizzle.  M and N
+// multiples of 256, K of 256; grid = 2 x pairs, cluster 2.
+__global__ void __launch_bounds__(kPairThreads, 1)
+    nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                           const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
+                           const __grid_constant__ CUtensorMap map_d, const float *g_a, const float *g_b, int M, int N,
+                           int K, int32_t *status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kPairStages], empty[kPairStages], acc_full, acc_empty, mma_done;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int issued_steps, consumed_steps;
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+
+    pdl_begin();
+    const int warp = (int)threadIdx.x >> 5, lane = (int)threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = (int)blockIdx.x >> 1, n_pairs = (int)gridDim.x >> 1;
+    const int tiles_m = M / kPairTileM;
+    const int n_tiles = tiles_m * (N / kPairTileN);
+    const int kt_steps = K / kGemmKStep;
+    const int sf_tiles_per_band = K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(&acc_full, 1);
+        mbar_init(&acc_empty, 2 * kPairEpiWarps);
+        mbar_init(&mma_done, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        issued_steps = 0;
+        consumed_steps = 0;
+    }
+    __syncwarp();
+    if (warp == 0)
+        tmem_alloc_pair(&tmem_slot, kPairTmemCols);
+    tc_fence_before();
+    cluster_sync(); // both CTAs' barriers initialised before any remote arrival
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+
+    bool timed_out = false;
+    if (warp == 0) {
+        // producer, both CTAs
+        int it = 0;
+        for (int t = pair; t < n_tiles && !timed_out; t += n_pairs) {
+            const int tm = t % tiles_m, tn = t / tiles_m;
+            for (int k = 0; k < kt_steps; ++k, ++it) {
+                const int s = it % kPairStages;
+                if (it >= kPairStages &&
+                    !__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], (uint32_t)((it / kPairStages) - 1) & 1u))) {
+                    timed_out = true;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t *st = smem + s * kPairStageBytes;
+                    uint8_t *sf = st + 2 * kGemmOpBytes;
+                    const uint32_t bar = cluster_addr(&full[s], 0);
+                    if (leader)
+                        mbar_expect_tx(&full[s], 2u * kPairStageBytes); // both CTAs' copies
+                    tma_load_2d_pair(st, &map_a, k * 128, tm * kPairTileM + (int)rank * kGemmTile, bar);
+                    tma_load_2d_pair(st + kGemmOpBytes, &map_b, k * 128, tn * kPairTileN + (int)rank * kGemmTile, bar);
+                    tma_load_2d_pair(sf, &map_sfa, 0, (tm * 2 + (int)rank) * sf_tiles_per_band + 4 * k, bar);
+                    tma_load_2d_pair(sf + kPairSfaBytes, &map_sfb, 0, (tn * 2) * sf_tiles_per_band + 4 * k, bar);
+                    tma_load_2d_pair(sf + kPairSfaBytes + 4 * 512, &map_sfb, 0,
+                                     (tn * 2 + 1) * sf_tiles_per_band + 4 * k, bar);
+                    issued_steps = it + 1;
+                }
+                __syncwarp();
+            }
+        }
+        // The last release of every stage (a commit arriving on this CTA's
+        // empty barrier) lands before the CTA can end.
+        for (int j = it - kPairStages > 0 ? it - kPairStages : 0; j < it; ++j)
+            (void)mbar_wait(&empty[j % kPairStages], (uint32_t)(j / kPairStages) & 1u);
+    } else if (warp == 1) {
+        if (leader) {
+            // MMA issuer
+            int it = 0, j = 0;
+            for (int t = pair; t < n_tiles; t += n_pairs, ++j) {
+                if (j > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&acc_empty, (uint32_t)(j - 1) & 1u))) {
+                    timed_out = true;
+                    break;
+                }
+                tc_fence_after();
+                for (int k = 0; k < kt_steps; ++k, ++it) {
+                    const int s = it % kPairStages;
+                    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (uint32_t)(it / kPairStages) & 1u))) {
+                        timed_out = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t a_addr = smem_addr(smem + s * kPairStageBytes);
+                        const uint32_t b_addr = a_addr + kGemmOpBytes;
+                        const uint32_t sfa_addr = a_addr + 2 * kGemmOpBytes;
+                        const uint32_t sfb_addr = sfa_addr + kPairSfaBytes;
+                        const uint32_t sfa_t = tmem + kPairTileN + (uint32_t)(it % kPairSfRing) * kPairSfCols;
+                        const uint32_t sfb_t = sfa_t + 16;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            tc_copy_sf_pair(sfa_t + 4 * i, smem_desc_sf(sfa_addr + 512 * i));
+                        // B's scales for MMA i: rows 0..127 in columns 8i..8i+3,
+                        // rows 128..255 in 8i+4..8i+7
+#pragma unroll
+                        for (int b = 0; b < 2; ++b)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                tc_copy_sf_pair(sfb_t + 8 * i + 4 * b, smem_desc_sf(sfb_addr + 512 * (4 * b + i)));
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) // four MMAs of K = 64 (32 bytes of each 128-byte row)
+                            tc_mma_nvfp4_pair(tmem, smem_desc_sw128(a_addr + 32 * i), smem_desc_sw128(b_addr + 32 * i),
+                                              kPairIdesc, sfa_t + 4 * i, sfb_t + 8 * i, (k | i) != 0);
+                        tc_commit_both(&empty[s]); // frees the stage in both CTAs
+                        consumed_steps = it + 1;
+                    }
+                    __syncwarp();
+                }
+                if (timed_out)
+                    break;
+                if (lane == 0)
+                    tc_commit_both(&acc_full);
+                __syncwarp();
+            }
+            // the epilogues have read the last accumulator
+            if (!timed_out && j > 0 &&
+                !__all_sync(0xFFFFFFFFu, mbar_wait(&acc_empty, (uint32_t)(j - 1) & 1u)))
+                timed_out = true;
+            // every MMA issued has finished before tensor memory is freed
+            if (lane == 0)
+                tc_commit_own(&mma_done);
+            __syncwarp();
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&mma_done, 0)))
+                timed_out = true;
+        }
+    } else {
+        // epilogue, both CTAs: lanes of warp % 4, columns 128 h .. 128 h + 127
+        const int q = warp & 3, h = (warp - 2) >> 2;
+        const float gg = __fmul_rn(__ldcg(g_a), __ldcg(g_b));
+        const uint32_t release = cluster_addr(&acc_empty, 0);
+        uint8_t *stg = smem + kPairOutOffset + (warp - 2) * kPairOutBytes;
+        int j = 0;
+        for (int t = pair; t < n_tiles; t += n_pairs, ++j) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full, (uint32_t)j & 1u))) {
+                timed_out = true;
+                break;
+            }
+            tc_fence_after();
+            float v[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                tc_load_32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128 + c * 32), v[c]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(release); // the accumulator may be overwritten now
+            const int tm = t % tiles_m, tn = t / tiles_m;
+            const int row0 = tm * kPairTileM + (int)rank * kGemmTile + q * 32;
+            // 32 x 32 chunks through this warp's staging tile: lane l writes
+            // row l, its 16-byte unit u at unit u ^ (l % 8) (the 128-byte
+            // swizzle; eight lanes cover all banks), then lane 0 stores the
+            // tile with TMA once the previous store has read it.
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (lane == 0)
+                    bulk_wait_read();
+                __syncwarp();
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<float4 *>(stg + lane * 128 + 16 * (u ^ (lane & 7))) =
+                        make_float4(__fmul_rn(v[c][4 * u], gg), __fmul_rn(v[c][4 * u + 1], gg),
+                                    __fmul_rn(v[c][4 * u + 2], gg), __fmul_rn(v[c][4 * u + 3], gg));
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0)
+                    tma_store_2d(&map_d, stg, tn * kPairTileN + h * 128 + c * 32, row0);
+            }
+        }
+        if (lane == 0)
+            bulk_wait_all(); // the stores have finished before the CTA ends
+    }
+    if (timed_out)
+        raise_status(status, kStatusTimeout);
+
+    tc_fence_before();
+    cluster_sync(); // every role of both CTAs is done
+    if (leader && warp == 0) {
+        // After a timeout only: copies of either CTA that the MMA warp never
+        // waited for complete on the leader's full barriers; wait (bounded).
+        const int peer_issued = ld_cluster_s32(cluster_addr(&issued_steps, 1));
+        const int last = issued_steps > peer_issued ? issued_steps : peer_issued;
+        for (int j = consumed_steps; j < last; ++j)
+            (void)mbar_wait(&full[j % kPairStages], (uint32_t)(j / kPairStages) & 1u);
+    }
+    cluster_sync(); // the peer stays until the leader's drain is done
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kPairTmemCols);
+    }
+}
+
 } // namespace fp4

@@ -313,14 +313,34 @@ fp4_status fp4_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t
  * its [M, K/16] scales; B: packed [N, K/2] (the K-grouping of a K x N
  * weight stored N x K) with scales_b_mma; global scales as the quantisers
  * write them.  M and N multiples of 128, K a multiple of 256 (else
- * FP4_ERR_SHAPE); packed, scales and d 16-byte aligned.  One kernel, one
- * CTA per 128 x 128 tile of D; a copy that never completes ends the kernel
- * with FP4_ERR_TIMEOUT in *status.  The accumulation order inside the
- * tensor core is the hardware's: D agrees with the exact product to fp32
- * accumulation accuracy, not bit for bit. */
+ * FP4_ERR_SHAPE); packed, scales and d 16-byte aligned.  One kernel: the
+ * CTA-pair kernel (below) when M and N are multiples of 256, K <= 8192 and
+ * its 256 x 256 tiles number at least half the SMs, else one CTA per 128 x
+ * 128 tile.
+ * A copy that never completes ends the kernel with FP4_ERR_TIMEOUT in
+ * *status.  The accumulation order inside the tensor core is the
+ * hardware's: D agrees with the exact product to fp32 accumulation
+ * accuracy, not bit for bit. */
 fp4_status fp4_nvfp4_gemm(const uint8_t *packed_a, const uint8_t *scales_a_mma, const float *global_scale_a,
                           const uint8_t *packed_b, const uint8_t *scales_b_mma, const float *global_scale_b,
                           int64_t M, int64_t N, int64_t K, float *d, int32_t *status, cudaStream_t stream);
+
+/* Which GEMM kernel fp4_nvfp4_gemm_ex runs. */
+typedef enum fp4_gemm_kernel {
+    FP4_GEMM_AUTO = 0,    /* the choice fp4_nvfp4_gemm makes */
+    FP4_GEMM_CTA = 1,     /* one CTA per 128 x 128 tile of D (cta_group::1) */
+    FP4_GEMM_CTA_PAIR = 2 /* persistent, one cluster of two CTAs per 256 x 256
+                             tile at a time (cta_group::2, M = N = 256 MMAs);
+                             M and N multiples of 256, else FP4_ERR_SHAPE */
+} fp4_gemm_kernel;
+
+/* fp4_nvfp4_gemm with the kernel named (FP4_ERR_INVALID_ARG for an unknown
+ * value).  Both kernels compute the same sums; the order of the fp32
+ * accumulation inside the tensor core may differ between them. */
+fp4_status fp4_nvfp4_gemm_ex(const uint8_t *packed_a, const uint8_t *scales_a_mma, const float *global_scale_a,
+                             const uint8_t *packed_b, const uint8_t *scales_b_mma, const float *global_scale_b,
+                             int64_t M, int64_t N, int64_t K, float *d, fp4_gemm_kernel kernel, int32_t *status,
+                             cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Grouped calls: many matrices per call, each with its own scales.

@@ -42,19 +42,25 @@ def operand(rows, K, codes_rows, scale_rows):
     return p, s
 
 
-def run_gemm(pa, sa, ga, pb, sb, gb, M, N, K):
+def run_gemm(pa, sa, ga, pb, sb, gb, M, N, K, kernel=fp4.GEMM_AUTO):
     qa = fp4.Quantized(fp4.NVFP4, torch.from_numpy(pa).to(DEV), torch.from_numpy(sa).to(DEV),
                        torch.tensor([ga], dtype=torch.float32, device=DEV), fp4.new_status(DEV), M, K)
     qb = fp4.Quantized(fp4.NVFP4, torch.from_numpy(pb).to(DEV), torch.from_numpy(sb).to(DEV),
                        torch.tensor([gb], dtype=torch.float32, device=DEV), fp4.new_status(DEV), N, K)
     st = fp4.new_status(DEV)
-    d = fp4.nvfp4_gemm(qa, qb, status=st)
+    d = fp4.nvfp4_gemm(qa, qb, status=st, kernel=kernel)
     torch.cuda.synchronize()
     assert st.item() == 0
     return d.cpu().numpy()
 
 
-def test_grouped_dot_of_the_page_on_the_tensor_cores():
+@pytest.mark.parametrize("kernel,size", [(fp4.GEMM_CTA, 128), (fp4.GEMM_CTA_PAIR, 256)])
+@pytest.mark.parametrize("where", ["first", "last"])
+def test_grouped_dot_of_the_page_on_the_tensor_cores(kernel, size, where):
+    """The page's worked group (two 16-element blocks) as one row of A and
+    one row of B; every other element is zero, so D holds the group's value
+    at one place and zeros elsewhere.  "last" puts it in the last row of A
+    and of B (the second CTA of a pair, the second half of its columns)."""
     gd = golden("grouped_dot.json")
     def codes(spec):
         out = []
@@ -62,18 +68,27 @@ def test_grouped_dot_of_the_page_on_the_tensor_cores():
             out += [oracle.e2m1_encode(value)] * count
         return out
     e4 = oracle.e4m3_encode
-    M = N = 128
+    M = N = size
     K = 256
     pa, sa = operand(M, K, [codes(gd["px"])], [[e4(v) for v in gd["bx"]]])
     pb, sb = operand(N, K, [codes(gd["pw"])], [[e4(v) for v in gd["bw"]]])
-    d = run_gemm(pa, sa, gd["ax"], pb, sb, gd["aw"], M, N, K)
-    assert d[0, 0] == gd["group_result"]
-    d[0, 0] = 0.0
+    r = 0 if where == "first" else size - 1
+    if r:
+        pa, sa, pb, sb = (np.roll(a, r, axis=0) for a in (pa, sa, pb, sb))
+    d = run_gemm(pa, sa, gd["ax"], pb, sb, gd["aw"], M, N, K, kernel)
+    assert d[r, r] == gd["group_result"]
+    d[r, r] = 0.0
     assert not d.any()
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 384, 512), (384, 128, 1280)])
-def test_gemm_matches_the_exact_product(M, N, K):
+CTA_SHAPES = [(128, 128, 256), (256, 384, 512), (384, 128, 1280)]
+PAIR_SHAPES = [(256, 256, 256), (512, 768, 1024), (256, 512, 2560), (768, 256, 512)]
+
+
+@pytest.mark.parametrize("M,N,K,kernel", [s + (fp4.GEMM_CTA,) for s in CTA_SHAPES] +
+                         [s + (fp4.GEMM_CTA_PAIR,) for s in PAIR_SHAPES] +
+                         [(512, 768, 1024, fp4.GEMM_CTA)])
+def test_gemm_matches_the_exact_product(M, N, K, kernel):
     g = torch.Generator().manual_seed(M + N + K)
     xa = torch.randn(M, K, generator=g) * torch.rand(M, 1, generator=g) * 3
     xb = torch.randn(N, K, generator=g) * 0.02
@@ -81,7 +96,7 @@ def test_gemm_matches_the_exact_product(M, N, K):
     qa = fp4.nvfp4_quantize(xa.to(torch.bfloat16).to(DEV))
     qb = fp4.nvfp4_quantize(xb.to(torch.bfloat16).to(DEV))
     st = fp4.new_status(DEV)
-    d = fp4.nvfp4_gemm(qa, qb, status=st)
+    d = fp4.nvfp4_gemm(qa, qb, status=st, kernel=kernel)
     torch.cuda.synchronize()
     qa.check()
     qb.check()
@@ -93,15 +108,22 @@ def test_gemm_matches_the_exact_product(M, N, K):
     assert (err <= tolerance(mag, K)).all(), f"max err {err.max()} vs tol {tolerance(mag, K).max()}"
 
 
-def test_gemm_large_sampled_rows():
-    M, N, K = 1024, 1024, 4096
+@pytest.mark.parametrize("M,N,K,kernel", [(1024, 1024, 4096, fp4.GEMM_CTA),
+                                           (1024, 1024, 4096, fp4.GEMM_CTA_PAIR),
+                                           (4096, 4096, 512, fp4.GEMM_CTA_PAIR)])
+def test_gemm_large_sampled_rows(M, N, K, kernel):
+    """Sampled rows against the exact product; 4096 x 4096 gives the pair
+    kernel 256 tiles, more than there are SM pairs, so clusters take several
+    tiles each (the persistent loop and the accumulator hand-over)."""
     g = torch.Generator().manual_seed(5)
     xa = (torch.randn(M, K, generator=g) * 0.5).to(torch.bfloat16).to(DEV)
     xb = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).to(DEV)
     qa, qb = fp4.nvfp4_quantize(xa), fp4.nvfp4_quantize(xb)
-    d = fp4.nvfp4_gemm(qa, qb)
+    st = fp4.new_status(DEV)
+    d = fp4.nvfp4_gemm(qa, qb, status=st, kernel=kernel)
     torch.cuda.synchronize()
-    rows = [0, 1, 127, 128, 500, 1023]
+    assert st.item() == 0
+    rows = sorted({0, 1, 127, 128, 255, 256, 500, M // 2 + 129, M - 1})
     pa = qa.packed.cpu().numpy()[rows]
     sa = qa.scales.cpu().numpy()[rows]
     want, mag = oracle.nvfp4_gemm(pa, sa, qa.global_scale.item(), qb.packed.cpu().numpy(),
@@ -115,3 +137,16 @@ def test_gemm_argument_errors():
     with pytest.raises(fp4.FP4Error) as e:
         fp4.nvfp4_gemm(q, q)
     assert e.value.status == fp4.ERR_SHAPE
+
+
+def test_pair_kernel_shape_and_argument_errors():
+    q = fp4.nvfp4_quantize(torch.randn(384, 256, device=DEV))  # 384 is not a multiple of 256
+    with pytest.raises(fp4.FP4Error) as e:
+        fp4.nvfp4_gemm(q, q, kernel=fp4.GEMM_CTA_PAIR)
+    assert e.value.status == fp4.ERR_SHAPE
+    d = fp4.nvfp4_gemm(q, q, kernel=fp4.GEMM_AUTO)  # falls back to one CTA per tile
+    torch.cuda.synchronize()
+    assert d.shape == (384, 384)
+    with pytest.raises(fp4.FP4Error) as e:
+        fp4.nvfp4_gemm(q, q, kernel=7)
+    assert e.value.status == fp4.ERR_INVALID_ARG
