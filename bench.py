@@ -10,7 +10,9 @@ search).  `value` is elements of x per second over the whole job, timed on
 the device with CUDA events around each step, L2 flushed (512 MiB write, 256 MiB read)
 between steps, max over ranks.  `e2e` times the same step through the same
 C-ABI calls starting from pinned host memory: host->device copy of x, the
-step, device->host copy of every quantised artefact and the status word.
+step, device->host copy of every quantised artefact and the status word,
+double-buffered over three streams as a caller streaming batches would run
+it (the upload of step k+1 overlaps step k's kernels and download).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle on host cores
@@ -205,6 +207,11 @@ class Path:
     OPS = OPS
     LAUNCHES = 6  # one kernel per entry point (the amax folds in its last CTA)
 
+    def twin(self, x2: torch.Tensor) -> "Path":
+        """The same step on another input buffer with its own outputs (the
+        second half of the double-buffered end-to-end pipeline)."""
+        return Path(x2)
+
     def step(self, events=None):
         for i, (fn, args) in enumerate(self.calls):
             st = fn(*args)
@@ -299,6 +306,9 @@ class LayoutPath:
     OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize"]
     LAUNCHES = 5
 
+    def twin(self, x2: torch.Tensor) -> "LayoutPath":
+        return LayoutPath(x2, self.kind)
+
     def __init__(self, x: torch.Tensor, kind: str):
         import block_scaled_fp4_reduce_b200 as fp4
         self.fp4 = fp4
@@ -362,20 +372,23 @@ class GemmPath:
     OPS = ["amax", "nvfp4_quantize", "scales_to_mma", "nvfp4_gemm"]
     LAUNCHES = 4
 
-    def __init__(self, x: torch.Tensor, w: torch.Tensor):
+    def __init__(self, x: torch.Tensor, w: torch.Tensor = None, shared: "GemmPath" = None):
         import block_scaled_fp4_reduce_b200 as fp4
         self.fp4 = fp4
         L = fp4.lib()
         dev = x.device
         M, K = x.shape
-        N = w.shape[0]
-        self.x, self.n, self.M, self.N, self.K = x, x.numel(), M, N, K
         u8 = torch.uint8
-        qw = fp4.nvfp4_quantize(w)
-        self.w_sf = fp4.scales_to_mma(qw.scales)
-        torch.cuda.synchronize()
-        qw.check()
+        if shared is None:
+            qw = fp4.nvfp4_quantize(w)
+            self.w_sf = fp4.scales_to_mma(qw.scales)
+            torch.cuda.synchronize()
+            qw.check()
+        else:  # the quantised weight of another path, read-only
+            qw, self.w_sf = shared.qw, shared.w_sf
         self.qw = qw
+        N = qw.rows
+        self.x, self.n, self.M, self.N, self.K = x, x.numel(), M, N, K
         self.amax = torch.empty(1, dtype=torch.float32, device=dev)
         self.ws = fp4.workspace_for(x)
         self.status = fp4.new_status(dev)
@@ -398,6 +411,80 @@ class GemmPath:
 
     step = Path.step
     check_status = Path.check_status
+
+    def twin(self, x2: torch.Tensor) -> "GemmPath":
+        return GemmPath(x2, shared=self)
+
+
+def e2e_serial(path, x, x_host, steps: int, flush_l2) -> tuple[float, str]:
+    """Milliseconds for `steps` steps, each on its own: L2 flush, upload of x
+    from pinned memory, the step, download of every result, wait."""
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in path.results]
+    ms = 0.0
+    for k in range(steps + 2):
+        flush_l2()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        x.copy_(x_host, non_blocking=True)
+        path.step()
+        for h, t in zip(host_out, path.results):
+            h.copy_(t, non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        if int(host_out[-1].item()) != 0:
+            raise RuntimeError("device status set during the end-to-end run")
+        if k >= 2:
+            ms += e0.elapsed_time(e1)
+    return ms, "serial: upload, step, download, wait; L2 flushed before each step"
+
+
+def e2e_pipelined(path, x, x_host, steps: int) -> tuple[float, str]:
+    """Milliseconds for `steps` steps streamed the way a caller feeds batches:
+    two device input buffers and two sets of outputs; step k's upload runs on
+    an upload stream, its kernels on the compute stream, its downloads on a
+    download stream, so the upload of step k+1 overlaps the kernels and the
+    download of step k (the link is full duplex).  Every step uploads its
+    whole input from pinned host memory and downloads every result; one
+    event pair on the device spans the first upload to the last download."""
+    paths = [path, path.twin(torch.empty_like(x))]
+    xs = [x, paths[1].x]
+    outs = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in p.results] for p in paths]
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def run(n: int) -> float:
+        ev = [[torch.cuda.Event() for _ in range(n)] for _ in range(3)]  # upload, compute, download
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(up)
+        for k in range(n):
+            b = k % 2
+            if k >= 2:
+                up.wait_event(ev[1][k - 2])  # the kernels of step k-2 have read xs[b]
+            with torch.cuda.stream(up):
+                xs[b].copy_(x_host, non_blocking=True)
+            ev[0][k].record(up)
+            comp.wait_event(ev[0][k])
+            if k >= 2:
+                comp.wait_event(ev[2][k - 2])  # outputs of step k-2 downloaded
+            paths[b].step()
+            ev[1][k].record(comp)
+            down.wait_event(ev[1][k])
+            with torch.cuda.stream(down):
+                for h, t in zip(outs[b], paths[b].results):
+                    h.copy_(t, non_blocking=True)
+            ev[2][k].record(down)
+        end.record(down)
+        end.synchronize()
+        for o in outs:
+            if int(o[-1].item()) != 0:
+                raise RuntimeError("device status set during the end-to-end run")
+        return start.elapsed_time(end)
+
+    run(4)  # warm-up: streams, pinned buffers, the twin's first launches
+    return run(steps), ("double-buffered: upload of step k+1 (upload stream) overlaps the kernels (compute "
+                        "stream) and the download (download stream) of step k; every step's input uploaded "
+                        "from pinned host memory, every result downloaded; no L2 flush between steps")
 
 
 def max_over_ranks(values: list[float], device, world: int) -> list[float]:
@@ -485,24 +572,12 @@ def run_ours(args, rank: int, world: int, local: int):
 
     # ---- end to end through the same calls from pinned host memory ---------
     Ke = max(3, min(K, args.e2e_steps))
-    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in path.results]
     h2d = x.numel() * x.element_size()
     d2h = sum(t.numel() * t.element_size() for t in path.results)
-    e2e_ms = 0.0
-    for k in range(Ke + 2):
-        flush_l2()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        x.copy_(x_host, non_blocking=True)
-        path.step()
-        for h, t in zip(host_out, path.results):
-            h.copy_(t, non_blocking=True)
-        e1.record()
-        e1.synchronize()
-        if int(host_out[-1].item()) != 0:
-            raise RuntimeError("device status set during the end-to-end run")
-        if k >= 2:
-            e2e_ms += e0.elapsed_time(e1)
+    if hasattr(path, "twin"):
+        e2e_ms, e2e_schedule = e2e_pipelined(path, x, x_host, Ke)
+    else:
+        e2e_ms, e2e_schedule = e2e_serial(path, x, x_host, Ke, flush_l2)
 
     total_ms, e2e_ms, *per_op_ms = max_over_ranks([total_ms, e2e_ms] + per_op_ms, dev, world)
     if world > 1:
@@ -569,7 +644,7 @@ def run_ours(args, rank: int, world: int, local: int):
         "kernels": kernels,
         "roofline": roof,
         "e2e": {"value": n_all * Ke / (e2e_ms / 1e3), "unit": "elements/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "schedule": e2e_schedule},
         "gpu_launches": path.LAUNCHES * K,
         "clocks": clk,
         "wall_s_timed": wall,
