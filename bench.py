@@ -8,7 +8,9 @@ the 4096 x 4096 bf16 LLM weight matrix, N(0, 0.02) with 0.1 % outliers x50):
 (6 kernel launches; the amax is shared by the NVFP4 quantiser and the
 search).  `value` is elements of x per second over the whole job, timed on
 the device with CUDA events around each step, L2 flushed (512 MiB write, 256 MiB read)
-between steps, max over ranks.  `e2e` times the same step through the same
+between steps, max over ranks; nothing is recorded between the launches of a
+step (an event there would serialise them).  Per-kernel times come from a
+second pass with an event after every launch.  `e2e` times the same step through the same
 C-ABI calls starting from pinned host memory: host->device copy of x, the
 step, device->host copy of every quantised artefact and the status word,
 double-buffered over three streams as a caller streaming batches would run
@@ -544,9 +546,13 @@ def run_ours(args, rank: int, world: int, local: int):
     torch.cuda.synchronize()
     path.check_status()
 
-    # ---- timed region: K steps, events around every entry point ----------
+    # ---- timed region: K steps, one event pair around each step -----------
+    # Nothing is recorded between the launches of a step: an event between
+    # two kernels serialises them and forfeits the programmatic dependent
+    # launch (each kernel's launch and ramp overlapping its predecessor's
+    # tail), ~26 us of a 100 us step on the default workload.
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nops + 1)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     clocks = ClockSampler(local)
     clocks.start()
     if world > 1:
@@ -556,19 +562,26 @@ def run_ours(args, rank: int, world: int, local: int):
     for k in range(K):
         flush_l2()
         evs[k][0].record()
-        path.step(evs[k])
+        path.step()
+        evs[k][1].record()
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
     path.check_status()
-    per_op_ms = [0.0] * nops
-    total_ms = 0.0
-    for k in range(K):
-        total_ms += evs[k][0].elapsed_time(evs[k][nops])
-        for i in range(nops):
-            per_op_ms[i] += evs[k][i].elapsed_time(evs[k][i + 1])
+    total_ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
+
+    # ---- per entry point: a second pass with an event after every launch ---
+    Kb = max(3, min(K, args.breakdown_steps))
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nops + 1)] for _ in range(Kb)]
+    for k in range(Kb):
+        flush_l2()
+        bevs[k][0].record()
+        path.step(bevs[k])
+    torch.cuda.synchronize()
+    path.check_status()
+    per_op_ms = [sum(bevs[k][i].elapsed_time(bevs[k][i + 1]) for k in range(Kb)) for i in range(nops)]
 
     # ---- end to end through the same calls from pinned host memory ---------
     Ke = max(3, min(K, args.e2e_steps))
@@ -594,9 +607,9 @@ def run_ours(args, rank: int, world: int, local: int):
         ab["nvfp4_gemm"] = (M_ + N_) * (K_ // 2 + K_ // 16) + 4 * M_ * N_
     kernels = {}
     for name, ms in zip(path.OPS, per_op_ms):
-        us = ms / K * 1e3
+        us = ms / Kb * 1e3
         gbs = ab[name] / (us * 1e-6) / 1e9
-        kernels[name] = {"us": round(us, 3), "share": round(ms / total_ms, 4), "gbs": round(gbs, 1),
+        kernels[name] = {"us": round(us, 3), "share": round(ms / sum(per_op_ms), 4), "gbs": round(gbs, 1),
                          "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
     dom = max(kernels, key=lambda k: kernels[k]["us"])
     n_cand = search_candidate_count(x, path.ss_g.item()) if dom == "scale_search" else None
@@ -642,6 +655,9 @@ def run_ours(args, rank: int, world: int, local: int):
                    "parallelism": f"replicas x{world} (independent tensors)" if world > 1 else "single GPU"},
         "hbm_gbs_step": sum(ab[o] for o in path.OPS) / (total_ms / K * 1e-3) / 1e9,
         "kernels": kernels,
+        "kernels_timing": (f"second pass of {Kb} steps, L2 flushed between steps, an event after every launch: "
+                           "the events serialise the launches, so each time includes its own launch and ramp "
+                           "and the times add up to more than ms_per_step"),
         "roofline": roof,
         "e2e": {"value": n_all * Ke / (e2e_ms / 1e3), "unit": "elements/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "schedule": e2e_schedule},
@@ -860,6 +876,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--breakdown-steps", type=int, default=500,
+                    help="steps of the per-entry-point pass (events between launches)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--model-layers", type=int, default=workloads.MODEL_LAYERS,
