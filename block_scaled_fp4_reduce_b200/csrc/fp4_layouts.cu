@@ -108,7 +108,7 @@ fp4_status columns(const T *x, int64_t rows, int64_t cols, const float *amax, ui
                    uint8_t *scales, float *global_scale, int32_t *status, cudaStream_t stream)
 {
     auto kernel = fp4::quantize_columns_kernel<T, kNv, kCeil>;
-    constexpr size_t kSmem = (size_t)fp4::kColStages * fp4::kColTileBytes;
+    constexpr size_t kSmem = (size_t)fp4::kColStages * fp4::kColTileBytes + (kNv ? 0 : fp4::kColStageBytes);
     static bool attr_set[kMaxDevices] = {false};
     int dev = 0;
     if (sm_count(dev) <= 0 || dev >= kMaxDevices)

@@ -323,12 +323,19 @@ __global__ void __launch_bounds__(kPadTile)
 // CTA has 128 threads per block row of the tile (64 / G block rows: 512
 // threads for NVFP4, 256 for MXFP4), and thread (j, w) quantises the
 // block(s) of block row j in word column w: one fp32 column, or the two bf16
-// columns that share the word.
+// columns that share the word.  NVFP4 stores its 8-byte blocks straight into
+// the output rows; MXFP4 (bound by its stores, not its instructions) stages a
+// tile's blocks in shared memory and stores each output row's 32 bytes from
+// one thread.
 // ---------------------------------------------------------------------------
 constexpr int kColWords = 128;
 constexpr int kColTileRows = 64;
 constexpr int kColTileBytes = kColTileRows * 512;
 constexpr int kColStages = 2;
+// Staging of one tile's results: packed codes (32 bytes per tile column:
+// 4 NVFP4 or 2 MXFP4 blocks) and scale bytes, for up to 256 columns.
+constexpr int kColStagePacked = 256 * 32;
+constexpr int kColStageBytes = kColStagePacked + 256 * 4;
 template <bool kNv> constexpr int col_threads() { return kColWords * (kColTileRows / (kNv ? 16 : 32)); }
 constexpr uint32_t kWaitTries = 1u << 22;
 
@@ -395,9 +402,11 @@ __device__ __forceinline__ ColTile col_tile(int t, int n_tc, int tile_cols)
 }
 
 // Quantises the G-element blocks of the tile rows [j*G, j*G + G) in this
-// thread's columns and stores them into the output rows (= columns of W).
+// thread's columns and stores them straight into the output rows (= columns
+// of W): the NVFP4 pass, which is bound by its instruction issue, not by
+// these partial-sector stores.
 template <typename T, bool kNv, bool kCeil, int G>
-__device__ __forceinline__ void column_blocks(const uint8_t *tile, int j, int w, int c_first, int C,
+__device__ __forceinline__ void column_blocks_direct(const uint8_t *tile, int j, int w, int c_first, int C,
                                               int blk, const NvScaleConsts &sc, uint8_t *packed,
                                               uint8_t *scales, int64_t prow, int nbo, bool &bad)
 {
@@ -431,6 +440,81 @@ __device__ __forceinline__ void column_blocks(const uint8_t *tile, int j, int w,
             mx_quantize_block<kCeil>(b, reinterpret_cast<uint4 *>(orow) + blk,
                                      scales + (int64_t)c * nbo + blk, bad);
     }
+}
+
+// Quantises the G-element blocks of the tile rows [j*G, j*G + G) in this
+// thread's columns into the staging tile: packed codes of block row j and
+// tile column c at stage_p + (j * kCols + c) * G/2, its scale byte at
+// stage_s[j * kCols + c] (block-row-major: a warp's writes are consecutive).
+template <typename T, bool kNv, bool kCeil, int G>
+__device__ __forceinline__ void column_blocks(const uint8_t *tile, int j, int w, const NvScaleConsts &sc,
+                                              uint8_t *stage_p, uint8_t *stage_s, bool &bad)
+{
+    constexpr int kPerThread = 4 / (int)sizeof(T); // columns per word: 2 (bf16) or 1 (fp32)
+    constexpr int kCols = kColWords * kPerThread;
+    const uint32_t *tw = reinterpret_cast<const uint32_t *>(tile) + j * G * kColWords + w;
+    uint32_t rowv[G]; // row i of this thread's word column
+#pragma unroll
+    for (int i = 0; i < G; ++i)
+        rowv[i] = tw[i * kColWords];
+#pragma unroll
+    for (int p = 0; p < kPerThread; ++p) {
+        const int c = w * kPerThread + p; // tile column
+        Blk<T, G> b;
+        if constexpr (sizeof(T) == 2) {
+            // bf16: a word holds columns 2t (low half) and 2t+1 (high half);
+            // gather one column's halves of rows 2i, 2i+1 into word i.
+#pragma unroll
+            for (int i = 0; i < G / 2; ++i)
+                b.w[i] = __byte_perm(rowv[2 * i], rowv[2 * i + 1], p ? 0x7632 : 0x5410);
+        } else {
+#pragma unroll
+            for (int i = 0; i < G; ++i)
+                b.w[i] = rowv[i];
+        }
+        uint8_t *dp = stage_p + (j * kCols + c) * (G / 2);
+        uint8_t *ds = stage_s + j * kCols + c;
+        if constexpr (kNv)
+            nv_quantize_block(b, sc, reinterpret_cast<uint2 *>(dp), ds);
+        else
+            mx_quantize_block<kCeil>(b, reinterpret_cast<uint4 *>(dp), ds, bad);
+    }
+}
+
+// Stores tile column c's staged blocks: kBR blocks of G/2 bytes (32 bytes)
+// contiguous in output row c, and their kBR scale bytes; only the n_valid
+// first ones when the column is cut by the padded length.  wide: the row's
+// 32 bytes start on a 32-byte boundary.
+template <int G, int kCols>
+__device__ __forceinline__ void column_store(const uint8_t *stage_p, const uint8_t *stage_s, int c,
+                                             uint8_t *orow, uint8_t *srow, int n_valid, bool wide)
+{
+    constexpr int kBR = kColTileRows / G; // block rows per tile: 4 (NVFP4) or 2 (MXFP4)
+    constexpr int kBytes = G / 2;         // packed bytes per block: 8 or 16
+    uint32_t wds[8];
+#pragma unroll
+    for (int j = 0; j < kBR; ++j) {
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(stage_p + (j * kCols + c) * kBytes);
+#pragma unroll
+        for (int i = 0; i < kBytes / 4; ++i)
+            wds[j * (kBytes / 4) + i] = src[i];
+    }
+    if (n_valid == kBR && wide) {
+        stg_v8(orow, wds);
+    } else {
+#pragma unroll
+        for (int j = 0; j < kBR; ++j)
+            if (j < n_valid) {
+#pragma unroll
+                for (int i = 0; i < kBytes / 8; ++i)
+                    *reinterpret_cast<uint2 *>(orow + j * kBytes + 8 * i) =
+                        make_uint2(wds[j * (kBytes / 4) + 2 * i], wds[j * (kBytes / 4) + 2 * i + 1]);
+            }
+    }
+#pragma unroll
+    for (int j = 0; j < kBR; ++j)
+        if (j < n_valid)
+            srow[j] = stage_s[j * kCols + c];
 }
 
 template <typename T, bool kNv, bool kCeil>
@@ -484,39 +568,93 @@ __global__ void __launch_bounds__(col_threads<kNv>())
             }
         }
     }
-    // Each warp waits for its tiles on full[s], releases them on empty[s];
-    // thread 0 refills a stage once every warp has released it.  All waits
-    // are bounded; a thread that gives up leaves the loop, and every wait
-    // that depended on it then runs out in turn.
     bool bad = false, timed_out = false;
     int k = 0;
-    for (int t = first_tile; t < n_tiles; t += stride, ++k) {
-        const int s = k % kColStages;
-        const uint32_t phase = (uint32_t)(k / kColStages) & 1u;
-        if (!mbar_wait(&full[s], phase)) {
-            timed_out = true;
-            break;
-        }
-        const ColTile ct = col_tile(t, n_tc, kCols);
-        const int blk_row = ct.r0 + jb * G;
-        if (blk_row < R)
-            column_blocks<T, kNv, kCeil, G>(smem + s * kColTileBytes, jb, w, ct.c0 + w * kPerWord, C,
-                                            blk_row / G, sc, packed, scales, prow, nbo, bad);
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0)
-            mbar_arrive(&empty[s]);
-        if (producer) {
-            const int tn = t + kColStages * stride;
-            if (tn < n_tiles) {
-                if (!mbar_wait(&empty[s], phase)) {
-                    timed_out = true;
-                    break;
+    if constexpr (kNv) {
+        // Each warp waits for its tiles on full[s], releases them on empty[s];
+        // thread 0 refills a stage once every warp has released it.  All waits
+        // are bounded; a thread that gives up leaves the loop, and every wait
+        // that depended on it then runs out in turn.
+        for (int t = first_tile; t < n_tiles; t += stride, ++k) {
+            const int s = k % kColStages;
+            const uint32_t phase = (uint32_t)(k / kColStages) & 1u;
+            if (!mbar_wait(&full[s], phase)) {
+                timed_out = true;
+                break;
+            }
+            const ColTile ct = col_tile(t, n_tc, kCols);
+            const int blk_row = ct.r0 + jb * G;
+            if (blk_row < R)
+                column_blocks_direct<T, kNv, kCeil, G>(smem + s * kColTileBytes, jb, w, ct.c0 + w * kPerWord,
+                                                       C, blk_row / G, sc, packed, scales, prow, nbo, bad);
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0)
+                mbar_arrive(&empty[s]);
+            if (producer) {
+                const int tn = t + kColStages * stride;
+                if (tn < n_tiles) {
+                    if (!mbar_wait(&empty[s], phase)) {
+                        timed_out = true;
+                        break;
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    const ColTile cn = col_tile(tn, n_tc, kCols);
+                    mbar_expect_tx(&full[s], kColTileBytes);
+                    tma_load_2d(smem + s * kColTileBytes, &map, cn.c0, cn.r0, &full[s]);
+                    ++issued;
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                const ColTile cn = col_tile(tn, n_tc, kCols);
-                mbar_expect_tx(&full[s], kColTileBytes);
-                tma_load_2d(smem + s * kColTileBytes, &map, cn.c0, cn.r0, &full[s]);
-                ++issued;
+            }
+        }
+    } else {
+        // MXFP4, bound by its stores: per tile every thread waits (bounded)
+        // for the tile on full[s], and the CTA votes: if any wait ran out,
+        // all threads leave the loop together (the barriers below must be
+        // reached by all or none).  The threads quantise their blocks into
+        // the staging tile, release the TMA stage (each warp on empty[s]),
+        // and after a barrier thread c < kCols stores tile column c's
+        // blocks: 32 contiguous bytes of one output row instead of 16 bytes
+        // from each of two warps.  Thread 0 refills the stage once every warp
+        // has released it; a refill wait that runs out goes into the next
+        // vote.
+        uint8_t *stage_p = smem + kColStages * kColTileBytes;
+        uint8_t *stage_s = stage_p + kColStagePacked;
+        const bool wide = (reinterpret_cast<uintptr_t>(packed) % 32u) == 0 && prow % 32 == 0;
+        for (int t = first_tile; t < n_tiles; t += stride, ++k) {
+            const int s = k % kColStages;
+            const uint32_t phase = (uint32_t)(k / kColStages) & 1u;
+            const bool ok = !timed_out && mbar_wait(&full[s], phase);
+            if (__syncthreads_or(!ok)) {
+                timed_out = true;
+                break;
+            }
+            const ColTile ct = col_tile(t, n_tc, kCols);
+            if (ct.r0 + jb * G < R)
+                column_blocks<T, kNv, kCeil, G>(smem + s * kColTileBytes, jb, w, sc, stage_p, stage_s, bad);
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0)
+                mbar_arrive(&empty[s]);
+            __syncthreads(); // staging tile complete
+            const int c = (int)threadIdx.x;
+            const int blk0 = ct.r0 / G;
+            if (c < kCols && ct.c0 + c < C) {
+                const int n_valid = nbo - blk0 < kColTileRows / G ? nbo - blk0 : kColTileRows / G;
+                const int64_t oc = ct.c0 + c;
+                column_store<G, kCols>(stage_p, stage_s, c, packed + oc * prow + (int64_t)blk0 * (G / 2),
+                                       scales + oc * nbo + blk0, n_valid, wide);
+            }
+            if (producer) {
+                const int tn = t + kColStages * stride;
+                if (tn < n_tiles) {
+                    if (!mbar_wait(&empty[s], phase)) {
+                        timed_out = true; // the next vote ends the loop for everyone
+                    } else {
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        const ColTile cn = col_tile(tn, n_tc, kCols);
+                        mbar_expect_tx(&full[s], kColTileBytes);
+                        tma_load_2d(smem + s * kColTileBytes, &map, cn.c0, cn.r0, &full[s]);
+                        ++issued;
+                    }
+                }
             }
         }
     }

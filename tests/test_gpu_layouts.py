@@ -105,7 +105,8 @@ def check_columns(x):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("shape", [(16, 8), (20, 8), (64, 256), (100, 264), (129, 520), (300, 1032), (65, 4)])
+@pytest.mark.parametrize("shape", [(16, 8), (20, 8), (64, 256), (100, 264), (129, 520), (300, 1032), (65, 4),
+                                   (256, 520), (192, 264)])
 def test_columns_parity(dtype, shape):
     R, C = shape
     if dtype == torch.bfloat16 and C % 8:
