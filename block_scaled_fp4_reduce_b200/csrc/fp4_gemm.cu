@@ -175,15 +175,13 @@ fp4_status fp4_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t
         return FP4_OK;
     if (!out || (rows * blocks > 0 && !scales))
         return FP4_ERR_INVALID_ARG;
-    if (words > INT_MAX || rows > INT_MAX || blocks > INT_MAX)
+    const int64_t bands = cdiv(rows, 128), kt = cdiv(blocks, 4), chunks = cdiv(kt, fp4::kSfKc);
+    if (words > INT_MAX || rows > INT_MAX || blocks > INT_MAX || chunks > 65535)
         return FP4_ERR_SHAPE;
     if (!aligned(out, 4))
         return FP4_ERR_ALIGN;
-    const int grid = grid_for(fp4::scales_to_mma_kernel, words, kThreads);
-    if (grid <= 0)
-        return FP4_ERR_CUDA;
-    return launch(fp4::scales_to_mma_kernel, grid, stream, scales, (int)rows, (int)blocks,
-                  (int)cdiv(blocks, 4), (int)words, reinterpret_cast<uint32_t *>(out));
+    return launch_cfg(fp4::scales_to_mma_kernel, dim3((unsigned)bands, (unsigned)chunks), 256, 0, stream, scales,
+                      (int)rows, (int)blocks, (int)kt, reinterpret_cast<uint32_t *>(out));
 }
 
 fp4_status fp4_nvfp4_gemm(const uint8_t *packed_a, const uint8_t *scales_a_mma, const float *global_scale_a,

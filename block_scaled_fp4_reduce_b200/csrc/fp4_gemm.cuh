@@ -50,31 +50,66 @@
 namespace fp4 {
 
 // ---------------------------------------------------------------------------
-// Scale layout for the MMA.  One thread per output 32-bit word: word
-// 4 r0 + r1 of tile t holds blocks 4 (t % kt) .. + 3 of row
-// (t / kt) * 128 + 32 r1 + r0 (kt = ceil(nb / 4) block tiles per row band).
+// Scale layout for the MMA, as a tiled transpose.  CTA (band, chunk) takes
+// the 128 rows of one band and kSfKc consecutive 4-block tiles (64 scale
+// bytes per row): it loads the 128 x 64-byte strip with row-contiguous
+// loads into shared memory (rows padded to 17 words, so that the column
+// reads below are free of bank conflicts), then writes the strip's output
+// tiles, which are contiguous in the MMA layout: 16 bytes per thread, word
+// 4 r0 + r1 of tile t = the four block scales of row 32 r1 + r0 in tile t.
+// Rows past `rows` and blocks past `nb` are 0.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads)
-    scales_to_mma_kernel(const uint8_t *__restrict__ s, int rows, int nb, int kt, int n_words,
-                         uint32_t *__restrict__ out)
+constexpr int kSfKc = 16;                 // 4-block tiles per CTA
+constexpr int kSfRowWords = kSfKc + 1;    // padded shared-memory row (words)
+
+__global__ void __launch_bounds__(256)
+    scales_to_mma_kernel(const uint8_t *__restrict__ s, int rows, int nb, int kt, uint32_t *__restrict__ out)
 {
+    __shared__ uint32_t strip[128 * kSfRowWords];
     pdl_begin();
-    const int stride = (int)(gridDim.x * blockDim.x);
-    for (int wi = (int)(blockIdx.x * blockDim.x + threadIdx.x); wi < n_words; wi += stride) {
-        const int tile = wi >> 7;    // 128 words per 512-byte tile
-        const int within = wi & 127; // word 4 r0 + r1 of the tile
-        const int r0 = within >> 2, r1 = within & 3;
-        const int row = (tile / kt) * 128 + r1 * 32 + r0;
-        const int j0 = (tile % kt) * 4;
-        uint32_t v = 0;
-        if (row < rows) {
-            const uint8_t *src = s + (int64_t)row * nb;
+    const int band = (int)blockIdx.x, kc0 = (int)blockIdx.y * kSfKc;
+    const int n_kt = kt - kc0 < kSfKc ? kt - kc0 : kSfKc;
+    const int t = (int)threadIdx.x;
+    {
+        // thread t: row t / 2 of the band, words 8 (t % 2) .. + 7 of its strip
+        const int r = t >> 1, h = t & 1;
+        const int row = band * 128 + r;
+        const int b0 = kc0 * 4 + h * 32; // first block of this thread's 32
+        const uint8_t *src = s + (int64_t)row * nb;
+        const bool words = (nb & 3) == 0 && (reinterpret_cast<uintptr_t>(s) & 3u) == 0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (j0 + j < nb)
-                    v |= (uint32_t)__ldcg(src + j0 + j) << (8 * j);
+        for (int i = 0; i < 8; ++i) {
+            const int b = b0 + 4 * i;
+            uint32_t v = 0;
+            if (row < rows) {
+                if (words && b + 3 < nb) {
+                    v = __ldcg(reinterpret_cast<const uint32_t *>(src + b));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (b + j < nb)
+                            v |= (uint32_t)__ldcg(src + b + j) << (8 * j);
+                }
+            }
+            strip[r * kSfRowWords + h * 8 + i] = v;
         }
-        out[wi] = v;
+    }
+    __syncthreads();
+    uint32_t *dst = out + ((int64_t)band * kt + kc0) * 128;
+    const bool vec = (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+    for (int i = t; i < n_kt * 32; i += 256) {
+        const int tt = i >> 5, q = i & 31; // tile, 16-byte chunk (= r0)
+        const uint4 v = make_uint4(strip[q * kSfRowWords + tt], strip[(32 + q) * kSfRowWords + tt],
+                                   strip[(64 + q) * kSfRowWords + tt], strip[(96 + q) * kSfRowWords + tt]);
+        uint32_t *o = dst + tt * 128 + 4 * q;
+        if (vec) {
+            *reinterpret_cast<uint4 *>(o) = v;
+        } else {
+            o[0] = v.x;
+            o[1] = v.y;
+            o[2] = v.z;
+            o[3] = v.w;
+        }
     }
 }
 

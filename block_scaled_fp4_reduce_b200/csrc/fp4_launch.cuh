@@ -88,11 +88,11 @@ int grid_for(K kernel, int64_t work, int64_t per_cta, int block = kThreads, size
 // the previous kernel on the stream finishes; it waits for it
 // (griddepcontrol.wait) before touching memory.
 template <typename... KArgs, typename... Args>
-fp4_status launch_cfg(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+fp4_status launch_cfg(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem,
                       cudaStream_t stream, Args... args)
 {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
+    cfg.gridDim = grid;
     cfg.blockDim = dim3((unsigned)block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
