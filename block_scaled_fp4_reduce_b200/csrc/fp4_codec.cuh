@@ -196,15 +196,59 @@ __device__ __forceinline__ uint32_t e4m3_code_from_f64(double t)
 // code.  Otherwise (never for t < 2^-11, which is always code 0) the rational
 // is formed as one correctly rounded double quotient (num * A_b and den are
 // exact in double).
+__device__ __forceinline__ uint32_t e4m3_rn(float t)
+{
+    uint16_t c;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(0.0f), "f"(t));
+    return (uint32_t)(c & 0xFFu);
+}
+
 __device__ __forceinline__ uint32_t nv_scale_code(float amax_b, float inv, double num, double den)
 {
     const float t = __fmul_rn(amax_b, inv);
     const uint32_t tb = __float_as_uint(t);
     if (tb > 0x3A000000u && ((tb + 16u) & 0x7FFFFu) < 32u)
         return e4m3_code_from_f64(__ddiv_rn(num * (double)amax_b, den));
-    uint16_t c;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(0.0f), "f"(t));
-    return (uint32_t)(c & 0xFFu);
+    return e4m3_rn(t);
+}
+
+// The same for t = amax_b / (m g) with m = 6 (the max-based scale) or 4,
+// inv = RN32(1 / (m g)), den = m g (exact in double), without the double
+// division where t lies near a grid point P with five significant bits in
+// the normal E4M3 range.  An E4M3 value P: t is within 18 ulps of it and
+// 2^19 ulps from either midpoint, so the conversion of t is right.  A
+// midpoint P: the sign of amax_b - P m g decides exactly -- P m is exact
+// (eight significant bits), P m g = hi + lo exactly (one fma), amax_b - hi
+// is exact (Sterbenz: amax_b is within 2^-18 of hi) -- and an exact tie
+// takes the even code.  The double path rounds the quotient to double
+// first, which makes no false tie: a nonzero amax_b - P m g is at least
+// ~2^-31 of it, far above double's 2^-53.
+__device__ __forceinline__ uint32_t nv_scale_code_mg(float amax_b, float inv, float g, float m, double den)
+{
+    const float t = __fmul_rn(amax_b, inv);
+    const uint32_t tb = __float_as_uint(t);
+    if (tb > 0x3A000000u && ((tb + 16u) & 0x7FFFFu) < 32u) {
+        const uint32_t pb = (tb + 16u) & ~0x7FFFFu;
+        const float P = __uint_as_float(pb);
+        if (P >= 0x1p-6f && g >= 0x1p-100f) {
+            if (!(pb & 0x80000u) && P <= 448.0f)
+                return e4m3_rn(t);
+            if ((pb & 0x80000u) && P < 448.0f) {
+                const float pm = __fmul_rn(P, m);
+                const float hi = __fmul_rn(pm, g);
+                const float lo = __fmaf_rn(pm, g, -hi);
+                const float d = __fsub_rn(amax_b, hi);
+                const uint32_t c_lo = e4m3_rn(__uint_as_float(pb & ~0x80000u));
+                if (d > lo)
+                    return c_lo + 1u;
+                if (d < lo)
+                    return c_lo;
+                return c_lo + (c_lo & 1u);
+            }
+        }
+        return e4m3_code_from_f64(__ddiv_rn((double)amax_b, den));
+    }
+    return e4m3_rn(t);
 }
 
 // Value of an E4M3 byte as f16 bits: every E4M3 value (2^-9 .. 448, NaN)

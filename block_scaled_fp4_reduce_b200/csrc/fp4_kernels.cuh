@@ -348,7 +348,7 @@ __device__ __forceinline__ void nv_quantize_block(const Blk<T, 16> &blk, const N
                                                   uint2 *packed, uint8_t *scale)
 {
     const float amax_b = __uint_as_float(absmax_bits(blk));
-    const uint32_t code = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
+    const uint32_t code = nv_scale_code_mg(amax_b, sc.inv6g, sc.g, 6.0f, sc.six_g);
     *packed = nv_block_codes(blk, code, sc.g);
     *scale = (uint8_t)code;
 }
@@ -787,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     for (int blk = (int)(blockIdx.x * blockDim.x + threadIdx.x); blk < n_blocks; blk += stride) {
         BlockSearch<T> bs;
         const float amax_b = bs.setup(x, blk, g, exact_always);
-        const uint32_t c_hi = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
+        const uint32_t c_hi = nv_scale_code_mg(amax_b, sc.inv6g, sc.g, 6.0f, sc.six_g);
         bs.c_lo = nv_scale_code(amax_b, inv_lo, 147.0, g1260);
         bs.best_c = c_hi;
         bs.next_c = c_hi;
@@ -826,8 +826,8 @@ __global__ void __launch_bounds__(kThreads)
     for (int blk = (int)(blockIdx.x * blockDim.x + threadIdx.x); blk < n_blocks; blk += stride) {
         BlockSearch<T> bs;
         const float amax_b = bs.setup(x, blk, g, exact_always);
-        const uint32_t c6 = nv_scale_code(amax_b, sc.inv6g, 1.0, sc.six_g);
-        const uint32_t c4 = nv_scale_code(amax_b, inv4g, 1.0, four_g);
+        const uint32_t c6 = nv_scale_code_mg(amax_b, sc.inv6g, sc.g, 6.0f, sc.six_g);
+        const uint32_t c4 = nv_scale_code_mg(amax_b, inv4g, sc.g, 4.0f, four_g);
         bs.best_c = c6;
         const Screen s0 = screen(bs.xk, c6, g, bs.k);
         bs.best = s0.s;
