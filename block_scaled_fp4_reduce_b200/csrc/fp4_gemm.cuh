@@ -16,9 +16,13 @@
 //                         contiguous; padding 0 (the sm100 block-scaled
 //                         layout; it is not on the pages)
 //   nvfp4_gemm_kernel     D [M, N] fp32 = g_a g_b A B^T for NVFP4 A [M, K]
-//                         and B [N, K] (both K-major, i.e. blocked along K)
+//                         and B [N, K] (both K-major, i.e. blocked along K),
+//                         one CTA per 128 x 128 tile of D
+//   nvfp4_gemm_pair_kernel the same on persistent clusters of two CTAs,
+//                         256 x 256 tiles, cta_group::2 (described with it
+//                         below)
 //
-// GEMM structure: one CTA per 128 x (128 kGemmHalves) tile of D (one
+// One-CTA GEMM structure: one CTA per 128 x (128 kGemmHalves) tile of D (one
 // accumulator of 128 columns per half, sharing the A tile), 128 threads.
 // Warp 0 is the producer (its lane 0 issues): per K step of 256 elements it
 // loads the A tile and the B tile(s) (128 rows x 128 bytes each, 2-D TMA
