@@ -203,8 +203,10 @@ fp4_status fp4_nvfp4_gemm_ex(const uint8_t *packed_a, const uint8_t *scales_a_mm
     if (M % fp4::kGemmTile || N % fp4::kGemmTile || K % fp4::kGemmKStep || M > INT_MAX || N > INT_MAX ||
         K > INT_MAX)
         return FP4_ERR_SHAPE;
+    // the pair kernel indexes its tiles and scale-tile rows with 32-bit ints
     const bool pair_shape = M % fp4::kPairTileM == 0 && N % fp4::kPairTileN == 0 && (M / 128) * (K / 64) <= INT_MAX &&
-                            (N / 128) * (K / 64) <= INT_MAX;
+                            (N / 128) * (K / 64) <= INT_MAX &&
+                            (M / fp4::kPairTileM) * (N / fp4::kPairTileN) <= INT_MAX;
     if (kernel == FP4_GEMM_CTA_PAIR && !pair_shape)
         return FP4_ERR_SHAPE;
     if (M == 0 || N == 0)
