@@ -82,6 +82,34 @@ def test_argument_errors_return_before_any_launch(L):
     assert L.fp4_nv_encode_quotient(P, P, P, -1, None) == fp4.ERR_INVALID_ARG
 
 
+def test_gemm_argument_errors_return_before_any_launch(L):
+    """fp4_nvfp4_gemm_ex: shape, kernel choice, pointers and alignment are
+    checked on the host before any CUDA call."""
+    f = L.fp4_nvfp4_gemm_ex
+    ok = (P, P, P, P, P, P)
+    assert f(*ok, 256, 256, 256, P, 7, P, None) == fp4.ERR_INVALID_ARG                  # unknown kernel
+    assert f(*ok, 256, 256, 256, P, fp4.GEMM_AUTO, None, None) == fp4.ERR_INVALID_ARG   # no status word
+    assert f(*ok, -128, 256, 256, P, fp4.GEMM_AUTO, P, None) == fp4.ERR_INVALID_ARG
+    assert f(*ok, 200, 256, 256, P, fp4.GEMM_AUTO, P, None) == fp4.ERR_SHAPE            # M % 128
+    assert f(*ok, 256, 256, 320, P, fp4.GEMM_CTA, P, None) == fp4.ERR_SHAPE             # K % 256
+    assert f(*ok, 384, 256, 256, P, fp4.GEMM_CTA_PAIR, P, None) == fp4.ERR_SHAPE        # pair: M % 256
+    assert f(*ok, 256, 384, 256, P, fp4.GEMM_CTA_PAIR, P, None) == fp4.ERR_SHAPE        # pair: N % 256
+    assert f(*ok, 0, 256, 256, P, fp4.GEMM_AUTO, P, None) == fp4.OK                     # empty D
+    assert f(P, P, P, None, P, P, 256, 256, 256, P, fp4.GEMM_AUTO, P, None) == fp4.ERR_INVALID_ARG
+    assert f(Q, P, P, P, P, P, 256, 256, 256, P, fp4.GEMM_AUTO, P, None) == fp4.ERR_ALIGN
+    assert f(*ok, 256, 256, 256, Q, fp4.GEMM_AUTO, P, None) == fp4.ERR_ALIGN           # d
+
+
+def test_scale_layout_argument_errors(L):
+    f = L.fp4_scales_to_mma_layout
+    assert f(P, -1, 4, P, None) == fp4.ERR_INVALID_ARG
+    assert f(P, 0, 0, P, None) == fp4.OK                   # nothing to write
+    assert f(P, 128, 4, None, None) == fp4.ERR_INVALID_ARG
+    assert f(P, 128, 4, P + 2, None) == fp4.ERR_ALIGN      # out must be 4-byte aligned
+    assert f(P, 128, 5_000_000, P, None) == fp4.ERR_SHAPE  # more scale tiles per band than one grid row
+    assert L.fp4_mma_scales_bytes(130, 5) == 256 * 8       # 128-row bands x 4-block tiles, zero padded
+
+
 def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
     monkeypatch.setattr(fp4, "_lib", None)
     monkeypatch.setattr(fp4, "LIB_PATH", str(tmp_path / "missing.so"))
