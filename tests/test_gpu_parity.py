@@ -124,7 +124,12 @@ def check_full(x: torch.Tensor, search: bool = True):
             assert res["ss"].global_scale.item() == g
             assert_same(res["ss"].scales, s, "search scales")
             assert_same(res["ss"].packed, p, "search packed")
-            assert_same(res["ss"].block_loss, loss.astype(np.float32), "search block loss")
+            # the fp32 rounding of the double loss: a block near +-FLT_MAX has a
+            # loss above FLT_MAX, which both sides round to +inf
+            with np.errstate(over="ignore"):
+                loss32 = loss.astype(np.float32)
+            assert np.array_equal(np.isinf(loss32), np.isinf(res["ss"].block_loss.cpu().numpy()))
+            assert_same(res["ss"].block_loss, loss32, "search block loss")
     return res
 
 

@@ -56,6 +56,11 @@ def test_gemm_is_the_product_of_the_dequantised_operands(oracle_mod):
 
 
 def test_scales_mma_layout_positions(oracle_mod):
+    """The pages do not give this layout (it is the sm100 block-scaled MMA's
+    operand layout), so nothing here can pin it to them: this test only
+    restates the oracle's index formula and checks the padding.  The layout's
+    real anchor is the tensor-core product in the GPU GEMM tests, which reads
+    these bytes: a wrong byte order there gives a wrong D."""
     o = oracle_mod
     rows, nb = 130, 5
     s = (np.arange(rows * nb) % 251 + 1).astype(np.uint8).reshape(rows, nb)
