@@ -1,27 +1,36 @@
 #!/usr/bin/env python
 """Benchmark of the block-scaled FP4 path on B200.
 
-One step = one pass of the whole path over one synthetic tensor (default:
-the 4096 x 4096 bf16 LLM weight matrix, N(0, 0.02) with 0.1 % outliers x50):
+One step = one pass of the whole path over one synthetic workload.  The
+default workload is the whole weight set of a 7B-class decoder (32 layers x
+(4 x 4096x4096 + 3 x 4096x14336) bf16, 224 matrices, 7.78e9 elements,
+15.6 GB), each matrix with its own tensor amax and global scale:
+  grouped tensor amax -> grouped NVFP4 quantise + pack -> grouped MXFP4
+  quantise + pack -> grouped NVFP4 and MXFP4 dequantise (bf16)
+(5 kernel launches).  The single-tensor workloads (--workload) run
   tensor amax -> NVFP4 quantise + pack -> MXFP4 quantise + pack ->
   NVFP4 dequantise (bf16) -> MXFP4 dequantise (bf16) -> NVFP4 scale search
-(6 kernel launches; the amax is shared by the NVFP4 quantiser and the
-search).  `value` is elements of x per second over the whole job, timed on
-the device with CUDA events around each step, L2 flushed (512 MiB write, 256 MiB read)
-between steps, max over ranks; nothing is recorded between the launches of a
-step (an event there would serialise them).  Per-kernel times come from a
-second pass with an event after every launch.  `e2e` times the same step through the same
-C-ABI calls starting from pinned host memory: host->device copy of x, the
-step, device->host copy of every quantised artefact and the status word,
-double-buffered over three streams as a caller streaming batches would run
-it (the upload of step k+1 overlaps step k's kernels and download).
+(6 launches; the amax is shared by the NVFP4 quantiser and the search).
+`value` is elements per second over the whole job, timed on the device
+with CUDA events around each step, L2 flushed (512 MiB write, 256 MiB read)
+between steps, max over ranks; nothing is recorded between the launches of
+a step (an event there would serialise them).  Per-kernel times come from a
+second pass with an event after every launch.  `e2e` times the same step
+through the same C-ABI calls starting from pinned host memory: host->device
+copy of x, the step, device->host copy of every quantised artefact and the
+status word.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle on host cores
 
-Multi-GPU (torchrun): every rank quantises its own tensor (independent
-weight matrices, seeds offset by rank): weak scaling, no collective on the
-data path; one max all-reduce of the timings.
+Multi-GPU (torchrun), two modes:
+  --shard replicas (default)  every rank quantises its own tensor or weight
+      set (independent problems, seeds offset by rank): weak scaling, no
+      collective on the data path; one max all-reduce of the timings.
+  --shard rows  one tensor of a single-tensor workload split by rows across
+      the ranks; the step's only exchange is one max all-reduce of the
+      4-byte tensor amax between the per-rank amax and the NVFP4
+      quantiser / search: strong scaling.
 """
 from __future__ import annotations
 
@@ -60,7 +69,7 @@ GEMM_WORKLOAD = "gemm-8192x4096x14336-nvfp4"
 LAYOUT_WORKLOADS = {"columns-4096x14336-bf16": "columns", "ragged-8192x14335-bf16": "padded",
                     "variants-8192x14336-bf16": "variants"}
 MODEL_WEIGHTS = "model-7b-weights-bf16"  # the whole weight set, grouped calls
-DEFAULT_WORKLOAD = "weight-4096x4096-bf16"
+DEFAULT_WORKLOAD = MODEL_WEIGHTS
 KERNEL_SOURCES = ["block_scaled_fp4_reduce_b200/csrc/fp4_kernels.cuh",
                   "block_scaled_fp4_reduce_b200/csrc/fp4_codec.cuh",
                   "block_scaled_fp4_reduce_b200/csrc/fp4_grouped.cuh"]
@@ -105,15 +114,20 @@ def algorithmic_bytes(w: workloads.Workload) -> dict:
 # ---------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed
-    region (every 100 ms)."""
-    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+    """nvidia-smi samples of SM clock and throttle reasons (every 100 ms,
+    read-only queries).  Sampling starts before the timed region and waits
+    for the first sample, so that even a short region is covered; `stop`
+    keeps the samples whose timestamps fall inside the region (all of them
+    when none does, and says so)."""
+    FIELDS = ["timestamp", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, device: int):
         self.proc = None
         self.out = None
+        self.t0 = self.t1 = None
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             self.target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
@@ -121,7 +135,7 @@ class ClockSampler:
             vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
             self.target = vis.split(",")[device] if vis else str(device)
 
-    def start(self):
+    def start(self, wait_s: float = 5.0):
         try:
             self.out = open(os.path.join("/tmp", f"clocks_{os.getpid()}.csv"), "w")
             self.proc = subprocess.Popen(
@@ -129,10 +143,31 @@ class ClockSampler:
                  "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        t_end = time.time() + wait_s  # until the first sample is written
+        while time.time() < t_end and self.proc.poll() is None:
+            if os.path.getsize(self.out.name) > 0:
+                break
+            time.sleep(0.02)
+
+    def mark(self, begin: bool):
+        """Wall-clock bounds of the timed region."""
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    @staticmethod
+    def _stamp(s: str):
+        try:
+            return datetime.datetime.strptime(s, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)  # one more sample after the region
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -148,18 +183,24 @@ class ClockSampler:
         os.unlink(self.out.name)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        window = "timed region"
+        if self.t0 is not None and self.t1 is not None:
+            inside = [r for r in rows if (t := self._stamp(r[0])) is not None and self.t0 - 0.05 <= t <= self.t1 + 0.15]
+            if inside:
+                rows = inside
+            else:
+                window = "sampler run (no sample inside the timed region)"
 
         def num(s):
             try:
                 return float(s)
             except ValueError:
                 return None
-        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
-        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        reasons = sorted({self.REASONS[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "window": window}
 
 
 # -------------------------------------------------------------- the step --
@@ -226,6 +267,68 @@ class Path:
         st = int(self.status.item())
         if st:
             raise self.fp4.FP4Error(st, "bench step")
+
+
+def shard_rows(rows: int, world: int, rank: int) -> tuple[int, int]:
+    """Rows [r0, r1) of rank `rank` when `rows` rows are split into `world`
+    contiguous shards, the first rows % world of them one row longer."""
+    base, extra = divmod(rows, world)
+    r0 = rank * base + min(rank, extra)
+    return r0, r0 + base + (1 if rank < extra else 0)
+
+
+def sharded_step(local_amax, all_reduce_max, rest):
+    """One row-sharded step: this rank's tensor amax, the max all-reduce
+    that makes it the whole tensor's A (the step's only exchange: the blocks
+    themselves are independent), then the rest of the step with that A.
+    The callables act on the amax in place; `rest` returns the step's
+    result."""
+    a = local_amax()
+    all_reduce_max(a)
+    return rest(a)
+
+
+class ShardedPath(Path):
+    """The single-tensor step on this rank's rows of a tensor split across
+    ranks: fp4_tensor_amax of the shard -> all-reduce(MAX) of the 4-byte A
+    over the ranks (NCCL) -> the NVFP4 quantiser and the search with that A
+    (fp4_*_with_amax), the MXFP4 quantiser and both dequantisers as on one
+    GPU.  Each rank reads only its own memory."""
+    OPS = ["amax", "amax_allreduce"] + OPS[1:]
+
+    def __init__(self, x: torch.Tensor):
+        super().__init__(x)
+        import torch.distributed as dist
+        self.dist = dist
+
+    def twin(self, x2: torch.Tensor) -> "ShardedPath":
+        return ShardedPath(x2)
+
+    def step(self, events=None):
+        def call(i):
+            fn, args = self.calls[i]
+            st = fn(*args)
+            if st != 0:
+                raise self.fp4.FP4Error(st, fn.__name__)
+
+        def local_amax():
+            call(0)
+            if events is not None:
+                events[1].record()
+            return self.amax
+
+        def all_reduce_max(a):
+            self.dist.all_reduce(a, op=self.dist.ReduceOp.MAX)
+            if events is not None:
+                events[2].record()
+
+        def rest(_a):
+            for i in range(1, len(self.calls)):
+                call(i)
+                if events is not None:
+                    events[i + 2].record()
+
+        sharded_step(local_amax, all_reduce_max, rest)
 
 
 class GroupedPath:
@@ -513,13 +616,31 @@ class L2Flush:
             self.r.sum()
 
 
+# Steps of each pass when not given: about a second of timed work.
+DEFAULT_STEPS = {MODEL_WEIGHTS: 40}
+DEFAULT_E2E_STEPS = {MODEL_WEIGHTS: 4}
+
+
+def step_counts(args) -> tuple[int, int, int]:
+    """(timed steps, per-kernel breakdown steps, end-to-end steps)."""
+    K = args.steps if args.steps is not None else DEFAULT_STEPS.get(args.workload, 4000)
+    Kb = max(3, min(K, args.breakdown_steps if args.breakdown_steps is not None else 500))
+    Ke = max(3, min(K, args.e2e_steps if args.e2e_steps is not None else DEFAULT_E2E_STEPS.get(args.workload, 200)))
+    return K, Kb, Ke
+
+
 def run_ours(args, rank: int, world: int, local: int):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    rows_mode = args.shard == "rows" and world > 1
     if world > 1:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    w = workloads.for_rank(WORKLOADS[args.workload], rank)
+    if args.shard == "rows" and (args.workload == MODEL_WEIGHTS or args.workload == GEMM_WORKLOAD
+                                 or args.workload in LAYOUT_WORKLOADS):
+        raise SystemExit("--shard rows takes a single-tensor workload (the weight set shards by matrix: "
+                         "use --shard replicas)")
+    w = WORKLOADS[args.workload] if rows_mode else workloads.for_rank(WORKLOADS[args.workload], rank)
     if args.workload == MODEL_WEIGHTS:
         path = GroupedPath(dev, rank, args.model_layers)
         if args.model_layers != workloads.MODEL_LAYERS:  # a profiling-sized subset of the set
@@ -529,15 +650,23 @@ def run_ours(args, rank: int, world: int, local: int):
         x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
         x_host.copy_(x)
     else:
-        x_host = workloads.generate(w).pin_memory()
+        full = workloads.generate(w)
+        if rows_mode:  # this rank's rows of the one tensor
+            r0, r1 = shard_rows(w.rows, world, rank)
+            full = full[r0:r1]
+        x_host = full.contiguous().pin_memory()
+        del full
         x = x_host.to(dev, non_blocking=False)
         kind = LAYOUT_WORKLOADS.get(args.workload)
         if args.workload == GEMM_WORKLOAD:
             path = GemmPath(x, workloads.generate(workloads.for_rank(workloads.GEMM_W, rank), device=dev))
+        elif kind:
+            path = LayoutPath(x, kind)
         else:
-            path = LayoutPath(x, kind) if kind else Path(x)
+            path = ShardedPath(x) if rows_mode else Path(x)
     flush_l2 = L2Flush(args.flush_mib, dev)
-    nops = len(path.calls)
+    nops = len(path.OPS)
+    K, Kb, Ke = step_counts(args)
 
     warmup = max(args.warmup, 3)
     for _ in range(warmup):
@@ -550,14 +679,14 @@ def run_ours(args, rank: int, world: int, local: int):
     # Nothing is recorded between the launches of a step: an event between
     # two kernels serialises them and forfeits the programmatic dependent
     # launch (each kernel's launch and ramp overlapping its predecessor's
-    # tail), ~26 us of a 100 us step on the default workload.
-    K = args.steps
+    # tail), ~26 us of a 100 us step on the 4096 x 4096 weight.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     clocks = ClockSampler(local)
     clocks.start()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    clocks.mark(True)
     wall0 = time.perf_counter()
     for k in range(K):
         flush_l2()
@@ -566,6 +695,7 @@ def run_ours(args, rank: int, world: int, local: int):
         evs[k][1].record()
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
+    clocks.mark(False)
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
@@ -573,7 +703,6 @@ def run_ours(args, rank: int, world: int, local: int):
     total_ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
 
     # ---- per entry point: a second pass with an event after every launch ---
-    Kb = max(3, min(K, args.breakdown_steps))
     bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nops + 1)] for _ in range(Kb)]
     for k in range(Kb):
         flush_l2()
@@ -584,7 +713,6 @@ def run_ours(args, rank: int, world: int, local: int):
     per_op_ms = [sum(bevs[k][i].elapsed_time(bevs[k][i + 1]) for k in range(Kb)) for i in range(nops)]
 
     # ---- end to end through the same calls from pinned host memory ---------
-    Ke = max(3, min(K, args.e2e_steps))
     h2d = x.numel() * x.element_size()
     d2h = sum(t.numel() * t.element_size() for t in path.results)
     if hasattr(path, "twin"):
@@ -598,23 +726,30 @@ def run_ours(args, rank: int, world: int, local: int):
     if rank != 0:
         return
 
-    n_all = w.numel * world
+    # whole-job elements: every rank's own tensor (replicas), or the one
+    # tensor the ranks share (rows)
+    n_all = w.numel if rows_mode else w.numel * world
+    w_rank = dataclasses.replace(w, rows=x.shape[0]) if rows_mode else w  # rank 0's share, per kernel
     value = n_all * K / (total_ms / 1e3)
     pk = peaks()
-    ab = algorithmic_bytes(w)
+    ab = algorithmic_bytes(w_rank)
     if args.workload == GEMM_WORKLOAD:  # operands, their scales and the fp32 output
         M_, N_, K_ = path.M, path.N, path.K
         ab["nvfp4_gemm"] = (M_ + N_) * (K_ // 2 + K_ // 16) + 4 * M_ * N_
     kernels = {}
     for name, ms in zip(path.OPS, per_op_ms):
         us = ms / Kb * 1e3
-        gbs = ab[name] / (us * 1e-6) / 1e9
-        kernels[name] = {"us": round(us, 3), "share": round(ms / sum(per_op_ms), 4), "gbs": round(gbs, 1),
-                         "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
-    dom = max(kernels, key=lambda k: kernels[k]["us"])
+        entry = {"us": round(us, 3), "share": round(ms / sum(per_op_ms), 4)}
+        if name in ab:
+            gbs = ab[name] / (us * 1e-6) / 1e9
+            entry.update(gbs=round(gbs, 1), frac_hbm=round(gbs / pk["hbm_gbs"], 4))
+        kernels[name] = entry
+    dom = max((k for k in kernels if k in ab), key=lambda k: kernels[k]["us"])
     n_cand = search_candidate_count(x, path.ss_g.item()) if dom == "scale_search" else None
     step_desc = ("amax, nvfp4 quantize, mxfp4 quantize, nvfp4 dequantize (bf16), mxfp4 dequantize (bf16), "
                  "nvfp4 64-candidate scale search")
+    if rows_mode:
+        step_desc = "per-rank amax, max all-reduce of the 4-byte amax (NCCL), then " + step_desc[len("amax, "):]
     if args.workload in LAYOUT_WORKLOADS:
         step_desc = {"columns": "amax, column-wise nvfp4 quantize (Q(W^T)), column-wise mxfp4 quantize, "
                                 "nvfp4 and mxfp4 dequantize of the transposed padded layouts (bf16)",
@@ -634,26 +769,33 @@ def run_ours(args, rank: int, world: int, local: int):
         dom = "nvfp4_gemm"  # the tensor-core kernel is the one this workload is about
     if LAYOUT_WORKLOADS.get(args.workload) == "variants" and dom == "nvfp4_quantize":
         # four over six: two screened candidates per block, ALU-bound like the search
-        n_cand = 2 * (w.numel // 16)
-        roof = roofline_for("scale_search", kernels[dom], w, pk, n_cand)
+        n_cand = 2 * (w_rank.numel // 16)
+        roof = roofline_for("scale_search", kernels[dom], w_rank, pk, n_cand)
         roof["kernel"] = "nvfp4_quantize_four_over_six"
         roof["work"] = roof["work"].replace("distinct candidates", "candidates (2 per block)")
     else:
-        roof = roofline_for(dom, kernels[dom], w, pk, n_cand, gemm_mnk)
+        roof = roofline_for(dom, kernels[dom], w_rank, pk, n_cand, gemm_mnk)
     line = {
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": K,
-        "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "strong" if rows_mode else "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name if world == 1 else WORKLOADS[args.workload].name,
+        "config": {"workload": w.name if world == 1 or rows_mode else WORKLOADS[args.workload].name,
                    "description": WORKLOADS[args.workload].description,
                    "shape": ([[r, c] for r, c in workloads.MODEL_MATRICES] if args.workload == MODEL_WEIGHTS
                              else [w.rows, w.cols]),
                    "input_dtype": str(w.dtype).replace("torch.", ""),
+                   "arithmetic": "fp32 (element quotients, block-scale decisions and dequantised products)",
                    "step": step_desc,
-                   "l2": f"flushed between steps outside the timed events ({args.flush_mib} MiB write, "
-                         f"then {args.flush_mib // 2} MiB read)",
-                   "parallelism": f"replicas x{world} (independent tensors)" if world > 1 else "single GPU"},
-        "hbm_gbs_step": sum(ab[o] for o in path.OPS) / (total_ms / K * 1e-3) / 1e9,
+                   "l2": (f"flushed between steps outside the timed events ({args.flush_mib} MiB write, "
+                          f"then {args.flush_mib // 2} MiB read)" if args.flush_mib else "not flushed") +
+                         (f"; input {w.numel * w.dtype.itemsize / 1e9:.1f} GB, larger than the 126 MB L2"
+                          if w.numel * w.dtype.itemsize > 126e6 else ""),
+                   "parallelism": (f"rows split over {world} ranks, one max all-reduce of the amax per step"
+                                   if rows_mode else
+                                   f"replicas x{world} (independent tensors)" if world > 1 else "single GPU")},
+        "hbm_gbs_step": sum(ab[o] for o in path.OPS if o in ab) * (world if rows_mode else 1)
+                        / (total_ms / K * 1e-3) / 1e9,
         "kernels": kernels,
         "kernels_timing": (f"second pass of {Kb} steps, L2 flushed between steps, an event after every launch: "
                            "the events serialise the launches, so each time includes its own launch and ramp "
@@ -665,6 +807,9 @@ def run_ours(args, rank: int, world: int, local: int):
         "clocks": clk,
         "wall_s_timed": wall,
     }
+    if dom != "nvfp4_quantize" and "nvfp4_quantize" in kernels and "nvfp4_quantize" in ab and not gemm_mnk \
+            and LAYOUT_WORKLOADS.get(args.workload) != "variants":
+        line["roofline_nvfp4_quantize"] = roofline_for("nvfp4_quantize", kernels["nvfp4_quantize"], w_rank, pk)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
     print(json.dumps(line), flush=True)
@@ -796,24 +941,64 @@ def oracle_sample_source(w: workloads.Workload):
     return workloads.generate(w), _oracle_step, w.name
 
 
-def cpu_baseline(w: workloads.Workload, budget_s: float = 15.0) -> dict:
-    """The oracle as it stands (single-threaded C) on a bounded row sample of
-    the same workload, the same steps; elements/s."""
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def time_oracle_rows(step, xo, r0: int, rows: int, threads: int) -> float:
+    """Seconds for `step` over rows [r0, r0 + rows) of xo, split into
+    `threads` contiguous row ranges run concurrently, one per thread (the
+    oracle is C called through ctypes, which releases the GIL for the
+    duration of each call).  The oracle itself is unchanged: each thread
+    runs the plain single-threaded code on its own rows."""
+    import concurrent.futures
+    bounds = [r0 + shard_rows(rows, threads, t)[0] for t in range(threads)] + [r0 + rows]
+    parts = [np.ascontiguousarray(xo[bounds[t]:bounds[t + 1]]) for t in range(threads)]
+    parts = [p for p in parts if p.shape[0]]
+    t0 = time.perf_counter()
+    if len(parts) == 1:
+        step(parts[0])
+    else:
+        with concurrent.futures.ThreadPoolExecutor(max_workers=len(parts)) as ex:
+            for f in [ex.submit(step, p) for p in parts]:
+                f.result()
+    return time.perf_counter() - t0
+
+
+def _rows_for(step, xo, budget_s: float, threads: int) -> int:
+    """Rows that keep one timing of `step` on `threads` threads near
+    budget_s, from a 32-row probe on one thread."""
+    R = xo.shape[0]
+    t_row = time_oracle_rows(step, xo, 0, min(R, 32), 1) / min(R, 32)
+    return int(max(min(threads, R), min(R, budget_s * threads / max(t_row, 1e-6))))
+
+
+def cpu_baseline(w: workloads.Workload, budget_s: float = 8.0) -> dict:
+    """The oracle as it stands (plain single-threaded C) on bounded row
+    samples of the same workload, the same steps, in elements/s: first on
+    one core, then on every host core at once (one row range per thread)."""
     import oracle
     oracle.build()
     x, step, what = oracle_sample_source(w)
     xo = workloads.as_oracle_array(x)
     R, C = xo.shape
-    rows = 32
-    t0 = time.perf_counter()
-    step(xo[:rows])
-    t1 = time.perf_counter() - t0
-    rows = int(max(4, min(R, rows * budget_s / max(t1, 1e-3) / 2)))
-    t0 = time.perf_counter()
-    step(np.ascontiguousarray(xo[:rows]))
-    dt = time.perf_counter() - t0
-    return {"value": rows * C / dt, "unit": "elements/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {rows} of {R} rows ({rows * C} elements) of {what}, whole step, {dt:.1f} s",
+    rows1 = _rows_for(step, xo, budget_s, 1)
+    dt1 = time_oracle_rows(step, xo, 0, rows1, 1)
+    cores = host_cores()
+    rowsn = min(R, rows1 * cores)
+    reps, dtn = 0, 0.0
+    while reps == 0 or dtn < budget_s / 2:  # repeat a sample the tensor's rows cap
+        dtn += time_oracle_rows(step, xo, 0, rowsn, cores)
+        reps += 1
+    return {"value": reps * rowsn * C / dtn, "unit": "elements/s", "cores": cores, "kind": "oracle",
+            "sample": (f"first {rowsn} of {R} rows ({rowsn * C} elements) of {what}, whole step, split over "
+                       f"{cores} threads, {reps} time(s), {dtn:.1f} s"),
+            "one_core": {"value": rows1 * C / dt1, "cores": 1,
+                         "sample": f"first {rows1} rows ({rows1 * C} elements), {dt1:.1f} s"},
             "cpu": _cpu_model()}
 
 
@@ -829,7 +1014,9 @@ def _cpu_model() -> str:
 
 
 def run_reference(args, rank: int, world: int):
-    """--impl reference: the CPU oracle on the host cores, rank 0 only."""
+    """--impl reference: the CPU oracle on every host core, rank 0 only;
+    each step a bounded row sample of the workload split into one row
+    range per core (the plain single-threaded oracle on each)."""
     if rank != 0:
         return
     import oracle
@@ -838,27 +1025,26 @@ def run_reference(args, rank: int, world: int):
     x, step, what = oracle_sample_source(w)
     xo = workloads.as_oracle_array(x)
     R, C = xo.shape
+    cores = host_cores()
     total_budget = 120.0
-    t0 = time.perf_counter()
-    step(np.ascontiguousarray(xo[:32]))
-    t_row = (time.perf_counter() - t0) / 32
-    steps, warm = args.steps, max(args.warmup, 0)
-    rows = int(max(1, min(R, total_budget / max(t_row, 1e-4) / (steps + warm))))
+    steps = args.steps if args.steps is not None else 20
+    warm = max(args.warmup, 0)
+    rows = min(R, _rows_for(step, xo, total_budget / (steps + warm), cores))
     for _ in range(warm):
-        step(np.ascontiguousarray(xo[:rows]))
-    t0 = time.perf_counter()
+        time_oracle_rows(step, xo, 0, rows, cores)
+    dt = 0.0
     for k in range(steps):
         r0 = (k * rows) % max(1, R - rows + 1)
-        step(np.ascontiguousarray(xo[r0:r0 + rows]))
-    dt = time.perf_counter() - t0
+        dt += time_oracle_rows(step, xo, r0, rows, cores)
     value = rows * C * steps / dt
     line = {
         "metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": steps,
         "warmup": warm, "ms_per_step": dt / steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
         "config": {"workload": w.name, "description": w.description, "shape": [w.rows, w.cols]},
-        "cpu_baseline": {"value": value, "unit": "elements/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{rows} rows x {C} per step (bounded sample of {what})",
+        "cpu_baseline": {"value": value, "unit": "elements/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} rows x {C} per step, split over {cores} threads "
+                                   f"(bounded sample of {what})",
                          "cpu": _cpu_model()},
         "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -871,14 +1057,19 @@ import numpy as np  # noqa: E402  (used by the reference leg)
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 40 on the weight set, 4000 on the single tensors)")
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
-    ap.add_argument("--e2e-steps", type=int, default=200)
-    ap.add_argument("--breakdown-steps", type=int, default=500,
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="steps of the end-to-end pass (default: 4 on the weight set, 200 otherwise)")
+    ap.add_argument("--breakdown-steps", type=int, default=None,
                     help="steps of the per-entry-point pass (events between launches)")
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget", type=float, default=8.0,
+                    help="seconds of each CPU-baseline leg (one core, then all cores)")
+    ap.add_argument("--shard", choices=["replicas", "rows"], default="replicas",
+                    help="multi-GPU mode: each rank its own tensor, or one tensor split by rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--model-layers", type=int, default=workloads.MODEL_LAYERS,
                     help="layers of the 7B weight set in model-7b-weights-bf16 (fewer only for profiler runs)")

@@ -36,55 +36,6 @@ fp4_status check_shape(int64_t rows, int64_t cols, int64_t block)
 }
 
 
-// Tensor amax (one launch) into *amax.
-fp4_status launch_amax(const void *x, fp4_dtype dt, int64_t n, uint32_t *ws, float *amax,
-                       int32_t *status, cudaStream_t stream)
-{
-    const int64_t elems_per_vec = dt == FP4_BF16 ? 16 : 8; // one 32-byte vector
-    const int64_t nvec = n / elems_per_vec;
-    const int64_t per_cta = (int64_t)kThreads * 4;
-    int grid;
-    if (dt == FP4_BF16)
-        grid = grid_for(fp4::amax_kernel<uint16_t>, nvec, per_cta);
-    else
-        grid = grid_for(fp4::amax_kernel<float>, nvec, per_cta);
-    if (grid <= 0)
-        return FP4_ERR_CUDA;
-    if (grid > kMaxPartials)
-        grid = kMaxPartials;
-    if (dt == FP4_BF16)
-        return launch(fp4::amax_kernel<uint16_t>, grid, stream, static_cast<const uint16_t *>(x), n,
-                      ws, amax, status);
-    return launch(fp4::amax_kernel<float>, grid, stream, static_cast<const float *>(x), n, ws, amax,
-                  status);
-}
-
-template <typename T>
-fp4_status launch_nv_quantize_t(const T *x, int64_t n, const float *amax, uint8_t *packed,
-                                uint8_t *scales, float *global_scale, int32_t *status,
-                                cudaStream_t stream)
-{
-    uint2 *pk = reinterpret_cast<uint2 *>(packed);
-    return for_chunks(n / 16, [&](int64_t first, int count) {
-        const int grid = grid_for(fp4::nvfp4_quantize_kernel<T>, count, (int64_t)kThreads * 2);
-        if (grid <= 0)
-            return FP4_ERR_CUDA;
-        return launch(fp4::nvfp4_quantize_kernel<T>, grid, stream, x + first * 16, count, amax,
-                      pk + first, scales + first, global_scale, status);
-    });
-}
-
-fp4_status launch_nv_quantize(const void *x, fp4_dtype dt, int64_t n, const float *amax,
-                              uint8_t *packed, uint8_t *scales, float *global_scale,
-                              int32_t *status, cudaStream_t stream)
-{
-    if (dt == FP4_BF16)
-        return launch_nv_quantize_t(static_cast<const uint16_t *>(x), n, amax, packed, scales,
-                                    global_scale, status, stream);
-    return launch_nv_quantize_t(static_cast<const float *>(x), n, amax, packed, scales,
-                                global_scale, status, stream);
-}
-
 } // namespace
 
 namespace {

@@ -218,9 +218,11 @@ fp4_status fp4_scale_search_with_amax(const void *x, fp4_dtype dtype, int64_t ro
  * for every shape -- a shape needing more would get FP4_ERR_WORKSPACE).
  * All calls on a device share that array: calls whose kernels overlap on
  * the GPU race and must be ordered by the caller.  Each call clears the
- * array's counter word on `stream` before its kernels.  The first call on a
- * device looks up the array's address with that device current; make it
- * before any stream capture. */
+ * array's counter word on `stream` before its kernels.  Every call looks up
+ * the array's address in the current context (a non-primary context, or a
+ * context created again after cudaDeviceReset, gets its own copy); the first
+ * call in a context also loads the library's device code there, so make it
+ * before any stream capture begins. */
 fp4_status fp4_nvfp4_quantize_noalloc(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
                                       uint8_t *packed, uint8_t *scales, float *global_scale,
                                       int32_t *status, cudaStream_t stream);
