@@ -677,9 +677,9 @@ def run_ours(args, rank: int, world: int, local: int):
 
     # ---- timed region: K steps, one event pair around each step -----------
     # Nothing is recorded between the launches of a step: an event between
-    # two kernels serialises them and forfeits the programmatic dependent
-    # launch (each kernel's launch and ramp overlapping its predecessor's
-    # tail), ~26 us of a 100 us step on the 4096 x 4096 weight.
+    # two kernels makes each launch wait for its predecessor's completion,
+    # where the programmatic serialisation lets it launch as the
+    # predecessor's CTAs retire.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     clocks = ClockSampler(local)
     clocks.start()

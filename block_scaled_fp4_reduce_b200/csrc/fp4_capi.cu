@@ -234,7 +234,8 @@ fp4_status fp4_dequantize(fp4_format fmt, const uint8_t *packed, const uint8_t *
     const uint2 *pk = reinterpret_cast<const uint2 *>(packed);
     auto run = [&](auto kernel, auto *yt) {
         return for_chunks(n / 16, [&](int64_t first, int count) {
-            const int grid = grid_for(kernel, count, (int64_t)kThreads * 4);
+            const int grid = grid_for(kernel, count, (int64_t)kThreads * fp4::kDequantUnits, kThreads, 0,
+                                      fp4::kDequantCtasPerSm);
             if (grid <= 0)
                 return FP4_ERR_CUDA;
             return launch(kernel, grid, stream, pk + first, scales + (nv ? first : first / 2),

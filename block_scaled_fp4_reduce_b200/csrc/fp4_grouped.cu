@@ -122,18 +122,17 @@ fp4_status nv_grouped_with_amax(const fp4_quant_item *items, int n_items,
 {
     return plan<fp4::NvGroup>(
         n_items, [&](int it) { return items[it].rows * items[it].cols / 16; },
-        [&](fp4::NvGroup &t, int k, int it, int64_t off, int64_t) {
+        [&](fp4::NvGroup &t, int k, int it, int64_t off, int64_t take) {
             t.x[k] = static_cast<const T *>(items[it].x) + off * 16;
             t.packed[k] = reinterpret_cast<uint2 *>(items[it].packed) + off;
             t.scales[k] = items[it].scales + off;
             t.amax[k] = amax_words + it;
             t.global_scale[k] = items[it].global_scale;
+            t.tile_first[k + 1] = t.tile_first[k] + fp4::grouped_tile_count(take, fp4::kNvGroupedU);
         },
         [&](const fp4::NvGroup &t) {
-            int64_t work = t.first[t.n];
-            if (work < t.n) // one thread per entry publishes its g
-                work = t.n;
-            const int grid = grid_for(fp4::nvfp4_quantize_grouped_kernel<T>, work, (int64_t)kThreads * 2);
+            // one CTA at least: its first threads publish every entry's g
+            const int grid = grid_for(fp4::nvfp4_quantize_grouped_kernel<T>, t.tile_first[t.n], 1);
             if (grid <= 0)
                 return FP4_ERR_CUDA;
             return launch(fp4::nvfp4_quantize_grouped_kernel<T>, grid, stream, t, status);
@@ -166,14 +165,14 @@ fp4_status mx_grouped(const fp4_quant_item *items, int n_items, int32_t *status,
 {
     return plan<fp4::MxGroup>(
         n_items, [&](int it) { return items[it].rows * items[it].cols / 32; },
-        [&](fp4::MxGroup &t, int k, int it, int64_t off, int64_t) {
+        [&](fp4::MxGroup &t, int k, int it, int64_t off, int64_t take) {
             t.x[k] = static_cast<const T *>(items[it].x) + off * 32;
             t.packed[k] = reinterpret_cast<uint4 *>(items[it].packed) + off;
             t.scales[k] = items[it].scales + off;
+            t.tile_first[k + 1] = t.tile_first[k] + fp4::grouped_tile_count(take, fp4::kMxGroupedU);
         },
         [&](const fp4::MxGroup &t) {
-            const int grid = grid_for(fp4::mxfp4_quantize_grouped_kernel<T, kCeil>, t.first[t.n],
-                                      (int64_t)kThreads * 2);
+            const int grid = grid_for(fp4::mxfp4_quantize_grouped_kernel<T, kCeil>, t.tile_first[t.n], 1);
             if (grid <= 0)
                 return FP4_ERR_CUDA;
             return launch(fp4::mxfp4_quantize_grouped_kernel<T, kCeil>, grid, stream, t, status);
@@ -185,15 +184,16 @@ fp4_status dq_grouped(const fp4_dequant_item *items, int n_items, cudaStream_t s
 {
     return plan<fp4::DqGroup>(
         n_items, [&](int it) { return items[it].rows * items[it].cols / 16; },
-        [&](fp4::DqGroup &t, int k, int it, int64_t off, int64_t) {
+        [&](fp4::DqGroup &t, int k, int it, int64_t off, int64_t take) {
             t.packed[k] = reinterpret_cast<const uint2 *>(items[it].packed) + off;
             t.scales[k] = items[it].scales + (kNv ? off : off / 2);
             t.global_scale[k] = items[it].global_scale;
             t.y[k] = static_cast<TOut *>(items[it].y) + off * 16;
+            t.tile_first[k + 1] = t.tile_first[k] + fp4::grouped_tile_count(take, fp4::kDequantUnits);
         },
         [&](const fp4::DqGroup &t) {
-            const int grid = grid_for(fp4::dequantize_grouped_kernel<kNv, TOut>, t.first[t.n],
-                                      (int64_t)kThreads * 4);
+            const int grid = grid_for(fp4::dequantize_grouped_kernel<kNv, TOut>, t.tile_first[t.n], 1,
+                                      kThreads, 0, fp4::kDequantCtasPerSm);
             if (grid <= 0)
                 return FP4_ERR_CUDA;
             return launch(fp4::dequantize_grouped_kernel<kNv, TOut>, grid, stream, t);

@@ -20,10 +20,14 @@
 // Everything is HBM-bound streaming except the scale search (issue-bound).
 //
 // Launch chaining: every kernel is launched with programmatic stream
-// serialisation.  It lets the next kernel on the stream launch at once
-// (griddepcontrol.launch_dependents) and waits for the previous one
-// (griddepcontrol.wait) before its first global memory access, so launch
-// latency and the CTA ramp overlap the previous kernel's tail.  Loads after
+// serialisation and waits for the previous kernel on the stream
+// (griddepcontrol.wait) before its first global memory access.  No kernel
+// triggers its dependents early (griddepcontrol.launch_dependents): the
+// persistent grids here leave room on the SMs, and a dependent grid launched
+// at the start of its predecessor parks CTAs there for the predecessor's
+// whole run, which measured slower -- 18.1 against 16.0 ms per step on the
+// 7B weight set, 79.5 against 72.4 us on the 4096 x 4096 weight.  The
+// dependent grid is launched as the previous one's CTAs exit.  Loads after
 // the wait go through L2 (.cg / coherent), never the non-coherent path.
 #pragma once
 
@@ -163,43 +167,11 @@ __device__ __forceinline__ void stream_units(int n, Load &&load, Work &&work)
     }
 }
 
-// The same with a blocked distribution: CTA c takes one contiguous range of
-// units (whole tiles of blockDim * U consecutive units), and within a tile
-// consecutive threads take consecutive units.  A thread's units then lie in
-// one short stretch of the unit space (used where per-stretch state, such as
-// the matrix of a grouped launch, is costly to switch).
-template <int U, typename Load, typename Work>
-__device__ __forceinline__ void stream_units_blocked(int n, Load &&load, Work &&work)
-{
-    const int tile = (int)blockDim.x * U;
-    const int tiles = (n + tile - 1) / tile;
-    const int per_cta = (tiles + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int t0 = (int)blockIdx.x * per_cta;
-    const int t1 = min(t0 + per_cta, tiles);
-    for (int t = t0; t < t1; ++t) {
-        const int base = t * tile + (int)threadIdx.x;
-        if (base + (U - 1) * (int)blockDim.x < n) {
-#pragma unroll
-            for (int u = 0; u < U; ++u)
-                load(u, base + u * (int)blockDim.x);
-#pragma unroll
-            for (int u = 0; u < U; ++u)
-                work(u, base + u * (int)blockDim.x);
-        } else {
-            for (int i = base; i < n; i += (int)blockDim.x) {
-                load(0, i);
-                work(0, i);
-            }
-        }
-    }
-}
-
 // Largest unit count one launch of a stream_units kernel takes.
 constexpr int64_t kMaxUnitsPerLaunch = (int64_t)1 << 30;
 
 __device__ __forceinline__ void pdl_begin()
 {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
@@ -417,7 +389,11 @@ __global__ void __launch_bounds__(kThreads)
 
 // ---------------------------------------------------------------------------
 // Dequantise.  One thread per 16 codes (8 packed bytes) -> 16 outputs (one
-// 32-byte bf16 store or two fp32 ones), four units in flight per thread.
+// 32-byte bf16 store or two fp32 ones), two units in flight per thread, at
+// most kDequantCtasPerSm CTAs per SM: the kernel writes 3.6 bytes for every
+// byte it reads, and fewer threads in flight measured faster on the
+// 8192 x 14336 activation (NVFP4 55.2 against 58.9 us with four units per
+// thread at full occupancy, MXFP4 54.3 against 57.4).
 // NVFP4: p * s_b is exact in any format with 6 significant bits and the
 // range 2^-10 .. 2688, so it is formed by the mixed-precision
 // `fma.rn.f32.f16` (f16 code value x f16 scale + -0, the -0 keeping the
@@ -501,6 +477,9 @@ __device__ __forceinline__ void dequant_unit(uint2 pk, uint32_t sbyte, uint64_t 
     }
 }
 
+constexpr int kDequantUnits = 2;
+constexpr int kDequantCtasPerSm = 4;
+
 template <bool kNv, typename TOut>
 __global__ void __launch_bounds__(kThreads)
     dequantize_kernel(const uint2 *__restrict__ packed, const uint8_t *__restrict__ scales,
@@ -509,9 +488,9 @@ __global__ void __launch_bounds__(kThreads)
     pdl_begin();
     const float g = kNv ? __ldcg(global_scale) : 1.0f;
     const uint64_t g2 = pack2(g, g);
-    uint2 pk[4];
-    uint32_t sbyte[4];
-    stream_units<4>(
+    uint2 pk[kDequantUnits];
+    uint32_t sbyte[kDequantUnits];
+    stream_units<kDequantUnits>(
         n_units,
         [&](int u, int i) {
             pk[u] = __ldcg(packed + i);

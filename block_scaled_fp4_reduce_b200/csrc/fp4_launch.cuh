@@ -69,23 +69,27 @@ template <typename K> int resident_ctas(K kernel, int dev, int block = kThreads,
 }
 
 // Persistent grid: enough CTAs for `work` items at `per_cta` items each,
-// at most SMs x resident CTAs, at least one.
+// at most SMs x resident CTAs (and at most SMs x max_per_sm when given), at
+// least one.
 template <typename K>
-int grid_for(K kernel, int64_t work, int64_t per_cta, int block = kThreads, size_t smem = 0)
+int grid_for(K kernel, int64_t work, int64_t per_cta, int block = kThreads, size_t smem = 0, int max_per_sm = 0)
 {
     int dev = 0;
     const int sms = sm_count(dev);
     if (sms <= 0)
         return -1;
-    const int64_t cap = (int64_t)sms * resident_ctas(kernel, dev, block, smem);
+    int per_sm = resident_ctas(kernel, dev, block, smem);
+    if (max_per_sm > 0 && per_sm > max_per_sm)
+        per_sm = max_per_sm;
+    const int64_t cap = (int64_t)sms * per_sm;
     int64_t want = (work + per_cta - 1) / per_cta;
     if (want < 1)
         want = 1;
     return (int)(want < cap ? want : cap);
 }
 
-// Launch with programmatic stream serialisation: the kernel may start while
-// the previous kernel on the stream finishes; it waits for it
+// Launch with programmatic stream serialisation: the kernel is launched as
+// the previous kernel on the stream retires its CTAs, and waits for it
 // (griddepcontrol.wait) before touching memory.
 template <typename... KArgs, typename... Args>
 fp4_status launch_cfg(void (*kernel)(KArgs...), dim3 grid, int block, size_t smem,

@@ -33,13 +33,12 @@ fp4_status nv_padded(const T *x, int64_t rows, int64_t cols, const float *amax, 
                      uint8_t *scales, float *global_scale, int32_t *status, cudaStream_t stream)
 {
     const int64_t nbp = ceil_div(cols, 16);
-    constexpr size_t kSmem = fp4::pad_smem_bytes<T>(16);
     return for_row_chunks(rows, nbp, [&](int64_t r0, int64_t nr) {
         const int n = (int)(nr * nbp);
-        const int grid = grid_for(fp4::nvfp4_quantize_padded_kernel<T>, n, fp4::kPadTile, fp4::kPadTile, kSmem);
+        const int grid = grid_for(fp4::nvfp4_quantize_padded_kernel<T>, n, (int64_t)kThreads * fp4::pad_units<16>());
         if (grid <= 0)
             return FP4_ERR_CUDA;
-        return launch_cfg(fp4::nvfp4_quantize_padded_kernel<T>, grid, fp4::kPadTile, kSmem, stream,
+        return launch(fp4::nvfp4_quantize_padded_kernel<T>, grid, stream,
                           x + r0 * cols, cols, fp4::fast_div_for((uint32_t)nbp), n, amax,
                           reinterpret_cast<uint2 *>(packed) + r0 * nbp, scales + r0 * nbp, global_scale,
                           status);
@@ -51,14 +50,13 @@ fp4_status mx_padded(const T *x, int64_t rows, int64_t cols, uint8_t *packed, ui
                      int32_t *status, cudaStream_t stream)
 {
     const int64_t nbp = ceil_div(cols, 32);
-    constexpr size_t kSmem = fp4::pad_smem_bytes<T>(32);
     return for_row_chunks(rows, nbp, [&](int64_t r0, int64_t nr) {
         const int n = (int)(nr * nbp);
-        const int grid = grid_for(fp4::mxfp4_quantize_padded_kernel<T, kCeil>, n, fp4::kPadTile,
-                                  fp4::kPadTile, kSmem);
+        const int grid = grid_for(fp4::mxfp4_quantize_padded_kernel<T, kCeil>, n,
+                                  (int64_t)kThreads * fp4::pad_units<32>());
         if (grid <= 0)
             return FP4_ERR_CUDA;
-        return launch_cfg(fp4::mxfp4_quantize_padded_kernel<T, kCeil>, grid, fp4::kPadTile, kSmem, stream,
+        return launch(fp4::mxfp4_quantize_padded_kernel<T, kCeil>, grid, stream,
                           x + r0 * cols, cols, fp4::fast_div_for((uint32_t)nbp), n,
                           reinterpret_cast<uint4 *>(packed) + r0 * nbp, scales + r0 * nbp, status);
     });

@@ -38,24 +38,24 @@ constexpr int32_t kStatusTimeout = 8;
 // Ragged rows.  Block b of the row-padded [R, Kp] matrix is row b / nbp,
 // block b % nbp of that row; it covers the elements [f, f + cnt) of the flat
 // input, f = (b / nbp) K + (b % nbp) G, cnt = min(G, K - (b % nbp) G), and
-// reads +0 past them.  Consecutive blocks cover consecutive flat elements,
-// so a tile of kPadTile blocks is one contiguous span of x.  The kernels
-// stage that span (rounded out to 32-byte vectors) in shared memory with
-// aligned 256-bit loads, or, for dequantisation, assemble it there and
-// write its interior back with 256-bit stores.  In shared memory each
-// 32-byte vector takes 36 bytes (one pad word per eight): a block that
+// reads +0 past them.  The quantisers read every block from its window of
+// aligned 32-byte vectors in registers (PadWin below).  Consecutive units
+// cover consecutive flat elements, so the dequantiser's tile of kPadTile
+// units is one contiguous span of y: it assembles the span in shared memory
+// and writes its interior back with 256-bit stores.  In shared memory each
+// 32-byte vector takes 36 bytes (one pad word per eight): a unit that
 // starts 32 bytes after its neighbour's then starts in another bank, so the
 // word accesses of a warp are conflict-free.
 // ---------------------------------------------------------------------------
-constexpr int kPadTile = 256; // blocks (quantise) or 16-code units (dequantise) per tile
+constexpr int kPadTile = 256; // 16-code units per tile of the dequantiser
 
 // Word w of the staged span lives at word w + w / 8.
 __device__ __forceinline__ int pad_word(int w) { return w + (w >> 3); }
 
 template <typename T> constexpr int pad_smem_bytes(int G)
 {
-    // span of kPadTile blocks of G elements, one vector of slack at each end,
-    // and room for the last block's reads past its real elements
+    // span of kPadTile units of G elements, one vector of slack at each end,
+    // and room for the last unit's writes past its real elements
     return (kPadTile * G * (int)sizeof(T) / 32 + 4) * 36;
 }
 
@@ -101,101 +101,92 @@ __device__ __forceinline__ int64_t pad_block_start(int b, const FastDiv &nbp, in
     return (int64_t)r * K + c0;
 }
 
-// Stages the flat elements [base, base + nvec * per_vec) of x into smem
-// (36-byte slots); elements at or past n read as +0.  base is 32-byte
-// aligned in memory; it precedes the tile's first element by less than one
-// vector, and lies before x only when x is a later row chunk of the caller's
-// tensor (memory of the same tensor; those words are never used).
-template <typename T>
-__device__ __forceinline__ void stage_span(const T *x, int64_t n, int64_t base, int nvec, uint32_t *sw)
+// A ragged block read straight from global memory.  Every block of a row
+// starts at the same offset within a 32-byte vector (row r starts at
+// element r K, and blocks are G elements = a whole number of vectors apart),
+// so a block lies in the kVecs aligned vectors from the one that holds its
+// first element: one more vector than the block fills.  The window is loaded
+// with 256-bit loads (the vector a block shares with its neighbour is read
+// twice, the second time from L2) and the block is cut out of it with
+// funnel shifts.  The word shift is the same for all the blocks of a row, so
+// a warp inside one row takes one branch of the switch below.  A vector that
+// starts at or past the end of the launch's rows is not read (zeros); the
+// vector that holds the last element is read whole (an aligned 32-byte
+// vector never crosses a page), and elements past the block's count are
+// masked to +0.
+template <typename T, int G> struct PadWin {
+    static constexpr int kVecs = G * (int)sizeof(T) / 32 + 1;
+    uint32_t w[kVecs * 8];
+    int shift; // byte offset of the block's first element in the window
+    int cnt;   // real elements of the block (the rest is padding)
+};
+
+template <typename T, int G>
+__device__ __forceinline__ void pad_win_load(const T *x, const char *x_end, int b, const FastDiv &nbp, int64_t K,
+                                             PadWin<T, G> &pw)
 {
-    constexpr int kPerVec = 32 / (int)sizeof(T);
-    for (int v = (int)threadIdx.x; v < nvec; v += (int)blockDim.x) {
-        const int64_t e = base + (int64_t)v * kPerVec;
-        uint32_t w[8];
-        if (e + kPerVec <= n) {
-            ldg_v8(x + e, w);
+    const int64_t f = pad_block_start(b, nbp, K, G, pw.cnt);
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(x + f);
+    const char *ab = reinterpret_cast<const char *>(pa & ~(uintptr_t)31);
+    pw.shift = (int)(pa & 31u);
+#pragma unroll
+    for (int m = 0; m < PadWin<T, G>::kVecs; ++m) {
+        if (ab + 32 * m < x_end) {
+            ldg_v8(ab + 32 * m, &pw.w[8 * m]);
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if constexpr (sizeof(T) == 2) {
-                    const uint32_t lo = e + 2 * i < n ? (uint32_t)__ldcg(reinterpret_cast<const unsigned short *>(x + e + 2 * i)) : 0u;
-                    const uint32_t hi = e + 2 * i + 1 < n ? (uint32_t)__ldcg(reinterpret_cast<const unsigned short *>(x + e + 2 * i + 1)) : 0u;
-                    w[i] = lo | (hi << 16);
-                } else {
-                    w[i] = e + i < n ? __float_as_uint(__ldcg(x + e + i)) : 0u;
-                }
-            }
+            for (int i = 0; i < 8; ++i)
+                pw.w[8 * m + i] = 0u;
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            sw[v * 9 + i] = w[i];
     }
 }
 
-// Block of N elements starting at staged element q (cnt of them real, the
-// rest +0) as a Blk.
-template <typename T, int N>
-__device__ __forceinline__ void staged_block(const uint32_t *sw, int q, int cnt, Blk<T, N> &k)
+// Words [S, S + W] of the window funnel-shifted right by sh bits.
+template <int S, int W, int N>
+__device__ __forceinline__ void pad_win_cut(const uint32_t (&w)[N], uint32_t sh, uint32_t *out)
 {
-    if constexpr (sizeof(T) == 2) {
-        const int w0 = q >> 1;
-        const uint32_t sh = (uint32_t)(q & 1) * 16u;
-        uint32_t prev = sw[pad_word(w0)];
+    static_assert(S + W < N, "window too short");
 #pragma unroll
-        for (int i = 0; i < N / 2; ++i) {
-            const uint32_t next = sw[pad_word(w0 + i + 1)];
-            k.w[i] = __funnelshift_r(prev, next, sh);
-            prev = next;
-        }
-        if (cnt < N) {
+    for (int i = 0; i < W; ++i)
+        out[i] = __funnelshift_r(w[S + i], w[S + i + 1], sh);
+}
+
+template <typename T, int G>
+__device__ __forceinline__ void pad_win_block(const PadWin<T, G> &pw, Blk<T, G> &k)
+{
+    constexpr int W = G * (int)sizeof(T) / 4;
+    const uint32_t sh = (uint32_t)(pw.shift & 3) * 8u;
+    switch (pw.shift >> 2) {
+    case 0: pad_win_cut<0, W>(pw.w, sh, k.w); break;
+    case 1: pad_win_cut<1, W>(pw.w, sh, k.w); break;
+    case 2: pad_win_cut<2, W>(pw.w, sh, k.w); break;
+    case 3: pad_win_cut<3, W>(pw.w, sh, k.w); break;
+    case 4: pad_win_cut<4, W>(pw.w, sh, k.w); break;
+    case 5: pad_win_cut<5, W>(pw.w, sh, k.w); break;
+    case 6: pad_win_cut<6, W>(pw.w, sh, k.w); break;
+    default: pad_win_cut<7, W>(pw.w, sh, k.w); break;
+    }
+    if (pw.cnt < G) {
 #pragma unroll
-            for (int i = 0; i < N / 2; ++i) {
-                if (2 * i >= cnt)
+        for (int i = 0; i < W; ++i) {
+            if constexpr (sizeof(T) == 2) {
+                if (2 * i >= pw.cnt)
                     k.w[i] = 0u;
-                else if (2 * i + 1 >= cnt)
+                else if (2 * i + 1 >= pw.cnt)
                     k.w[i] &= 0xFFFFu;
+            } else if (i >= pw.cnt) {
+                k.w[i] = 0u;
             }
         }
-    } else {
-#pragma unroll
-        for (int i = 0; i < N; ++i)
-            k.w[i] = i < cnt ? sw[pad_word(q + i)] : 0u;
     }
 }
 
-// Tile loop shared by the padded quantisers: stage each tile's span, then
-// hand every thread its block (kPadTile threads).
-template <typename T, int G, typename Body>
-__device__ __forceinline__ void padded_tiles(const T *x, int64_t K, const FastDiv &nbp, int n_blocks,
-                                             Body &&body)
-{
-    constexpr int kPerVec = 32 / (int)sizeof(T);
-    extern __shared__ __align__(16) uint32_t sw[];
-    const int64_t n = (int64_t)nbp.div(n_blocks) * K; // whole rows in this launch
-    for (int b0 = (int)blockIdx.x * kPadTile; b0 < n_blocks; b0 += (int)gridDim.x * kPadTile) {
-        const int nb = min(kPadTile, n_blocks - b0);
-        int cnt0, cnt1;
-        const int64_t f0 = pad_block_start(b0, nbp, K, G, cnt0);
-        const int64_t f1 = pad_block_start(b0 + nb - 1, nbp, K, G, cnt1) + cnt1;
-        const int64_t base = span_base(x, f0);
-        const int nvec = (int)((f1 - base + kPerVec - 1) / kPerVec);
-        stage_span(x, n, base, nvec, sw);
-        __syncthreads();
-        if ((int)threadIdx.x < nb) {
-            const int b = b0 + (int)threadIdx.x;
-            int cnt;
-            const int64_t f = pad_block_start(b, nbp, K, G, cnt);
-            Blk<T, G> blk;
-            staged_block(sw, (int)(f - base), cnt, blk);
-            body(b, blk);
-        }
-        __syncthreads();
-    }
-}
+// Units per thread of the padded quantisers (the window of an MXFP4 block
+// is twice as long).
+template <int G> constexpr int pad_units() { return G == 16 ? 2 : 1; }
 
 template <typename T>
-__global__ void __launch_bounds__(kPadTile)
+__global__ void __launch_bounds__(kThreads)
     nvfp4_quantize_padded_kernel(const T *__restrict__ x, int64_t K, FastDiv nbp, int n_blocks,
                                  const float *amax, uint2 *__restrict__ packed,
                                  uint8_t *__restrict__ scales, float *global_scale, int32_t *status)
@@ -205,22 +196,36 @@ __global__ void __launch_bounds__(kPadTile)
     if (!nv_prologue(amax, global_scale, status, g))
         return;
     const NvScaleConsts sc = nv_scale_consts(g);
-    padded_tiles<T, 16>(x, K, nbp, n_blocks, [&](int b, const Blk<T, 16> &blk) {
-        nv_quantize_block(blk, sc, packed + b, scales + b);
-    });
+    const char *x_end = reinterpret_cast<const char *>(x + (int64_t)nbp.div(n_blocks) * K);
+    constexpr int U = pad_units<16>();
+    PadWin<T, 16> pw[U];
+    stream_units<U>(
+        n_blocks, [&](int u, int b) { pad_win_load(x, x_end, b, nbp, K, pw[u]); },
+        [&](int u, int b) {
+            Blk<T, 16> blk;
+            pad_win_block(pw[u], blk);
+            nv_quantize_block(blk, sc, packed + b, scales + b);
+        });
 }
 
 template <typename T, bool kCeil>
-__global__ void __launch_bounds__(kPadTile)
+__global__ void __launch_bounds__(kThreads)
     mxfp4_quantize_padded_kernel(const T *__restrict__ x, int64_t K, FastDiv nbp, int n_blocks,
                                  uint4 *__restrict__ packed, uint8_t *__restrict__ scales,
                                  int32_t *status)
 {
     pdl_begin();
     bool bad = false;
-    padded_tiles<T, 32>(x, K, nbp, n_blocks, [&](int b, const Blk<T, 32> &blk) {
-        mx_quantize_block<kCeil>(blk, packed + b, scales + b, bad);
-    });
+    const char *x_end = reinterpret_cast<const char *>(x + (int64_t)nbp.div(n_blocks) * K);
+    constexpr int U = pad_units<32>();
+    PadWin<T, 32> pw[U];
+    stream_units<U>(
+        n_blocks, [&](int u, int b) { pad_win_load(x, x_end, b, nbp, K, pw[u]); },
+        [&](int u, int b) {
+            Blk<T, 32> blk;
+            pad_win_block(pw[u], blk);
+            mx_quantize_block<kCeil>(blk, packed + b, scales + b, bad);
+        });
     if (bad)
         raise_status(status, kStatusNonFinite);
 }

@@ -119,8 +119,9 @@ fp4_status fp4_tensor_amax(const void *x, fp4_dtype dtype, int64_t n, float *ama
  * NONFINITE, RANGE.
  *
  * Every kernel of the library is launched with programmatic stream
- * serialisation: it may start while the previous kernel on the stream is
- * finishing and waits for it before touching memory. */
+ * serialisation: it is launched as the previous kernel on the stream retires
+ * its CTAs and waits for that kernel's memory operations before touching
+ * memory. */
 fp4_status fp4_nvfp4_quantize(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
                               uint8_t *packed, uint8_t *scales, float *global_scale,
                               void *workspace, size_t workspace_bytes, int32_t *status,
