@@ -837,13 +837,15 @@ SEARCH_OPS_PER_EVAL = 7
 
 def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict, n_cand: int | None = None,
                  gemm_mnk=None) -> dict:
+    # DRAM bytes per launch from an ncu capture (profiles/traffic.json), used
+    # only while the kernel sources are the ones it was captured from
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         with open(tpath) as f:
             t = json.load(f)
-        ent = t.get("kernels", {}).get(name)
-        if ent and ent.get("source_hash") == kernel_source_hash() and ent.get("workload") == w.name:
+        ent = t.get("workloads", {}).get(w.name, {}).get(name)
+        if ent and ent.get("source_hash") == kernel_source_hash():
             traffic = ent.get("bytes_per_launch")
     if name == "nvfp4_gemm" and gemm_mnk:
         # tensor-bound: 2 M N K flops per launch against the FP4 dense peak,
