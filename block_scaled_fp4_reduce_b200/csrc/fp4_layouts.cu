@@ -67,14 +67,12 @@ fp4_status dq_padded(const uint8_t *packed, const uint8_t *scales, const float *
                      int64_t rows, int64_t cols, TOut *y, cudaStream_t stream)
 {
     const int64_t nup = ceil_div(cols, kNv ? 16 : 32) * (kNv ? 1 : 2); // 16-code units per row
-    constexpr size_t kSmem = fp4::pad_smem_bytes<TOut>(16);
     return for_row_chunks(rows, nup, [&](int64_t r0, int64_t nr) {
         const int n = (int)(nr * nup);
-        const int grid = grid_for(fp4::dequantize_padded_kernel<kNv, TOut>, n, fp4::kPadTile, fp4::kPadTile,
-                                  kSmem);
+        const int grid = grid_for(fp4::dequantize_padded_kernel<kNv, TOut>, n, (int64_t)kThreads * 2);
         if (grid <= 0)
             return FP4_ERR_CUDA;
-        return launch_cfg(fp4::dequantize_padded_kernel<kNv, TOut>, grid, fp4::kPadTile, kSmem, stream,
+        return launch(fp4::dequantize_padded_kernel<kNv, TOut>, grid, stream,
                           reinterpret_cast<const uint2 *>(packed) + r0 * nup,
                           scales + (kNv ? r0 * nup : r0 * nup / 2), global_scale, cols,
                           fp4::fast_div_for((uint32_t)nup), n, y + r0 * cols);
@@ -101,12 +99,35 @@ template <typename T> fp4_status column_map(const T *x, int64_t rows, int64_t co
     return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
 }
 
-template <typename T, bool kNv, bool kCeil>
-fp4_status columns(const T *x, int64_t rows, int64_t cols, const float *amax, uint8_t *packed,
-                   uint8_t *scales, float *global_scale, int32_t *status, cudaStream_t stream)
+template <typename T>
+fp4_status nv_columns(const T *x, int64_t rows, int64_t cols, const float *amax, uint8_t *packed,
+                      uint8_t *scales, float *global_scale, int32_t *status, cudaStream_t stream)
 {
-    auto kernel = fp4::quantize_columns_kernel<T, kNv, kCeil>;
-    constexpr size_t kSmem = (size_t)fp4::kColStages * fp4::kColTileBytes + (kNv ? 0 : fp4::kColStageBytes);
+    const int64_t cw = cols * (int64_t)sizeof(T) / 4; // 4-byte words per row (rows are 16-byte aligned)
+    const int64_t tiles = ceil_div(rows, fp4::kNvColRows) * ceil_div(cw, 32);
+    const int64_t nbo = ceil_div(rows, 16);
+    // the widest stores every output row allows: four blocks (32 bytes) and
+    // four scale bytes at once
+    int layout = 0;
+    if ((nbo * 8) % 32 == 0 && aligned(packed, 32))
+        layout |= fp4::kColPacked32;
+    if ((nbo * 8) % 16 == 0 && aligned(packed, 16))
+        layout |= fp4::kColPacked16;
+    if (nbo % 4 == 0 && aligned(scales, 4))
+        layout |= fp4::kColScales4;
+    const int grid = grid_for(fp4::nvfp4_quantize_columns_kernel<T>, tiles, 1);
+    if (grid <= 0)
+        return FP4_ERR_CUDA;
+    return launch(fp4::nvfp4_quantize_columns_kernel<T>, grid, stream, reinterpret_cast<const uint32_t *>(x),
+                  (int)rows, (int)cw, (int)cols, amax, packed, scales, global_scale, status, layout);
+}
+
+template <typename T, bool kCeil>
+fp4_status mx_columns(const T *x, int64_t rows, int64_t cols, uint8_t *packed, uint8_t *scales, int32_t *status,
+                      cudaStream_t stream)
+{
+    auto kernel = fp4::mxfp4_quantize_columns_kernel<T, kCeil>;
+    constexpr size_t kSmem = (size_t)fp4::kColStages * fp4::kColTileBytes + fp4::kColStageBytes;
     static bool attr_set[kMaxDevices] = {false};
     int dev = 0;
     if (sm_count(dev) <= 0 || dev >= kMaxDevices)
@@ -128,12 +149,11 @@ fp4_status columns(const T *x, int64_t rows, int64_t cols, const float *amax, ui
         if (st != FP4_OK)
             return st;
     }
-    constexpr int kBlock = fp4::col_threads<kNv>();
-    const int grid = grid_for(kernel, n_tiles, 1, kBlock, kSmem);
+    const int grid = grid_for(kernel, n_tiles, 1, fp4::kMxColThreads, kSmem);
     if (grid <= 0)
         return FP4_ERR_CUDA;
-    return launch_cfg(kernel, grid, kBlock, kSmem, stream, map, (int)rows, (int)cols,
-                      (int)n_tiles, amax, packed, scales, global_scale, status);
+    return launch_cfg(kernel, grid, fp4::kMxColThreads, kSmem, stream, map, (int)rows, (int)cols, (int)n_tiles,
+                      packed, scales, status);
 }
 
 // Common checks of the quantisers here; NV also needs a workspace.
@@ -270,10 +290,10 @@ fp4_status fp4_nvfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t ro
     if (st != FP4_OK)
         return st;
     if (dtype == FP4_BF16)
-        return columns<uint16_t, true, false>(static_cast<const uint16_t *>(x), rows, cols, amax, packed,
-                                              scales, global_scale, status, stream);
-    return columns<float, true, false>(static_cast<const float *>(x), rows, cols, amax, packed, scales,
-                                       global_scale, status, stream);
+        return nv_columns(static_cast<const uint16_t *>(x), rows, cols, amax, packed, scales, global_scale,
+                          status, stream);
+    return nv_columns(static_cast<const float *>(x), rows, cols, amax, packed, scales, global_scale, status,
+                      stream);
 }
 
 fp4_status fp4_mxfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
@@ -291,12 +311,12 @@ fp4_status fp4_mxfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t ro
     const uint16_t *xb = static_cast<const uint16_t *>(x);
     const float *xf = static_cast<const float *>(x);
     if (bf && ceil)
-        return columns<uint16_t, false, true>(xb, rows, cols, nullptr, packed, scales, nullptr, status, stream);
+        return mx_columns<uint16_t, true>(xb, rows, cols, packed, scales, status, stream);
     if (bf)
-        return columns<uint16_t, false, false>(xb, rows, cols, nullptr, packed, scales, nullptr, status, stream);
+        return mx_columns<uint16_t, false>(xb, rows, cols, packed, scales, status, stream);
     if (ceil)
-        return columns<float, false, true>(xf, rows, cols, nullptr, packed, scales, nullptr, status, stream);
-    return columns<float, false, false>(xf, rows, cols, nullptr, packed, scales, nullptr, status, stream);
+        return mx_columns<float, true>(xf, rows, cols, packed, scales, status, stream);
+    return mx_columns<float, false>(xf, rows, cols, packed, scales, status, stream);
 }
 
 } // extern "C"

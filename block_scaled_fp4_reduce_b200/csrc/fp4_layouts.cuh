@@ -11,17 +11,21 @@
 //     Q(W^T) run down the columns of W [R, C]; the output is the plain
 //     row-padded layout of the [C, R] transpose, produced from W directly.
 //
-// The column-wise quantiser stages 64-row x 512-byte tiles of W in shared
-// memory with 2-D TMA loads (cp.async.bulk.tensor, no multicast), two
-// stages deep: each stage has a "full" mbarrier (the TMA bytes landed) and
-// an "empty" one (every warp released the tile), and thread 0 refills a
-// stage as soon as it is empty, so no CTA-wide barrier sits in the loop.
-// Each thread then quantises whole 16- or 32-element blocks down one (fp32)
-// or two (bf16) tile columns.  Rows past R read as zeros (TMA out-of-bounds
-// fill), which is the +0 padding.  Every mbarrier wait is bounded: a thread
-// that runs out records FP4_ERR_TIMEOUT and leaves the loop, the waits that
-// depended on it run out in turn, and thread 0 waits (bounded again) for
-// every copy it started before the CTA ends.
+// The NVFP4 column-wise quantiser reads W straight from global memory: a
+// CTA takes a tile of 256 rows x a 128-byte strip, every lane of a warp one
+// 4-byte word column of 32 rows, quantises the blocks of its columns in
+// registers and stages them in shared memory, from where the CTA stores
+// whole 128-byte output rows.  The MXFP4 one stages 64-row x 512-byte tiles
+// of W in shared memory with 2-D TMA loads (cp.async.bulk.tensor, no
+// multicast), two stages deep: each stage has a "full" mbarrier (the TMA
+// bytes landed) and an "empty" one (every warp released the tile), and
+// thread 0 refills a stage as soon as it is empty.  Each thread then
+// quantises whole 32-element blocks down one (fp32) or two (bf16) tile
+// columns.  Rows past R read as zeros (TMA out-of-bounds fill), which is the
+// +0 padding.  Every mbarrier wait is bounded: a thread that runs out
+// records FP4_ERR_TIMEOUT and leaves the loop, the waits that depended on it
+// run out in turn, and thread 0 waits (bounded again) for every copy it
+// started before the CTA ends.
 #pragma once
 
 #include <cstdint>
@@ -39,36 +43,10 @@ constexpr int32_t kStatusTimeout = 8;
 // block b % nbp of that row; it covers the elements [f, f + cnt) of the flat
 // input, f = (b / nbp) K + (b % nbp) G, cnt = min(G, K - (b % nbp) G), and
 // reads +0 past them.  The quantisers read every block from its window of
-// aligned 32-byte vectors in registers (PadWin below).  Consecutive units
-// cover consecutive flat elements, so the dequantiser's tile of kPadTile
-// units is one contiguous span of y: it assembles the span in shared memory
-// and writes its interior back with 256-bit stores.  In shared memory each
-// 32-byte vector takes 36 bytes (one pad word per eight): a unit that
-// starts 32 bytes after its neighbour's then starts in another bank, so the
-// word accesses of a warp are conflict-free.
+// aligned 32-byte vectors in registers (PadWin below); the dequantiser
+// writes whole aligned vectors of y assembled across a warp with shuffles
+// (dequantize_padded_kernel).
 // ---------------------------------------------------------------------------
-constexpr int kPadTile = 256; // 16-code units per tile of the dequantiser
-
-// Word w of the staged span lives at word w + w / 8.
-__device__ __forceinline__ int pad_word(int w) { return w + (w >> 3); }
-
-template <typename T> constexpr int pad_smem_bytes(int G)
-{
-    // span of kPadTile units of G elements, one vector of slack at each end,
-    // and room for the last unit's writes past its real elements
-    return (kPadTile * G * (int)sizeof(T) / 32 + 4) * 36;
-}
-
-// First element of the span of [f0, ...) that starts a 32-byte vector at
-// the absolute address (p: the array, element-aligned; the result may lie a
-// few elements before f0 when p itself is not 32-byte aligned).
-template <typename T> __device__ __forceinline__ int64_t span_base(const T *p, int64_t f0)
-{
-    constexpr int kPerVec = 32 / (int)sizeof(T);
-    const int64_t mis = (int64_t)((reinterpret_cast<uintptr_t>(p) / sizeof(T)) % kPerVec);
-    return f0 - (f0 + mis) % kPerVec;
-}
-
 // Division of a 31-bit unsigned n by a launch-invariant d >= 1 (the round-up
 // method of Granlund and Montgomery, "Division by invariant integers using
 // multiplication", 1994): l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1,
@@ -91,14 +69,20 @@ inline FastDiv fast_div_for(uint32_t d)
     return FastDiv{d, (uint32_t)m, l};
 }
 
-// First flat element of block b and its element count.
-__device__ __forceinline__ int64_t pad_block_start(int b, const FastDiv &nbp, int64_t K, int G, int &cnt)
+// First flat element of block b, its element count and its row.
+__device__ __forceinline__ int64_t pad_block_start(int b, const FastDiv &nbp, int64_t K, int G, int &cnt, int &r)
 {
-    const int r = nbp.div(b);
+    r = nbp.div(b);
     const int j = b - r * (int)nbp.d;
     const int64_t c0 = (int64_t)j * G;
     cnt = (int)min((int64_t)G, K - c0);
     return (int64_t)r * K + c0;
+}
+
+__device__ __forceinline__ int64_t pad_block_start(int b, const FastDiv &nbp, int64_t K, int G, int &cnt)
+{
+    int r;
+    return pad_block_start(b, nbp, K, G, cnt, r);
 }
 
 // A ragged block read straight from global memory.  Every block of a row
@@ -231,117 +215,387 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // Dequantise a row-padded layout into the logical [R, K] output.  Unit i is
-// 16 codes of the padded matrix (row i / nup, columns (i % nup) * 16 ..);
-// each thread writes its unit's logical outputs (columns below K) into the
-// staged span, then the CTA stores the span: whole 32-byte vectors with
-// 256-bit stores (the span starts on a 32-byte boundary of y), the two edge
-// vectors, shared with the neighbouring tiles, element by element.
+// 16 codes of the padded matrix (row i / nup, columns (i % nup) * 16 ..); a
+// warp takes a chunk of 32 consecutive units.  The outputs of consecutive
+// units are contiguous in y, and every unit of a row starts at the same
+// offset s within a 32-byte vector (units are 16 elements apart).  A chunk
+// whose 32 units are whole (16 logical elements each) and lie in one row is
+// written as whole aligned vectors: lane L assembles the vector(s) that
+// start s bytes before its unit from the tail of unit L-1 (moved over by a
+// shuffle) and its own head, and writes them with 256-bit stores; lane 0
+// writes its own head and lane 31 its own tail -- the parts of the chunk's
+// two edge vectors that are theirs -- with the fewest aligned stores that
+// cover them (at most one each of 2, 4, 8 and 16 bytes).  Every store is an
+// L2 write request, and requests are what this kernel runs out of: written
+// element by element, the edges took 89 against 63 us without them on
+// 8192 x 14335.  Any other chunk (a row boundary, a partial unit, the end
+// of the launch) writes each unit's logical elements one by one.  Every
+// output element is written once.
+template <int K4, int W>
+__device__ __forceinline__ void pad_join(const uint32_t (&q)[2 * W], uint32_t sh, uint32_t *out)
+{
+    // out[j] = the words of q from word W - K4 on, shifted right by sh bits
+#pragma unroll
+    for (int j = 0; j < W; ++j)
+        out[j] = __funnelshift_r(q[W - K4 + j], q[W - K4 + j + 1], sh);
+}
+
+template <typename TOut> __device__ __forceinline__ void pad_store_elem(TOut *y, int64_t e, uint32_t word, int half)
+{
+    if constexpr (sizeof(TOut) == 2)
+        y[e] = (uint16_t)(word >> (16 * half));
+    else
+        y[e] = __uint_as_float(word);
+}
+
+// Bytes [LO, HI) of the 32-byte-aligned span p, whose image is the words w,
+// in the fewest aligned stores.
+template <int LO, int HI>
+__device__ __forceinline__ void store_range(uint8_t *p, const uint32_t *w)
+{
+    if constexpr (LO < HI) {
+        constexpr int a = (LO % 32 == 0 && LO + 32 <= HI)   ? 32
+                          : (LO % 16 == 0 && LO + 16 <= HI) ? 16
+                          : (LO % 8 == 0 && LO + 8 <= HI)   ? 8
+                          : (LO % 4 == 0 && LO + 4 <= HI)   ? 4
+                                                            : 2;
+        constexpr int k = LO / 4;
+        if constexpr (a == 32)
+            stg_v8(p + LO, w + k);
+        else if constexpr (a == 16)
+            *reinterpret_cast<uint4 *>(p + LO) = make_uint4(w[k], w[k + 1], w[k + 2], w[k + 3]);
+        else if constexpr (a == 8)
+            *reinterpret_cast<uint2 *>(p + LO) = make_uint2(w[k], w[k + 1]);
+        else if constexpr (a == 4)
+            *reinterpret_cast<uint32_t *>(p + LO) = w[k];
+        else
+            *reinterpret_cast<uint16_t *>(p + LO) = (uint16_t)(w[k] >> (8 * (LO % 4)));
+        store_range<LO + a, HI>(p, w);
+    }
+}
+
+// The head [sb, span) or the tail [0, sb) of a span of 4 W bytes, for a
+// warp-uniform sb (a multiple of the element size, 0 < sb < 32).
+template <int W, bool kHead>
+__device__ __forceinline__ void store_edge(uint8_t *p, const uint32_t *w, int sb)
+{
+    constexpr int S = 4 * W;
+#define FP4_EDGE(SB)                                                                                 \
+    case SB:                                                                                         \
+        if constexpr (kHead)                                                                         \
+            store_range<SB, S>(p, w);                                                                \
+        else                                                                                         \
+            store_range<0, SB>(p, w);                                                                \
+        break;
+    switch (sb) {
+        FP4_EDGE(2) FP4_EDGE(4) FP4_EDGE(6) FP4_EDGE(8) FP4_EDGE(10) FP4_EDGE(12) FP4_EDGE(14)
+        FP4_EDGE(16) FP4_EDGE(18) FP4_EDGE(20) FP4_EDGE(22) FP4_EDGE(24) FP4_EDGE(26) FP4_EDGE(28)
+        FP4_EDGE(30)
+    default: break;
+    }
+#undef FP4_EDGE
+}
+
+constexpr int kPadDqChunks = 4; // chunks of 32 units per warp whose loads go out together
+
 template <bool kNv, typename TOut>
-__global__ void __launch_bounds__(kPadTile)
+__global__ void __launch_bounds__(kThreads)
     dequantize_padded_kernel(const uint2 *__restrict__ packed, const uint8_t *__restrict__ scales,
                              const float *__restrict__ global_scale, int64_t K, FastDiv nup,
                              int n_units, TOut *__restrict__ y)
 {
-    constexpr int kPerVec = 32 / (int)sizeof(TOut);
-    extern __shared__ __align__(16) uint32_t sw[];
-    uint16_t *sh = reinterpret_cast<uint16_t *>(sw);
+    constexpr int kE = (int)sizeof(TOut);
+    constexpr int kW = 16 * kE / 4; // output words of a unit: 8 (bf16) or 16 (fp32)
     pdl_begin();
     const float g = kNv ? __ldcg(global_scale) : 1.0f;
     const uint64_t g2 = pack2(g, g);
-    for (int i0 = (int)blockIdx.x * kPadTile; i0 < n_units; i0 += (int)gridDim.x * kPadTile) {
-        const int nu = min(kPadTile, n_units - i0);
-        int cnt0, cnt1;
-        const int64_t f0 = pad_block_start(i0, nup, K, 16, cnt0);
-        const int64_t f1 = pad_block_start(i0 + nu - 1, nup, K, 16, cnt1) + cnt1;
-        const int64_t base = span_base(y, f0);
-        const int lo = (int)(f0 - base), hi = (int)(f1 - base); // the span, relative to base
-        if ((int)threadIdx.x < nu) {
-            const int i = i0 + (int)threadIdx.x;
-            int cnt;
-            const int q = (int)(pad_block_start(i, nup, K, 16, cnt) - base);
+    const int lane = (int)(threadIdx.x & 31u);
+    const int warp_stride = (int)(gridDim.x * (blockDim.x >> 5)) * 32;
+    constexpr int U = kPadDqChunks;
+    uint2 pkv[U];
+    uint32_t sbv[U];
+    int chunk = 0;
+    for (int base = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32; base < n_units;
+         base += warp_stride, chunk = (chunk + 1) % U) {
+        // the codes and scale bytes of the next U chunks, loaded together
+        if (chunk == 0) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int iu = base + u * warp_stride + lane;
+                if (iu < n_units) {
+                    pkv[u] = __ldcg(packed + iu);
+                    sbv[u] = __ldcg(scales + (kNv ? iu : (iu >> 1)));
+                }
+            }
+        }
+        const int i = base + lane;
+        int cnt = 0;
+        int row = -1;
+        int64_t f = 0;
+        uint32_t o[kW];
+        if (i < n_units) {
+            f = pad_block_start(i, nup, K, 16, cnt, row);
+            uint2 pk = pkv[0];
+            uint32_t sbyte = sbv[0];
+#pragma unroll
+            for (int u = 1; u < U; ++u)
+                if (chunk == u) {
+                    pk = pkv[u];
+                    sbyte = sbv[u];
+                }
             float y16[16];
-            dequant_floats<kNv>(__ldcg(packed + i), __ldcg(scales + (kNv ? i : (i >> 1))), g2, y16);
-            if constexpr (sizeof(TOut) == 2) {
-                uint32_t pr[8]; // bf16 pairs (y[2k], y[2k+1]), low half first
+            dequant_floats<kNv>(pk, sbyte, g2, y16);
+            if constexpr (kE == 2) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(pr[k]) : "f"(y16[2 * k + 1]), "f"(y16[2 * k]));
-                const int w0 = q >> 1;
-                if (cnt == 16 && !(q & 1)) {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        sw[pad_word(w0 + k)] = pr[k];
-                } else if (cnt == 16) {
-                    // odd start: y[0] is the high half of word w0, y[15] the
-                    // low half of word w0 + 8 (the other halves belong to the
-                    // neighbouring units); words in between hold (y[2k-1], y[2k])
-                    sh[2 * pad_word(w0) + 1] = (uint16_t)pr[0];
-#pragma unroll
-                    for (int k = 1; k < 8; ++k)
-                        sw[pad_word(w0 + k)] = __byte_perm(pr[k - 1], pr[k], 0x5432);
-                    sh[2 * pad_word(w0 + 8)] = (uint16_t)(pr[7] >> 16);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        if (j >= cnt)
-                            break;
-                        const int e = q + j;
-                        sh[2 * pad_word(e >> 1) + (e & 1)] = (uint16_t)(pr[j >> 1] >> (16 * (j & 1)));
-                    }
-                }
+                    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[k]) : "f"(y16[2 * k + 1]), "f"(y16[2 * k]));
             } else {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    if (j >= cnt)
-                        break;
-                    sw[pad_word(q + j)] = __float_as_uint(y16[j]);
-                }
+                for (int k = 0; k < 16; ++k)
+                    o[k] = __float_as_uint(y16[k]);
             }
         }
-        __syncthreads();
-        const int nvec = (hi + kPerVec - 1) / kPerVec;
-        for (int v = (int)threadIdx.x; v < nvec; v += (int)blockDim.x) {
-            const int e = v * kPerVec;
-            if (e >= lo && e + kPerVec <= hi) {
-                uint32_t w[8];
+        const int row0 = __shfl_sync(0xFFFFFFFFu, row, 0);
+        if (__all_sync(0xFFFFFFFFu, cnt == 16 && row == row0)) {
+            const uintptr_t start = reinterpret_cast<uintptr_t>(y + f);
+            const int sb = (int)(start & 31u); // the same in every lane
+            uint8_t *vec = reinterpret_cast<uint8_t *>(start - (uintptr_t)sb);
+            if (sb == 0) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    w[k] = sw[v * 9 + k];
-                stg_v8(y + base + e, w);
-            } else {
-                for (int k = max(lo - e, 0); k < min(kPerVec, hi - e); ++k) {
-                    const int ei = e + k;
-                    if constexpr (sizeof(TOut) == 2)
-                        y[base + ei] = sh[2 * pad_word(ei >> 1) + (ei & 1)];
-                    else
-                        y[base + ei] = __uint_as_float(sw[pad_word(ei)]);
-                }
+                for (int v = 0; v < kW / 8; ++v)
+                    stg_v8(vec + 32 * v, o + 8 * v);
+                continue;
             }
+            uint32_t q[2 * kW];
+#pragma unroll
+            for (int k = 0; k < kW; ++k) {
+                q[k] = __shfl_up_sync(0xFFFFFFFFu, o[k], 1);
+                q[kW + k] = o[k];
+            }
+            uint32_t out[kW]; // the image of the span at vec (lane 0: its own bytes only)
+            const uint32_t sh = (uint32_t)((32 - sb) & 3) * 8u;
+            switch ((sb + 3) >> 2) { // words of unit L-1 in the first vector
+            case 1: pad_join<1, kW>(q, sh, out); break;
+            case 2: pad_join<2, kW>(q, sh, out); break;
+            case 3: pad_join<3, kW>(q, sh, out); break;
+            case 4: pad_join<4, kW>(q, sh, out); break;
+            case 5: pad_join<5, kW>(q, sh, out); break;
+            case 6: pad_join<6, kW>(q, sh, out); break;
+            case 7: pad_join<7, kW>(q, sh, out); break;
+            default: pad_join<8, kW>(q, sh, out); break;
+            }
+            if (lane > 0) {
+#pragma unroll
+                for (int v = 0; v < kW / 8; ++v)
+                    stg_v8(vec + 32 * v, out + 8 * v);
+            } else {
+                store_edge<kW, true>(vec, out, sb);
+            }
+            if (lane == 31) {
+                // the bytes past the span: the image of the next span holds
+                // this unit's last sb bytes first
+                uint32_t tail[kW];
+#pragma unroll
+                for (int k = 0; k < kW; ++k)
+                    q[k] = o[k];
+                switch ((sb + 3) >> 2) {
+                case 1: pad_join<1, kW>(q, sh, tail); break;
+                case 2: pad_join<2, kW>(q, sh, tail); break;
+                case 3: pad_join<3, kW>(q, sh, tail); break;
+                case 4: pad_join<4, kW>(q, sh, tail); break;
+                case 5: pad_join<5, kW>(q, sh, tail); break;
+                case 6: pad_join<6, kW>(q, sh, tail); break;
+                case 7: pad_join<7, kW>(q, sh, tail); break;
+                default: pad_join<8, kW>(q, sh, tail); break;
+                }
+                store_edge<kW, false>(vec + 4 * kW, tail, sb);
+            }
+        } else if (i < n_units) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                if (e < cnt)
+                    pad_store_elem(y, f + e, o[e * kE / 4], kE == 2 ? (e & 1) : 0);
         }
-        __syncthreads();
     }
 }
 
 // ---------------------------------------------------------------------------
-// Column-wise quantisation.  Tiles of kColTileRows rows x 512 bytes of W
-// (256 bf16 or 128 fp32 columns).  A tile row is 128 four-byte words; the
-// CTA has 128 threads per block row of the tile (64 / G block rows: 512
-// threads for NVFP4, 256 for MXFP4), and thread (j, w) quantises the
-// block(s) of block row j in word column w: one fp32 column, or the two bf16
-// columns that share the word.  NVFP4 stores its 8-byte blocks straight into
-// the output rows; MXFP4 (bound by its stores, not its instructions) stages a
-// tile's blocks in shared memory and stores each output row's 32 bytes from
-// one thread.
+// Column-wise NVFP4, straight from global memory, results staged in shared
+// memory.  A CTA takes a tile of 256 rows x one 128-byte strip of W (64
+// bf16 or 32 fp32 columns); warp k quantises rows [32k, 32k + 32) of it:
+// each lane loads its 4-byte word of 16 rows at a time (one coalesced
+// 128-byte row segment per warp load), assembles the 16-row block of each
+// of its columns in registers and quantises it.  The blocks go to a staging
+// tile in shared memory, one 128-byte row per output row (column of W), and
+// after a barrier the CTA stores every output row's 128 bytes of codes and
+// 16 scale bytes with 32-byte and 4-byte stores.  Every global store is an
+// L2 write request: storing each lane's blocks straight into its two output
+// rows took four requests per 32 rows and column, against 2 / 64 here, and
+// the stores, not the loads or the arithmetic, bounded that kernel.  Staging
+// is double-buffered, so one barrier per tile suffices: a warp that reaches
+// the next-but-one tile has passed the barrier that every warp reaches only
+// after storing this tile.  Rows past R read as +0 (the padding); blocks past
+// the padded column length are not stored.
+// ---------------------------------------------------------------------------
+constexpr int kNvColRows = 256;               // rows of W per tile: 8 warps x 32 rows
+constexpr int kNvColBlocks = kNvColRows / 16; // blocks per output row per tile
+constexpr int kNvColCtasPerSm = 4;
+static_assert(kNvColRows == 32 * (kThreads / 32), "one warp per 32 rows of a tile");
+static_assert(kNvColBlocks * 8 == 128, "a tile's output row is 128 bytes of codes");
+
+// Store layout flags of the column-wise NVFP4 outputs (host computed).
+constexpr int kColPacked32 = 1; // every output row's packed bytes start 32-byte aligned
+constexpr int kColPacked16 = 2; // ... 16-byte aligned
+constexpr int kColScales4 = 4;  // every output row's scale bytes start 4-byte aligned
+
+// Staging-tile position (8-byte chunk) of block j of tile column cl: chunk j
+// of the column's 128-byte row, XOR-swizzled so that the 16 lanes of a
+// half-warp storing one block each of 16 different columns hit all 32 banks
+// once, and the 8 rows x 4 quarter rows read by a warp in the store phase
+// hit every bank exactly twice (the minimum for 256 bytes).
+template <int kPerWord> __device__ __forceinline__ int col_swizzle(int cl)
+{
+    return kPerWord == 2 ? (((cl >> 1) ^ ((cl & 1) << 3)) & 15) : (cl & 15);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, kNvColCtasPerSm)
+    nvfp4_quantize_columns_kernel(const uint32_t *__restrict__ xw, int R, int Cw, int C,
+                                  const float *amax, uint8_t *__restrict__ packed,
+                                  uint8_t *__restrict__ scales, float *global_scale, int32_t *status,
+                                  int layout)
+{
+    constexpr int kPerWord = 4 / (int)sizeof(T); // columns per word
+    constexpr int kTileCols = 32 * kPerWord;     // columns of W (output rows) per tile
+    constexpr int kScaleRow = 20;                // staged scale bytes per output row (16 + 4 of padding)
+    __shared__ __align__(16) uint8_t st_packed[2][kTileCols * 128];
+    __shared__ __align__(16) uint8_t st_scales[2][kTileCols * kScaleRow];
+    pdl_begin();
+    float g;
+    if (!nv_prologue(amax, global_scale, status, g))
+        return;
+    const NvScaleConsts sc = nv_scale_consts(g);
+    const int lane = (int)(threadIdx.x & 31u), warp = (int)(threadIdx.x >> 5);
+    const int n_strips = (Cw + 31) / 32;
+    const int n_tiles = ((R + kNvColRows - 1) / kNvColRows) * n_strips;
+    const int nbo = (R + 15) / 16;         // blocks (scale bytes) per output row
+    const int64_t prow = (int64_t)nbo * 8; // packed bytes per output row
+    int s = 0;
+    for (int tile = (int)blockIdx.x; tile < n_tiles; tile += (int)gridDim.x, s ^= 1) {
+        const int band = tile / n_strips;
+        const int strip = tile - band * n_strips;
+        const int w = strip * 32 + lane;                     // word column of W
+        const int r0 = band * kNvColRows + warp * 32;      // this warp's first row
+        if (w < Cw && r0 < R) {
+            uint32_t sb2[kPerWord]; // the two scale bytes of each column
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int rh = r0 + 16 * h;
+                uint32_t v[16];
+                const uint32_t *src = xw + (int64_t)rh * Cw + w;
+                if (rh + 16 <= R) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i, src += Cw)
+                        v[i] = __ldcg(src);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i, src += Cw)
+                        v[i] = rh + i < R ? __ldcg(src) : 0u;
+                }
+#pragma unroll
+                for (int p = 0; p < kPerWord; ++p) {
+                    Blk<T, 16> b;
+                    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            b.w[i] = __byte_perm(v[2 * i], v[2 * i + 1], p ? 0x7632 : 0x5410);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            b.w[i] = v[i];
+                    }
+                    uint2 q;
+                    uint8_t sbyte;
+                    nv_quantize_block(b, sc, &q, &sbyte);
+                    const int cl = lane * kPerWord + p;
+                    const int chunk = (2 * warp + h) ^ col_swizzle<kPerWord>(cl);
+                    *reinterpret_cast<uint2 *>(&st_packed[s][cl * 128 + 8 * chunk]) = q;
+                    sb2[p] = h ? sb2[p] | ((uint32_t)sbyte << 8) : (uint32_t)sbyte;
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < kPerWord; ++p) {
+                const int cl = lane * kPerWord + p;
+                *reinterpret_cast<uint16_t *>(&st_scales[s][cl * kScaleRow + 2 * warp]) = (uint16_t)sb2[p];
+            }
+        }
+        __syncthreads();
+        // store phase: four threads per output row, a quarter row each
+        const int b0 = band * kNvColBlocks;     // first block of the tile in an output row
+        const int nbt = min(kNvColBlocks, nbo - b0); // blocks of the tile inside the padded length
+        for (int t = (int)threadIdx.x; t < kTileCols * 4; t += kThreads) {
+            const int cl = t >> 2, qr = t & 3;
+            const int c = strip * kTileCols + cl;
+            if (c >= C || 4 * qr >= nbt)
+                continue;
+            const int f = col_swizzle<kPerWord>(cl);
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint2 q = *reinterpret_cast<const uint2 *>(&st_packed[s][cl * 128 + 8 * ((4 * qr + i) ^ f)]);
+                o[2 * i] = q.x;
+                o[2 * i + 1] = q.y;
+            }
+            const int nq = min(4, nbt - 4 * qr); // blocks of this quarter row inside the padded length
+            uint8_t *orow = packed + (int64_t)c * prow + (int64_t)(b0 + 4 * qr) * 8;
+            if (nq == 4 && (layout & kColPacked32)) {
+                stg_v8(orow, o);
+            } else if (layout & kColPacked16) {
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    if (2 * k + 2 <= nq)
+                        reinterpret_cast<uint4 *>(orow)[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+                    else if (2 * k < nq)
+                        reinterpret_cast<uint2 *>(orow)[2 * k] = make_uint2(o[4 * k], o[4 * k + 1]);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (k < nq)
+                        reinterpret_cast<uint2 *>(orow)[k] = make_uint2(o[2 * k], o[2 * k + 1]);
+            }
+            const uint32_t sw = *reinterpret_cast<const uint32_t *>(&st_scales[s][cl * kScaleRow + 4 * qr]);
+            uint8_t *srow = scales + (int64_t)c * nbo + b0 + 4 * qr;
+            if (nq == 4 && (layout & kColScales4)) {
+                *reinterpret_cast<uint32_t *>(srow) = sw;
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (k < nq)
+                        srow[k] = (uint8_t)(sw >> (8 * k));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Column-wise MXFP4.  Tiles of kColTileRows rows x 512 bytes of W (256 bf16
+// or 128 fp32 columns) arrive by TMA.  A tile row is 128 four-byte words;
+// the CTA has 128 threads per 32-row block row of the tile (256 threads),
+// and thread (j, w) quantises the block(s) of block row j in word column w:
+// one fp32 column, or the two bf16 columns that share the word.  The blocks
+// go to a staging tile in shared memory, and each output row's 32 bytes are
+// stored by one thread.
 // ---------------------------------------------------------------------------
 constexpr int kColWords = 128;
 constexpr int kColTileRows = 64;
 constexpr int kColTileBytes = kColTileRows * 512;
 constexpr int kColStages = 2;
 // Staging of one tile's results: packed codes (32 bytes per tile column:
-// 4 NVFP4 or 2 MXFP4 blocks) and scale bytes, for up to 256 columns.
+// two MXFP4 blocks) and scale bytes, for up to 256 columns.
 constexpr int kColStagePacked = 256 * 32;
 constexpr int kColStageBytes = kColStagePacked + 256 * 4;
-template <bool kNv> constexpr int col_threads() { return kColWords * (kColTileRows / (kNv ? 16 : 32)); }
+constexpr int kMxColThreads = kColWords * (kColTileRows / 32);
 constexpr uint32_t kWaitTries = 1u << 22;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -407,54 +661,14 @@ __device__ __forceinline__ ColTile col_tile(int t, int n_tc, int tile_cols)
 }
 
 // Quantises the G-element blocks of the tile rows [j*G, j*G + G) in this
-// thread's columns and stores them straight into the output rows (= columns
-// of W): the NVFP4 pass, which is bound by its instruction issue, not by
-// these partial-sector stores.
-template <typename T, bool kNv, bool kCeil, int G>
-__device__ __forceinline__ void column_blocks_direct(const uint8_t *tile, int j, int w, int c_first, int C,
-                                              int blk, const NvScaleConsts &sc, uint8_t *packed,
-                                              uint8_t *scales, int64_t prow, int nbo, bool &bad)
-{
-    constexpr int kPerThread = 4 / (int)sizeof(T); // columns per word: 2 (bf16) or 1 (fp32)
-    const uint32_t *tw = reinterpret_cast<const uint32_t *>(tile) + j * G * kColWords + w;
-    uint32_t rowv[G]; // row i of this thread's word column
-#pragma unroll
-    for (int i = 0; i < G; ++i)
-        rowv[i] = tw[i * kColWords];
-#pragma unroll
-    for (int p = 0; p < kPerThread; ++p) {
-        const int c = c_first + p;
-        if (c >= C)
-            continue;
-        Blk<T, G> b;
-        if constexpr (sizeof(T) == 2) {
-            // bf16: a word holds columns 2t (low half) and 2t+1 (high half);
-            // gather one column's halves of rows 2i, 2i+1 into word i.
-#pragma unroll
-            for (int i = 0; i < G / 2; ++i)
-                b.w[i] = __byte_perm(rowv[2 * i], rowv[2 * i + 1], p ? 0x7632 : 0x5410);
-        } else {
-#pragma unroll
-            for (int i = 0; i < G; ++i)
-                b.w[i] = rowv[i];
-        }
-        uint8_t *orow = packed + (int64_t)c * prow;
-        if constexpr (kNv)
-            nv_quantize_block(b, sc, reinterpret_cast<uint2 *>(orow) + blk, scales + (int64_t)c * nbo + blk);
-        else
-            mx_quantize_block<kCeil>(b, reinterpret_cast<uint4 *>(orow) + blk,
-                                     scales + (int64_t)c * nbo + blk, bad);
-    }
-}
-
-// Quantises the G-element blocks of the tile rows [j*G, j*G + G) in this
 // thread's columns into the staging tile: packed codes of block row j and
 // tile column c at stage_p + (j * kCols + c) * G/2, its scale byte at
 // stage_s[j * kCols + c] (block-row-major: a warp's writes are consecutive).
-template <typename T, bool kNv, bool kCeil, int G>
-__device__ __forceinline__ void column_blocks(const uint8_t *tile, int j, int w, const NvScaleConsts &sc,
-                                              uint8_t *stage_p, uint8_t *stage_s, bool &bad)
+template <typename T, bool kCeil>
+__device__ __forceinline__ void column_blocks(const uint8_t *tile, int j, int w, uint8_t *stage_p,
+                                              uint8_t *stage_s, bool &bad)
 {
+    constexpr int G = 32;
     constexpr int kPerThread = 4 / (int)sizeof(T); // columns per word: 2 (bf16) or 1 (fp32)
     constexpr int kCols = kColWords * kPerThread;
     const uint32_t *tw = reinterpret_cast<const uint32_t *>(tile) + j * G * kColWords + w;
@@ -479,10 +693,7 @@ __device__ __forceinline__ void column_blocks(const uint8_t *tile, int j, int w,
         }
         uint8_t *dp = stage_p + (j * kCols + c) * (G / 2);
         uint8_t *ds = stage_s + j * kCols + c;
-        if constexpr (kNv)
-            nv_quantize_block(b, sc, reinterpret_cast<uint2 *>(dp), ds);
-        else
-            mx_quantize_block<kCeil>(b, reinterpret_cast<uint4 *>(dp), ds, bad);
+        mx_quantize_block<kCeil>(b, reinterpret_cast<uint4 *>(dp), ds, bad);
     }
 }
 
@@ -522,27 +733,19 @@ __device__ __forceinline__ void column_store(const uint8_t *stage_p, const uint8
             srow[j] = stage_s[j * kCols + c];
 }
 
-template <typename T, bool kNv, bool kCeil>
-__global__ void __launch_bounds__(col_threads<kNv>())
-    quantize_columns_kernel(const __grid_constant__ CUtensorMap map, int R, int C, int n_tiles,
-                            const float *amax, uint8_t *__restrict__ packed,
-                            uint8_t *__restrict__ scales, float *global_scale, int32_t *status)
+template <typename T, bool kCeil>
+__global__ void __launch_bounds__(kMxColThreads)
+    mxfp4_quantize_columns_kernel(const __grid_constant__ CUtensorMap map, int R, int C, int n_tiles,
+                                  uint8_t *__restrict__ packed, uint8_t *__restrict__ scales, int32_t *status)
 {
-    constexpr int G = kNv ? 16 : 32;
+    constexpr int G = 32;
     constexpr int kCols = 512 / (int)sizeof(T);          // tile columns
-    constexpr int kPerWord = 4 / (int)sizeof(T);         // columns per 4-byte word
-    constexpr int kWarps = col_threads<kNv>() / 32;
+    constexpr int kWarps = kMxColThreads / 32;
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ __align__(8) uint64_t full[kColStages];  // tile landed (TMA bytes)
     __shared__ __align__(8) uint64_t empty[kColStages]; // every warp is done with the tile
 
     pdl_begin();
-    float g = 1.0f;
-    if constexpr (kNv) {
-        if (!nv_prologue(amax, global_scale, status, g))
-            return;
-    }
-    const NvScaleConsts sc = nv_scale_consts(g);
     const int n_tc = (C + kCols - 1) / kCols;
     const int Rp = (R + G - 1) / G * G;                  // padded column length
     const int64_t prow = Rp / 2;                         // packed bytes per output row
@@ -575,90 +778,52 @@ __global__ void __launch_bounds__(col_threads<kNv>())
     }
     bool bad = false, timed_out = false;
     int k = 0;
-    if constexpr (kNv) {
-        // Each warp waits for its tiles on full[s], releases them on empty[s];
-        // thread 0 refills a stage once every warp has released it.  All waits
-        // are bounded; a thread that gives up leaves the loop, and every wait
-        // that depended on it then runs out in turn.
-        for (int t = first_tile; t < n_tiles; t += stride, ++k) {
-            const int s = k % kColStages;
-            const uint32_t phase = (uint32_t)(k / kColStages) & 1u;
-            if (!mbar_wait(&full[s], phase)) {
-                timed_out = true;
-                break;
-            }
-            const ColTile ct = col_tile(t, n_tc, kCols);
-            const int blk_row = ct.r0 + jb * G;
-            if (blk_row < R)
-                column_blocks_direct<T, kNv, kCeil, G>(smem + s * kColTileBytes, jb, w, ct.c0 + w * kPerWord,
-                                                       C, blk_row / G, sc, packed, scales, prow, nbo, bad);
-            __syncwarp();
-            if ((threadIdx.x & 31) == 0)
-                mbar_arrive(&empty[s]);
-            if (producer) {
-                const int tn = t + kColStages * stride;
-                if (tn < n_tiles) {
-                    if (!mbar_wait(&empty[s], phase)) {
-                        timed_out = true;
-                        break;
-                    }
+    // Per tile every thread waits (bounded) for the tile on full[s], and the
+    // CTA votes: if any wait ran out, all threads leave the loop together
+    // (the barriers below must be reached by all or none).  The threads
+    // quantise their blocks into the staging tile, release the TMA stage
+    // (each warp on empty[s]), and after a barrier thread c < kCols stores
+    // tile column c's blocks: 32 contiguous bytes of one output row instead
+    // of 16 bytes from each of two warps.  Thread 0 refills the stage once
+    // every warp has released it; a refill wait that runs out goes into the
+    // next vote.
+    uint8_t *stage_p = smem + kColStages * kColTileBytes;
+    uint8_t *stage_s = stage_p + kColStagePacked;
+    const bool wide = (reinterpret_cast<uintptr_t>(packed) % 32u) == 0 && prow % 32 == 0;
+    for (int t = first_tile; t < n_tiles; t += stride, ++k) {
+        const int s = k % kColStages;
+        const uint32_t phase = (uint32_t)(k / kColStages) & 1u;
+        const bool ok = !timed_out && mbar_wait(&full[s], phase);
+        if (__syncthreads_or(!ok)) {
+            timed_out = true;
+            break;
+        }
+        const ColTile ct = col_tile(t, n_tc, kCols);
+        if (ct.r0 + jb * G < R)
+            column_blocks<T, kCeil>(smem + s * kColTileBytes, jb, w, stage_p, stage_s, bad);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0)
+            mbar_arrive(&empty[s]);
+        __syncthreads(); // staging tile complete
+        const int c = (int)threadIdx.x;
+        const int blk0 = ct.r0 / G;
+        if (c < kCols && ct.c0 + c < C) {
+            const int n_valid = nbo - blk0 < kColTileRows / G ? nbo - blk0 : kColTileRows / G;
+            const int64_t oc = ct.c0 + c;
+            column_store<G, kCols>(stage_p, stage_s, c, packed + oc * prow + (int64_t)blk0 * (G / 2),
+                                   scales + oc * nbo + blk0, n_valid, wide);
+        }
+        if (producer) {
+            const int tn = t + kColStages * stride;
+            if (tn < n_tiles) {
+                if (!mbar_wait(&empty[s], phase)) {
+                    timed_out = true; // the next vote ends the loop for everyone
+                } else {
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     const ColTile cn = col_tile(tn, n_tc, kCols);
                     mbar_expect_tx(&full[s], kColTileBytes);
                     tma_load_2d(smem + s * kColTileBytes, &map, cn.c0, cn.r0, &full[s]);
                     ++issued;
-                }
-            }
-        }
-    } else {
-        // MXFP4, bound by its stores: per tile every thread waits (bounded)
-        // for the tile on full[s], and the CTA votes: if any wait ran out,
-        // all threads leave the loop together (the barriers below must be
-        // reached by all or none).  The threads quantise their blocks into
-        // the staging tile, release the TMA stage (each warp on empty[s]),
-        // and after a barrier thread c < kCols stores tile column c's
-        // blocks: 32 contiguous bytes of one output row instead of 16 bytes
-        // from each of two warps.  Thread 0 refills the stage once every warp
-        // has released it; a refill wait that runs out goes into the next
-        // vote.
-        uint8_t *stage_p = smem + kColStages * kColTileBytes;
-        uint8_t *stage_s = stage_p + kColStagePacked;
-        const bool wide = (reinterpret_cast<uintptr_t>(packed) % 32u) == 0 && prow % 32 == 0;
-        for (int t = first_tile; t < n_tiles; t += stride, ++k) {
-            const int s = k % kColStages;
-            const uint32_t phase = (uint32_t)(k / kColStages) & 1u;
-            const bool ok = !timed_out && mbar_wait(&full[s], phase);
-            if (__syncthreads_or(!ok)) {
-                timed_out = true;
-                break;
-            }
-            const ColTile ct = col_tile(t, n_tc, kCols);
-            if (ct.r0 + jb * G < R)
-                column_blocks<T, kNv, kCeil, G>(smem + s * kColTileBytes, jb, w, sc, stage_p, stage_s, bad);
-            __syncwarp();
-            if ((threadIdx.x & 31) == 0)
-                mbar_arrive(&empty[s]);
-            __syncthreads(); // staging tile complete
-            const int c = (int)threadIdx.x;
-            const int blk0 = ct.r0 / G;
-            if (c < kCols && ct.c0 + c < C) {
-                const int n_valid = nbo - blk0 < kColTileRows / G ? nbo - blk0 : kColTileRows / G;
-                const int64_t oc = ct.c0 + c;
-                column_store<G, kCols>(stage_p, stage_s, c, packed + oc * prow + (int64_t)blk0 * (G / 2),
-                                       scales + oc * nbo + blk0, n_valid, wide);
-            }
-            if (producer) {
-                const int tn = t + kColStages * stride;
-                if (tn < n_tiles) {
-                    if (!mbar_wait(&empty[s], phase)) {
-                        timed_out = true; // the next vote ends the loop for everyone
-                    } else {
-                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                        const ColTile cn = col_tile(tn, n_tc, kCols);
-                        mbar_expect_tx(&full[s], kColTileBytes);
-                        tma_load_2d(smem + s * kColTileBytes, &map, cn.c0, cn.r0, &full[s]);
-                        ++issued;
-                    }
                 }
             }
         }
