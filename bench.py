@@ -404,10 +404,11 @@ class LayoutPath:
     "variants" = amax, NVFP4 four over six (it runs its own amax: two
     launches), MXFP4 with the ceil scale rule, dequantisation of both to
     bf16; "columns" = amax,
-    column-wise NVFP4 quantise (Q(W^T), g from the amax), column-wise MXFP4
+    column-wise NVFP4 quantise (Q(W^T), g from that amax), column-wise MXFP4
     quantise, dequantisation of both padded layouts of the [K, R] transpose
-    to bf16; "padded" = amax, NVFP4 and MXFP4 quantise of rows padded to
-    whole blocks, dequantisation of both back to the logical [R, K] bf16."""
+    to bf16; "padded" = amax, NVFP4 (from that amax) and MXFP4 quantise of
+    rows padded to whole blocks, dequantisation of both back to the logical
+    [R, K] bf16."""
     OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize"]
     LAUNCHES = 5
 
@@ -446,9 +447,11 @@ class LayoutPath:
                                                            None, P(self.ws), ws_bytes, P(self.status), st))
             mx_call = (L.fp4_mxfp4_quantize_ceil, (P(x), dt, R, K, P(self.mx_p), P(self.mx_s), P(self.status), st))
         else:
-            nvq = L.fp4_nvfp4_quantize_columns if kind == "columns" else L.fp4_nvfp4_quantize_padded
+            # the NV call takes the step's amax (one amax pass per step, as on the row path)
+            nvq = (L.fp4_nvfp4_quantize_columns_with_amax if kind == "columns"
+                   else L.fp4_nvfp4_quantize_padded_with_amax)
             mxq = L.fp4_mxfp4_quantize_columns if kind == "columns" else L.fp4_mxfp4_quantize_padded
-            nv_call = (nvq, (P(x), dt, R, K, P(self.nv_p), P(self.nv_s), P(self.nv_g), P(self.ws), ws_bytes,
+            nv_call = (nvq, (P(x), dt, R, K, P(self.amax), P(self.nv_p), P(self.nv_s), P(self.nv_g),
                              P(self.status), st))
             mx_call = (mxq, (P(x), dt, R, K, fp4.MX_FLOOR, P(self.mx_p), P(self.mx_s), P(self.status), st))
         self.calls = [

@@ -80,9 +80,11 @@ def lib() -> ctypes.CDLL:
             "fp4_nvfp4_gemm": (I, [P, P, P, P, P, P, I64, I64, I64, P, P, P]),
             "fp4_nvfp4_gemm_ex": (I, [P, P, P, P, P, P, I64, I64, I64, P, I, P, P]),
             "fp4_nvfp4_quantize_padded": (I, [P, I, I64, I64, P, P, P, P, SZ, P, P]),
+            "fp4_nvfp4_quantize_padded_with_amax": (I, [P, I, I64, I64, P, P, P, P, P, P]),
             "fp4_mxfp4_quantize_padded": (I, [P, I, I64, I64, I, P, P, P, P]),
             "fp4_dequantize_padded": (I, [I, P, P, P, I64, I64, P, I, P]),
             "fp4_nvfp4_quantize_columns": (I, [P, I, I64, I64, P, P, P, P, SZ, P, P]),
+            "fp4_nvfp4_quantize_columns_with_amax": (I, [P, I, I64, I64, P, P, P, P, P, P]),
             "fp4_mxfp4_quantize_columns": (I, [P, I, I64, I64, I, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
@@ -393,17 +395,24 @@ def _padded(n: int, group: int) -> int:
     return -(-n // group) * group
 
 
-def nvfp4_quantize_padded(x: torch.Tensor, workspace=None, status=None, stream=None) -> Quantized:
+def nvfp4_quantize_padded(x: torch.Tensor, workspace=None, status=None, stream=None, amax=None) -> Quantized:
     """NVFP4 of x [R, K] for any K: rows padded with +0 to whole 16-blocks
-    (packed [R, ceil(K/16)*8], scales [R, ceil(K/16)])."""
+    (packed [R, ceil(K/16)*8], scales [R, ceil(K/16)]).  With `amax` (a
+    device float32 holding the tensor amax) the call skips its own amax
+    pass (fp4_nvfp4_quantize_padded_with_amax)."""
     R, K = _shape2(x)
     dev = x.device
     Kp = _padded(K, 16)
     packed = torch.empty((R, Kp // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty((R, Kp // 16), dtype=torch.uint8, device=dev)
     g = torch.empty(1, dtype=torch.float32, device=dev)
-    ws = workspace if workspace is not None else workspace_for(x)
     st = status if status is not None else new_status(dev)
+    if amax is not None:
+        _check(lib().fp4_nvfp4_quantize_padded_with_amax(_p(x), _dtype_code(x), R, K, _p(amax), _p(packed),
+                                                         _p(scales), _p(g), _p(st), _stream(stream)),
+               "fp4_nvfp4_quantize_padded_with_amax")
+        return Quantized(NVFP4, packed, scales, g, st, R, K)
+    ws = workspace if workspace is not None else workspace_for(x)
     _check(lib().fp4_nvfp4_quantize_padded(_p(x), _dtype_code(x), R, K, _p(packed), _p(scales), _p(g), _p(ws),
                                            ws.numel() * ws.element_size(), _p(st), _stream(stream)),
            "fp4_nvfp4_quantize_padded")
@@ -431,17 +440,24 @@ def dequantize_padded(q: Quantized, out_dtype=torch.bfloat16, out=None, stream=N
     return y
 
 
-def nvfp4_quantize_columns(x: torch.Tensor, workspace=None, status=None, stream=None) -> Quantized:
+def nvfp4_quantize_columns(x: torch.Tensor, workspace=None, status=None, stream=None, amax=None) -> Quantized:
     """NVFP4 of W^T for x = W [R, C]: blocks down the columns of W; the
-    result describes the logical [C, R] transpose in the padded layout."""
+    result describes the logical [C, R] transpose in the padded layout.
+    With `amax` (device float32, the amax of W) the call skips its own amax
+    pass (fp4_nvfp4_quantize_columns_with_amax)."""
     R, C = _shape2(x)
     dev = x.device
     Rp = _padded(R, 16)
     packed = torch.empty((C, Rp // 2), dtype=torch.uint8, device=dev)
     scales = torch.empty((C, Rp // 16), dtype=torch.uint8, device=dev)
     g = torch.empty(1, dtype=torch.float32, device=dev)
-    ws = workspace if workspace is not None else workspace_for(x)
     st = status if status is not None else new_status(dev)
+    if amax is not None:
+        _check(lib().fp4_nvfp4_quantize_columns_with_amax(_p(x), _dtype_code(x), R, C, _p(amax), _p(packed),
+                                                          _p(scales), _p(g), _p(st), _stream(stream)),
+               "fp4_nvfp4_quantize_columns_with_amax")
+        return Quantized(NVFP4, packed, scales, g, st, C, R)
+    ws = workspace if workspace is not None else workspace_for(x)
     _check(lib().fp4_nvfp4_quantize_columns(_p(x), _dtype_code(x), R, C, _p(packed), _p(scales), _p(g), _p(ws),
                                             ws.numel() * ws.element_size(), _p(st), _stream(stream)),
            "fp4_nvfp4_quantize_columns")

@@ -194,6 +194,27 @@ fp4_status check_columns(fp4_dtype dtype, int64_t rows, int64_t cols)
 
 extern "C" {
 
+fp4_status fp4_nvfp4_quantize_padded_with_amax(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                               const float *amax, uint8_t *packed, uint8_t *scales,
+                                               float *global_scale, int32_t *status, cudaStream_t stream)
+{
+    fp4_status st = check_quant(x, dtype, rows, cols, packed, scales, status);
+    if (st != FP4_OK)
+        return st;
+    if (!global_scale || !amax)
+        return FP4_ERR_INVALID_ARG;
+    if (!aligned(amax, 4))
+        return FP4_ERR_ALIGN;
+    if (cols % 16 == 0)
+        return fp4_nvfp4_quantize_with_amax(x, dtype, rows, cols, amax, packed, scales, global_scale, status,
+                                            stream);
+    if (dtype == FP4_BF16)
+        return nv_padded(static_cast<const uint16_t *>(x), rows, cols, amax, packed, scales,
+                         global_scale, status, stream);
+    return nv_padded(static_cast<const float *>(x), rows, cols, amax, packed, scales, global_scale,
+                     status, stream);
+}
+
 fp4_status fp4_nvfp4_quantize_padded(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
                                      uint8_t *packed, uint8_t *scales, float *global_scale,
                                      void *workspace, size_t workspace_bytes, int32_t *status,
@@ -206,18 +227,12 @@ fp4_status fp4_nvfp4_quantize_padded(const void *x, fp4_dtype dtype, int64_t row
         return FP4_ERR_INVALID_ARG;
     if ((st = check_ws(workspace, workspace_bytes)) != FP4_OK)
         return st;
-    if (cols % 16 == 0)
-        return fp4_nvfp4_quantize(x, dtype, rows, cols, packed, scales, global_scale, workspace,
-                                  workspace_bytes, status, stream);
     float *amax = reinterpret_cast<float *>(static_cast<uint32_t *>(workspace) + kWsAmax);
     st = fp4_tensor_amax(x, dtype, rows * cols, amax, workspace, workspace_bytes, status, stream);
     if (st != FP4_OK)
         return st;
-    if (dtype == FP4_BF16)
-        return nv_padded(static_cast<const uint16_t *>(x), rows, cols, amax, packed, scales,
-                         global_scale, status, stream);
-    return nv_padded(static_cast<const float *>(x), rows, cols, amax, packed, scales, global_scale,
-                     status, stream);
+    return fp4_nvfp4_quantize_padded_with_amax(x, dtype, rows, cols, amax, packed, scales, global_scale, status,
+                                               stream);
 }
 
 fp4_status fp4_mxfp4_quantize_padded(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
@@ -271,6 +286,26 @@ fp4_status fp4_dequantize_padded(fp4_format fmt, const uint8_t *packed, const ui
     return dq_padded<false>(packed, scales, global_scale, rows, cols, static_cast<float *>(y), stream);
 }
 
+fp4_status fp4_nvfp4_quantize_columns_with_amax(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                                const float *amax, uint8_t *packed, uint8_t *scales,
+                                                float *global_scale, int32_t *status, cudaStream_t stream)
+{
+    fp4_status st = check_quant(x, dtype, rows, cols, packed, scales, status);
+    if (st != FP4_OK)
+        return st;
+    if (!global_scale || !amax)
+        return FP4_ERR_INVALID_ARG;
+    if ((st = check_columns(dtype, rows, cols)) != FP4_OK)
+        return st;
+    if (!aligned(amax, 4))
+        return FP4_ERR_ALIGN;
+    if (dtype == FP4_BF16)
+        return nv_columns(static_cast<const uint16_t *>(x), rows, cols, amax, packed, scales, global_scale,
+                          status, stream);
+    return nv_columns(static_cast<const float *>(x), rows, cols, amax, packed, scales, global_scale, status,
+                      stream);
+}
+
 fp4_status fp4_nvfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
                                       uint8_t *packed, uint8_t *scales, float *global_scale,
                                       void *workspace, size_t workspace_bytes, int32_t *status,
@@ -289,11 +324,8 @@ fp4_status fp4_nvfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t ro
     st = fp4_tensor_amax(x, dtype, rows * cols, amax, workspace, workspace_bytes, status, stream);
     if (st != FP4_OK)
         return st;
-    if (dtype == FP4_BF16)
-        return nv_columns(static_cast<const uint16_t *>(x), rows, cols, amax, packed, scales, global_scale,
-                          status, stream);
-    return nv_columns(static_cast<const float *>(x), rows, cols, amax, packed, scales, global_scale, status,
-                      stream);
+    return fp4_nvfp4_quantize_columns_with_amax(x, dtype, rows, cols, amax, packed, scales, global_scale, status,
+                                                stream);
 }
 
 fp4_status fp4_mxfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,

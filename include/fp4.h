@@ -263,6 +263,15 @@ fp4_status fp4_nvfp4_quantize_padded(const void *x, fp4_dtype dtype, int64_t row
                                      void *workspace, size_t workspace_bytes, int32_t *status,
                                      cudaStream_t stream);
 
+/* fp4_nvfp4_quantize_padded given the tensor amax already in device memory
+ * (e.g. from fp4_tensor_amax, or a max all-reduce of per-rank amaxes), as
+ * fp4_nvfp4_quantize_with_amax is to fp4_nvfp4_quantize: A = *amax (4-byte
+ * aligned), one kernel, no workspace.  Outputs and data errors as
+ * fp4_nvfp4_quantize_padded. */
+fp4_status fp4_nvfp4_quantize_padded_with_amax(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                               const float *amax, uint8_t *packed, uint8_t *scales,
+                                               float *global_scale, int32_t *status, cudaStream_t stream);
+
 /* MXFP4 quantise + pack of x [rows, cols], any cols >= 0, padded layout,
  * with scale rule `rule`.  Errors as fp4_mxfp4_quantize. */
 fp4_status fp4_mxfp4_quantize_padded(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
@@ -283,6 +292,13 @@ fp4_status fp4_nvfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t ro
                                       uint8_t *packed, uint8_t *scales, float *global_scale,
                                       void *workspace, size_t workspace_bytes, int32_t *status,
                                       cudaStream_t stream);
+
+/* fp4_nvfp4_quantize_columns given the amax of W already in device memory
+ * (4-byte aligned): one kernel, no workspace.  Outputs and data errors as
+ * fp4_nvfp4_quantize_columns. */
+fp4_status fp4_nvfp4_quantize_columns_with_amax(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
+                                                const float *amax, uint8_t *packed, uint8_t *scales,
+                                                float *global_scale, int32_t *status, cudaStream_t stream);
 
 /* MXFP4 quantise + pack of W^T for x = W [rows, cols], padded layout of the
  * transpose, scale rule `rule`.  Data errors NONFINITE, TIMEOUT. */

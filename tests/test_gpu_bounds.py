@@ -166,15 +166,18 @@ def test_padded_and_column_layouts(shape, dtype, launch_limit):
     pad = lambda n, gsz: -(-n // gsz) * gsz  # noqa: E731
     refs = {"nv": fp4.nvfp4_quantize_padded(x), "mx": fp4.mxfp4_quantize_padded(x, fp4.MX_FLOOR)}
     columns = (K * (2 if dtype == torch.bfloat16 else 4)) % 16 == 0  # a TMA row pitch of whole 16 bytes
+    refs["nva"] = refs["nv"]  # the same outputs from the _with_amax call
     if columns:
         refs["nvc"] = fp4.nvfp4_quantize_columns(x)
         refs["mxc"] = fp4.mxfp4_quantize_columns(x, fp4.MX_CEIL)
+        refs["nvca"] = refs["nvc"]
+    amax, _ = fp4.tensor_amax(x)
     st = new_status()
     for fill in FILLS:
         ws = Guarded((ws_bytes(),), torch.uint8, fill)
         ws.t.zero_()
         for key, ref in refs.items():
-            OR, OC = (K, R) if key.endswith("c") else (R, K)
+            OR, OC = (K, R) if key in ("nvc", "mxc", "nvca") else (R, K)
             G = 16 if key.startswith("nv") else 32
             p = Guarded((OR, pad(OC, G) // 2), torch.uint8, fill)
             s = Guarded((OR, pad(OC, G) // G), torch.uint8, fill)
@@ -185,6 +188,12 @@ def test_padded_and_column_layouts(shape, dtype, launch_limit):
             elif key == "mx":
                 rc = L.fp4_mxfp4_quantize_padded(x.data_ptr(), dt, R, K, fp4.MX_FLOOR, p.ptr, s.ptr,
                                                  st.data_ptr(), stream())
+            elif key == "nva":
+                rc = L.fp4_nvfp4_quantize_padded_with_amax(x.data_ptr(), dt, R, K, amax.data_ptr(), p.ptr, s.ptr,
+                                                           g.ptr, st.data_ptr(), stream())
+            elif key == "nvca":
+                rc = L.fp4_nvfp4_quantize_columns_with_amax(x.data_ptr(), dt, R, K, amax.data_ptr(), p.ptr, s.ptr,
+                                                            g.ptr, st.data_ptr(), stream())
             elif key == "nvc":
                 rc = L.fp4_nvfp4_quantize_columns(x.data_ptr(), dt, R, K, p.ptr, s.ptr, g.ptr, ws.ptr, ws.n,
                                                   st.data_ptr(), stream())

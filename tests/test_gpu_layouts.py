@@ -180,3 +180,64 @@ def test_columns_full_size_weight_sampled_columns():
     p, s = oracle.mxfp4_quantize(sub)
     assert_same(mx.packed[cols], p, "MX columns packed (sampled)")
     assert_same(mx.scales[cols], s, "MX columns scales (sampled)")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_with_amax_entry_points(dtype):
+    """The _with_amax calls are the plain ones minus their amax pass: byte
+    for byte the same outputs for the tensor's own amax, and, for a larger
+    amax handed in (a max over shards), the oracle's quantisation at
+    g = fl32(A / 2688) of that amax."""
+    for R, K in ((5, 33), (129, 4099), (4, 64)):
+        x = rand(R, K, dtype, seed=R + 11 * K)
+        xd = x.to(DEV)
+        a, _ = fp4.tensor_amax(xd)
+        q0 = fp4.nvfp4_quantize_padded(xd)
+        q1 = fp4.nvfp4_quantize_padded(xd, amax=a)
+        big = torch.full((1,), 4.0 * a.item(), dtype=torch.float32, device=DEV)
+        q2 = fp4.nvfp4_quantize_padded(xd, amax=big)
+        torch.cuda.synchronize()
+        for q in (q0, q1, q2):
+            q.check()
+        assert torch.equal(q0.packed, q1.packed) and torch.equal(q0.scales, q1.scales)
+        assert q0.global_scale.item() == q1.global_scale.item()
+        g = oracle.nv_global_scale(big.item())
+        assert q2.global_scale.item() == g
+        p, s = oracle.nvfp4_quantize_with_g(oracle.pad_rows(odata(x), 16), g)
+        assert_same(q2.packed, p, f"NV padded with amax {R}x{K}")
+        assert_same(q2.scales, s, f"NV padded scales with amax {R}x{K}")
+    for R, C in ((100, 264), (300, 1032), (20, 8)):
+        x = rand(R, C, dtype, seed=R + 13 * C)
+        xd = x.to(DEV)
+        a, _ = fp4.tensor_amax(xd)
+        q0 = fp4.nvfp4_quantize_columns(xd)
+        q1 = fp4.nvfp4_quantize_columns(xd, amax=a)
+        big = torch.full((1,), 3.0 * a.item(), dtype=torch.float32, device=DEV)
+        q2 = fp4.nvfp4_quantize_columns(xd, amax=big)
+        torch.cuda.synchronize()
+        for q in (q0, q1, q2):
+            q.check()
+        assert torch.equal(q0.packed, q1.packed) and torch.equal(q0.scales, q1.scales)
+        assert q0.global_scale.item() == q1.global_scale.item()
+        g = oracle.nv_global_scale(big.item())
+        assert q2.global_scale.item() == g
+        p, s = oracle.nvfp4_quantize_with_g(oracle.pad_rows(oracle.transpose(odata(x)), 16), g)
+        assert_same(q2.packed, p, f"NV columns with amax {R}x{C}")
+        assert_same(q2.scales, s, f"NV columns scales with amax {R}x{C}")
+
+
+def test_with_amax_argument_errors():
+    L = fp4.lib()
+    x = torch.randn(8, 40, device=DEV)
+    pk = torch.empty(8 * 24, dtype=torch.uint8, device=DEV)
+    sc = torch.empty(8 * 3, dtype=torch.uint8, device=DEV)
+    g = torch.empty(1, dtype=torch.float32, device=DEV)
+    st = fp4.new_status(DEV)
+    a = torch.zeros(2, dtype=torch.float32, device=DEV)
+    ab = a.view(torch.uint8)
+    P = lambda t: t.data_ptr()  # noqa: E731
+    for fn in (L.fp4_nvfp4_quantize_padded_with_amax, L.fp4_nvfp4_quantize_columns_with_amax):
+        assert fn(P(x), fp4.F32, 8, 40, None, P(pk), P(sc), P(g), P(st), None) == fp4.ERR_INVALID_ARG
+        assert fn(P(x), fp4.F32, 8, 40, P(ab[1:]), P(pk), P(sc), P(g), P(st), None) == fp4.ERR_ALIGN
+        assert fn(P(x), fp4.F32, 8, 40, P(a), P(pk), P(sc), None, P(st), None) == fp4.ERR_INVALID_ARG
+    torch.cuda.synchronize()
