@@ -1,10 +1,9 @@
 // fp4_layouts.cu -- entry points of include/fp4.h for ragged rows (padded
-// to whole blocks) and column-wise grouping.  Argument checks, the TMA
-// tensor map of the column-wise pass, and the launches.
+// to whole blocks) and column-wise grouping: argument checks, store-layout
+// flags and the launches.
 #include <climits>
 #include <cstdint>
 
-#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "fp4.h"
@@ -81,29 +80,11 @@ fp4_status dq_padded(const uint8_t *packed, const uint8_t *scales, const float *
 
 // ----------------------------------------------------------- column-wise --
 
-// Tensor map of W [rows, cols] (innermost: cols), box 512 bytes x 64 rows,
-// no swizzle, zero fill out of bounds.
-template <typename T> fp4_status column_map(const T *x, int64_t rows, int64_t cols, CUtensorMap *map)
-{
-    EncodeTiled enc = encode_tiled();
-    if (!enc)
-        return FP4_ERR_CUDA;
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)cols * sizeof(T)};
-    const cuuint32_t box[2] = {512u / (cuuint32_t)sizeof(T), (cuuint32_t)fp4::kColTileRows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(map, sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                           2, const_cast<T *>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
-}
-
 template <typename T>
 fp4_status nv_columns(const T *x, int64_t rows, int64_t cols, const float *amax, uint8_t *packed,
                       uint8_t *scales, float *global_scale, int32_t *status, cudaStream_t stream)
 {
-    const int64_t cw = cols * (int64_t)sizeof(T) / 4; // 4-byte words per row (rows are 16-byte aligned)
+    const int64_t cw = cols * (int64_t)sizeof(T) / 4; // 4-byte words per row (rows are 4-byte aligned)
     const int64_t tiles = ceil_div(rows, fp4::kNvColRows) * ceil_div(cw, 32);
     const int64_t nbo = ceil_div(rows, 16);
     // the widest stores every output row allows: four blocks (32 bytes) and
@@ -126,34 +107,22 @@ template <typename T, bool kCeil>
 fp4_status mx_columns(const T *x, int64_t rows, int64_t cols, uint8_t *packed, uint8_t *scales, int32_t *status,
                       cudaStream_t stream)
 {
+    const int64_t cw = cols * (int64_t)sizeof(T) / 4; // 4-byte words per row (rows are 4-byte aligned)
+    const int64_t tiles = ceil_div(rows, fp4::kMxColRows) * ceil_div(cw, 32);
+    const int64_t nbo = ceil_div(rows, 32);
+    // the widest stores every output row allows: two blocks (32 bytes) and
+    // four scale bytes at once
+    int layout = 0;
+    if ((nbo * 16) % 32 == 0 && aligned(packed, 32))
+        layout |= fp4::kColPacked32;
+    if (nbo % 4 == 0 && aligned(scales, 4))
+        layout |= fp4::kColScales4;
     auto kernel = fp4::mxfp4_quantize_columns_kernel<T, kCeil>;
-    constexpr size_t kSmem = (size_t)fp4::kColStages * fp4::kColTileBytes + fp4::kColStageBytes;
-    static bool attr_set[kMaxDevices] = {false};
-    int dev = 0;
-    if (sm_count(dev) <= 0 || dev >= kMaxDevices)
-        return FP4_ERR_CUDA;
-    if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem) !=
-            cudaSuccess) {
-            (void)cudaGetLastError();
-            return FP4_ERR_CUDA;
-        }
-        attr_set[dev] = true;
-    }
-    CUtensorMap map;
-    memset(&map, 0, sizeof(map));
-    const int64_t tile_cols = 512 / (int64_t)sizeof(T);
-    const int64_t n_tiles = (rows > 0 && cols > 0) ? ceil_div(rows, fp4::kColTileRows) * ceil_div(cols, tile_cols) : 0;
-    if (n_tiles > 0) {
-        const fp4_status st = column_map(x, rows, cols, &map);
-        if (st != FP4_OK)
-            return st;
-    }
-    const int grid = grid_for(kernel, n_tiles, 1, fp4::kMxColThreads, kSmem);
+    const int grid = grid_for(kernel, tiles, 1);
     if (grid <= 0)
         return FP4_ERR_CUDA;
-    return launch_cfg(kernel, grid, fp4::kMxColThreads, kSmem, stream, map, (int)rows, (int)cols, (int)n_tiles,
-                      packed, scales, status);
+    return launch(kernel, grid, stream, reinterpret_cast<const uint32_t *>(x), (int)rows, (int)cw, (int)cols,
+                  packed, scales, status, layout);
 }
 
 // Common checks of the quantisers here; NV also needs a workspace.
@@ -185,7 +154,7 @@ fp4_status check_columns(fp4_dtype dtype, int64_t rows, int64_t cols)
 {
     if (rows > INT_MAX || cols > INT_MAX)
         return FP4_ERR_SHAPE;
-    if ((cols * (dtype == FP4_BF16 ? 2 : 4)) % 16)
+    if ((cols * (dtype == FP4_BF16 ? 2 : 4)) % 4) // the kernels read rows as 4-byte words
         return FP4_ERR_ALIGN;
     return FP4_OK;
 }

@@ -11,32 +11,20 @@
 //     Q(W^T) run down the columns of W [R, C]; the output is the plain
 //     row-padded layout of the [C, R] transpose, produced from W directly.
 //
-// The NVFP4 column-wise quantiser reads W straight from global memory: a
-// CTA takes a tile of 256 rows x a 128-byte strip, every lane of a warp one
-// 4-byte word column of 32 rows, quantises the blocks of its columns in
-// registers and stages them in shared memory, from where the CTA stores
-// whole 128-byte output rows.  The MXFP4 one stages 64-row x 512-byte tiles
-// of W in shared memory with 2-D TMA loads (cp.async.bulk.tensor, no
-// multicast), two stages deep: each stage has a "full" mbarrier (the TMA
-// bytes landed) and an "empty" one (every warp released the tile), and
-// thread 0 refills a stage as soon as it is empty.  Each thread then
-// quantises whole 32-element blocks down one (fp32) or two (bf16) tile
-// columns.  Rows past R read as zeros (TMA out-of-bounds fill), which is the
-// +0 padding.  Every mbarrier wait is bounded: a thread that runs out
-// records FP4_ERR_TIMEOUT and leaves the loop, the waits that depended on it
-// run out in turn, and thread 0 waits (bounded again) for every copy it
-// started before the CTA ends.
+// The column-wise quantisers read W straight from global memory: a CTA
+// takes a tile of 256 rows x a 128-byte strip, every lane of a warp one
+// 4-byte word column of 32 rows (one coalesced 128-byte row segment per warp
+// load), quantises the blocks of its columns in registers and stages them in
+// shared memory, from where the CTA stores whole output rows with wide
+// stores.  Rows past R read as +0, which is the padding.  No kernel here
+// waits on another thread beyond __syncthreads.
 #pragma once
 
 #include <cstdint>
 
-#include <cuda.h>
-
 #include "fp4_kernels.cuh"
 
 namespace fp4 {
-
-constexpr int32_t kStatusTimeout = 8;
 
 // ---------------------------------------------------------------------------
 // Ragged rows.  Block b of the row-padded [R, Kp] matrix is row b / nbp,
@@ -579,262 +567,122 @@ __global__ void __launch_bounds__(kThreads, kNvColCtasPerSm)
 }
 
 // ---------------------------------------------------------------------------
-// Column-wise MXFP4.  Tiles of kColTileRows rows x 512 bytes of W (256 bf16
-// or 128 fp32 columns) arrive by TMA.  A tile row is 128 four-byte words;
-// the CTA has 128 threads per 32-row block row of the tile (256 threads),
-// and thread (j, w) quantises the block(s) of block row j in word column w:
-// one fp32 column, or the two bf16 columns that share the word.  The blocks
-// go to a staging tile in shared memory, and each output row's 32 bytes are
-// stored by one thread.
+// Column-wise MXFP4, the same way: a CTA takes a tile of 256 rows x one
+// 128-byte strip of W, warp k rows [32k, 32k + 32) -- one 32-row block per
+// column -- each lane its 4-byte word of all 32 rows (32 coalesced row
+// segments per warp in flight).  The blocks are staged in shared memory, 16
+// bytes each, 8 per output row, 16-byte chunks XOR-swizzled (chunk k of
+// column c at k ^ ((c >> 1) & 7) ^ (c & 1)) so that the eight lanes of a
+// quarter-warp writing one block each, and the eight threads of a quarter-warp
+// reading two rows' quarters in the store phase, hit eight different chunks;
+// after one barrier per tile the CTA stores each output row's 128 bytes with
+// 32-byte stores and its 8 scale bytes with 4-byte stores.  Rows past R read
+// as +0; blocks past the padded column length are not stored.
 // ---------------------------------------------------------------------------
-constexpr int kColWords = 128;
-constexpr int kColTileRows = 64;
-constexpr int kColTileBytes = kColTileRows * 512;
-constexpr int kColStages = 2;
-// Staging of one tile's results: packed codes (32 bytes per tile column:
-// two MXFP4 blocks) and scale bytes, for up to 256 columns.
-constexpr int kColStagePacked = 256 * 32;
-constexpr int kColStageBytes = kColStagePacked + 256 * 4;
-constexpr int kMxColThreads = kColWords * (kColTileRows / 32);
-constexpr uint32_t kWaitTries = 1u << 22;
+constexpr int kMxColRows = 256;                 // rows of W per tile: 8 warps x 32 rows
+constexpr int kMxColBlocks = kMxColRows / 32;   // blocks per output row per tile
+constexpr int kMxColCtasPerSm = 3;
+static_assert(kMxColRows == 32 * (kThreads / 32), "one warp per 32 rows of a tile");
 
-__device__ __forceinline__ uint32_t smem_addr(const void *p)
+template <int kPerWord> __device__ __forceinline__ int mx_col_swizzle(int cl)
 {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-                 : "memory");
-}
-
-// Bounded wait for phase `parity` of the barrier; false when the tries run out.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
-{
-    for (uint32_t t = 0; t < kWaitTries; ++t) {
-        uint32_t done;
-        asm volatile("{\n\t"
-                     ".reg .pred p;\n\t"
-                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                     "selp.u32 %0, 1, 0, p;\n\t"
-                     "}"
-                     : "=r"(done)
-                     : "r"(smem_addr(bar)), "r"(parity)
-                     : "memory");
-        if (done)
-            return true;
-    }
-    return false;
-}
-
-// 2-D TMA tile load of box (x = column, y = row) into shared memory,
-// completing on `bar`.  x is a multiple of 512 bytes' worth of elements.
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
-{
-    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-                 " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
-                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
-                 : "memory");
-}
-
-// Tile t of the column-wise pass: column tile t % n_tc, row tile t / n_tc
-// (consecutive CTAs sweep across the columns of one row band together).
-struct ColTile {
-    int r0, c0;
-};
-
-__device__ __forceinline__ ColTile col_tile(int t, int n_tc, int tile_cols)
-{
-    const int tr = t / n_tc;
-    return {tr * kColTileRows, (t - tr * n_tc) * tile_cols};
-}
-
-// Quantises the G-element blocks of the tile rows [j*G, j*G + G) in this
-// thread's columns into the staging tile: packed codes of block row j and
-// tile column c at stage_p + (j * kCols + c) * G/2, its scale byte at
-// stage_s[j * kCols + c] (block-row-major: a warp's writes are consecutive).
-template <typename T, bool kCeil>
-__device__ __forceinline__ void column_blocks(const uint8_t *tile, int j, int w, uint8_t *stage_p,
-                                              uint8_t *stage_s, bool &bad)
-{
-    constexpr int G = 32;
-    constexpr int kPerThread = 4 / (int)sizeof(T); // columns per word: 2 (bf16) or 1 (fp32)
-    constexpr int kCols = kColWords * kPerThread;
-    const uint32_t *tw = reinterpret_cast<const uint32_t *>(tile) + j * G * kColWords + w;
-    uint32_t rowv[G]; // row i of this thread's word column
-#pragma unroll
-    for (int i = 0; i < G; ++i)
-        rowv[i] = tw[i * kColWords];
-#pragma unroll
-    for (int p = 0; p < kPerThread; ++p) {
-        const int c = w * kPerThread + p; // tile column
-        Blk<T, G> b;
-        if constexpr (sizeof(T) == 2) {
-            // bf16: a word holds columns 2t (low half) and 2t+1 (high half);
-            // gather one column's halves of rows 2i, 2i+1 into word i.
-#pragma unroll
-            for (int i = 0; i < G / 2; ++i)
-                b.w[i] = __byte_perm(rowv[2 * i], rowv[2 * i + 1], p ? 0x7632 : 0x5410);
-        } else {
-#pragma unroll
-            for (int i = 0; i < G; ++i)
-                b.w[i] = rowv[i];
-        }
-        uint8_t *dp = stage_p + (j * kCols + c) * (G / 2);
-        uint8_t *ds = stage_s + j * kCols + c;
-        mx_quantize_block<kCeil>(b, reinterpret_cast<uint4 *>(dp), ds, bad);
-    }
-}
-
-// Stores tile column c's staged blocks: kBR blocks of G/2 bytes (32 bytes)
-// contiguous in output row c, and their kBR scale bytes; only the n_valid
-// first ones when the column is cut by the padded length.  wide: the row's
-// 32 bytes start on a 32-byte boundary.
-template <int G, int kCols>
-__device__ __forceinline__ void column_store(const uint8_t *stage_p, const uint8_t *stage_s, int c,
-                                             uint8_t *orow, uint8_t *srow, int n_valid, bool wide)
-{
-    constexpr int kBR = kColTileRows / G; // block rows per tile: 4 (NVFP4) or 2 (MXFP4)
-    constexpr int kBytes = G / 2;         // packed bytes per block: 8 or 16
-    uint32_t wds[8];
-#pragma unroll
-    for (int j = 0; j < kBR; ++j) {
-        const uint32_t *src = reinterpret_cast<const uint32_t *>(stage_p + (j * kCols + c) * kBytes);
-#pragma unroll
-        for (int i = 0; i < kBytes / 4; ++i)
-            wds[j * (kBytes / 4) + i] = src[i];
-    }
-    if (n_valid == kBR && wide) {
-        stg_v8(orow, wds);
-    } else {
-#pragma unroll
-        for (int j = 0; j < kBR; ++j)
-            if (j < n_valid) {
-#pragma unroll
-                for (int i = 0; i < kBytes / 8; ++i)
-                    *reinterpret_cast<uint2 *>(orow + j * kBytes + 8 * i) =
-                        make_uint2(wds[j * (kBytes / 4) + 2 * i], wds[j * (kBytes / 4) + 2 * i + 1]);
-            }
-    }
-#pragma unroll
-    for (int j = 0; j < kBR; ++j)
-        if (j < n_valid)
-            srow[j] = stage_s[j * kCols + c];
+    return kPerWord == 2 ? (((cl >> 1) & 7) ^ (cl & 1)) : (cl & 7);
 }
 
 template <typename T, bool kCeil>
-__global__ void __launch_bounds__(kMxColThreads)
-    mxfp4_quantize_columns_kernel(const __grid_constant__ CUtensorMap map, int R, int C, int n_tiles,
-                                  uint8_t *__restrict__ packed, uint8_t *__restrict__ scales, int32_t *status)
+__global__ void __launch_bounds__(kThreads, kMxColCtasPerSm)
+    mxfp4_quantize_columns_kernel(const uint32_t *__restrict__ xw, int R, int Cw, int C,
+                                         uint8_t *__restrict__ packed, uint8_t *__restrict__ scales,
+                                         int32_t *status, int layout)
 {
-    constexpr int G = 32;
-    constexpr int kCols = 512 / (int)sizeof(T);          // tile columns
-    constexpr int kWarps = kMxColThreads / 32;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ __align__(8) uint64_t full[kColStages];  // tile landed (TMA bytes)
-    __shared__ __align__(8) uint64_t empty[kColStages]; // every warp is done with the tile
-
+    constexpr int kPerWord = 4 / (int)sizeof(T); // columns per word
+    constexpr int kTileCols = 32 * kPerWord;     // columns of W (output rows) per tile
+    __shared__ __align__(16) uint8_t st_packed[2][kTileCols * 128];
+    __shared__ __align__(16) uint8_t st_scales[2][kTileCols * 8];
     pdl_begin();
-    const int n_tc = (C + kCols - 1) / kCols;
-    const int Rp = (R + G - 1) / G * G;                  // padded column length
-    const int64_t prow = Rp / 2;                         // packed bytes per output row
-    const int nbo = Rp / G;                              // blocks (scale bytes) per output row
-    const int first_tile = blockIdx.x;
-    const int stride = gridDim.x;
-    const int w = (int)threadIdx.x % kColWords;          // word column of the tile
-    const int jb = (int)threadIdx.x / kColWords;         // block row of the tile
-    const bool producer = threadIdx.x == 0;
-
-    if (producer) {
-        for (int s = 0; s < kColStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kWarps);
-        }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-    int issued = 0; // tiles of this CTA whose copy thread 0 has started
-    if (producer) {
-        for (int s = 0; s < kColStages; ++s) {
-            const int t = first_tile + s * stride;
-            if (t < n_tiles) {
-                const ColTile ct = col_tile(t, n_tc, kCols);
-                mbar_expect_tx(&full[s], kColTileBytes);
-                tma_load_2d(smem + s * kColTileBytes, &map, ct.c0, ct.r0, &full[s]);
-                ++issued;
+    const int lane = (int)(threadIdx.x & 31u), warp = (int)(threadIdx.x >> 5);
+    const int n_strips = (Cw + 31) / 32;
+    const int n_tiles = ((R + kMxColRows - 1) / kMxColRows) * n_strips;
+    const int nbo = (R + 31) / 32;          // blocks (scale bytes) per output row
+    const int64_t prow = (int64_t)nbo * 16; // packed bytes per output row
+    bool bad = false;
+    int s = 0;
+    for (int tile = (int)blockIdx.x; tile < n_tiles; tile += (int)gridDim.x, s ^= 1) {
+        const int band = tile / n_strips;
+        const int strip = tile - band * n_strips;
+        const int w = strip * 32 + lane;                 // word column of W
+        const int r0 = band * kMxColRows + warp * 32;    // this warp's first row
+        if (w < Cw && r0 < R) {
+            uint32_t v[32];
+            const uint32_t *src = xw + (int64_t)r0 * Cw + w;
+            if (r0 + 32 <= R) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i, src += Cw)
+                    v[i] = __ldcg(src);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i, src += Cw)
+                    v[i] = r0 + i < R ? __ldcg(src) : 0u;
+            }
+#pragma unroll
+            for (int p = 0; p < kPerWord; ++p) {
+                Blk<T, 32> b;
+                if constexpr (sizeof(T) == 2) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        b.w[i] = __byte_perm(v[2 * i], v[2 * i + 1], p ? 0x7632 : 0x5410);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        b.w[i] = v[i];
+                }
+                uint4 q;
+                uint8_t sbyte;
+                mx_quantize_block<kCeil>(b, &q, &sbyte, bad);
+                const int cl = lane * kPerWord + p;
+                const int chunk = warp ^ mx_col_swizzle<kPerWord>(cl);
+                *reinterpret_cast<uint4 *>(&st_packed[s][cl * 128 + 16 * chunk]) = q;
+                st_scales[s][cl * 8 + warp] = sbyte;
             }
         }
-    }
-    bool bad = false, timed_out = false;
-    int k = 0;
-    // Per tile every thread waits (bounded) for the tile on full[s], and the
-    // CTA votes: if any wait ran out, all threads leave the loop together
-    // (the barriers below must be reached by all or none).  The threads
-    // quantise their blocks into the staging tile, release the TMA stage
-    // (each warp on empty[s]), and after a barrier thread c < kCols stores
-    // tile column c's blocks: 32 contiguous bytes of one output row instead
-    // of 16 bytes from each of two warps.  Thread 0 refills the stage once
-    // every warp has released it; a refill wait that runs out goes into the
-    // next vote.
-    uint8_t *stage_p = smem + kColStages * kColTileBytes;
-    uint8_t *stage_s = stage_p + kColStagePacked;
-    const bool wide = (reinterpret_cast<uintptr_t>(packed) % 32u) == 0 && prow % 32 == 0;
-    for (int t = first_tile; t < n_tiles; t += stride, ++k) {
-        const int s = k % kColStages;
-        const uint32_t phase = (uint32_t)(k / kColStages) & 1u;
-        const bool ok = !timed_out && mbar_wait(&full[s], phase);
-        if (__syncthreads_or(!ok)) {
-            timed_out = true;
-            break;
-        }
-        const ColTile ct = col_tile(t, n_tc, kCols);
-        if (ct.r0 + jb * G < R)
-            column_blocks<T, kCeil>(smem + s * kColTileBytes, jb, w, stage_p, stage_s, bad);
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0)
-            mbar_arrive(&empty[s]);
-        __syncthreads(); // staging tile complete
-        const int c = (int)threadIdx.x;
-        const int blk0 = ct.r0 / G;
-        if (c < kCols && ct.c0 + c < C) {
-            const int n_valid = nbo - blk0 < kColTileRows / G ? nbo - blk0 : kColTileRows / G;
-            const int64_t oc = ct.c0 + c;
-            column_store<G, kCols>(stage_p, stage_s, c, packed + oc * prow + (int64_t)blk0 * (G / 2),
-                                   scales + oc * nbo + blk0, n_valid, wide);
-        }
-        if (producer) {
-            const int tn = t + kColStages * stride;
-            if (tn < n_tiles) {
-                if (!mbar_wait(&empty[s], phase)) {
-                    timed_out = true; // the next vote ends the loop for everyone
-                } else {
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    const ColTile cn = col_tile(tn, n_tc, kCols);
-                    mbar_expect_tx(&full[s], kColTileBytes);
-                    tma_load_2d(smem + s * kColTileBytes, &map, cn.c0, cn.r0, &full[s]);
-                    ++issued;
+        __syncthreads();
+        // store phase: four threads per output row, a quarter row (two blocks) each
+        const int b0 = band * kMxColBlocks;             // first block of the tile in an output row
+        const int nbt = min(kMxColBlocks, nbo - b0);    // blocks of the tile inside the padded length
+        for (int t = (int)threadIdx.x; t < kTileCols * 4; t += kThreads) {
+            const int cl = t >> 2, qr = t & 3;
+            const int c = strip * kTileCols + cl;
+            const int nq = min(2, nbt - 2 * qr); // blocks of this quarter row inside the padded length
+            if (c >= C || nq <= 0)
+                continue;
+            const int f = mx_col_swizzle<kPerWord>(cl);
+            const uint4 q0 = *reinterpret_cast<const uint4 *>(&st_packed[s][cl * 128 + 16 * ((2 * qr) ^ f)]);
+            const uint4 q1 = *reinterpret_cast<const uint4 *>(&st_packed[s][cl * 128 + 16 * ((2 * qr + 1) ^ f)]);
+            uint8_t *orow = packed + (int64_t)c * prow + (int64_t)(b0 + 2 * qr) * 16;
+            if (nq == 2 && (layout & kColPacked32)) {
+                const uint32_t o[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                stg_v8(orow, o);
+            } else {
+                reinterpret_cast<uint4 *>(orow)[0] = q0;
+                if (nq == 2)
+                    reinterpret_cast<uint4 *>(orow)[1] = q1;
+            }
+            if (qr < 2) { // scale bytes 4 qr .. 4 qr + 3 of the row
+                const int ns = min(4, nbt - 4 * qr);
+                if (ns > 0) {
+                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(&st_scales[s][cl * 8 + 4 * qr]);
+                    uint8_t *srow = scales + (int64_t)c * nbo + b0 + 4 * qr;
+                    if (ns == 4 && (layout & kColScales4)) {
+                        *reinterpret_cast<uint32_t *>(srow) = sw;
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (j < ns)
+                                srow[j] = (uint8_t)(sw >> (8 * j));
+                    }
                 }
             }
         }
-    }
-    if (timed_out)
-        raise_status(status, kStatusTimeout);
-    if (producer) {
-        // Before the CTA can end, every copy thread 0 started must have
-        // landed: wait (bounded) for those not consumed above.
-        for (int j = k; j < issued; ++j)
-            (void)mbar_wait(&full[j % kColStages], (uint32_t)(j / kColStages) & 1u);
     }
     if (bad)
         raise_status(status, kStatusNonFinite);

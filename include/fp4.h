@@ -250,10 +250,10 @@ fp4_status fp4_nvfp4_quantize_noalloc(const void *x, fp4_dtype dtype, int64_t ro
  * x [rows, cols], without materialising it: the outputs are the padded
  * layout of W^T (packed [cols, ceil(rows/G)*G/2], scales [cols,
  * ceil(rows/G)]); decode them with fp4_dequantize_padded(rows = cols of x,
- * cols = rows of x).  x is read through a TMA tensor map: rows, cols below
- * 2^31 (else FP4_ERR_SHAPE) and a row pitch (cols * element size) that is a
- * multiple of 16 bytes (else FP4_ERR_ALIGN).  A copy that never completes
- * ends the kernel with FP4_ERR_TIMEOUT in *status instead of a hang.
+ * cols = rows of x).  x is read in 4-byte words down its columns: rows,
+ * cols below 2^31 (else FP4_ERR_SHAPE) and a row pitch (cols * element
+ * size) that is a multiple of 4 bytes, i.e. an even cols for bf16 (else
+ * FP4_ERR_ALIGN).
  * ------------------------------------------------------------------------ */
 
 /* NVFP4 quantise + pack of x [rows, cols], any cols >= 0, padded layout.
@@ -287,7 +287,7 @@ fp4_status fp4_dequantize_padded(fp4_format fmt, const uint8_t *packed, const ui
 
 /* NVFP4 quantise + pack of W^T for x = W [rows, cols] (column-wise blocks),
  * padded layout of the [cols, rows] transpose; g from the amax of W.
- * Workspace as fp4_nvfp4_quantize.  Data errors NONFINITE, RANGE, TIMEOUT. */
+ * Workspace as fp4_nvfp4_quantize.  Data errors NONFINITE, RANGE. */
 fp4_status fp4_nvfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
                                       uint8_t *packed, uint8_t *scales, float *global_scale,
                                       void *workspace, size_t workspace_bytes, int32_t *status,
@@ -301,7 +301,7 @@ fp4_status fp4_nvfp4_quantize_columns_with_amax(const void *x, fp4_dtype dtype, 
                                                 float *global_scale, int32_t *status, cudaStream_t stream);
 
 /* MXFP4 quantise + pack of W^T for x = W [rows, cols], padded layout of the
- * transpose, scale rule `rule`.  Data errors NONFINITE, TIMEOUT. */
+ * transpose, scale rule `rule`.  Data error NONFINITE. */
 fp4_status fp4_mxfp4_quantize_columns(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols,
                                       fp4_mx_rule rule, uint8_t *packed, uint8_t *scales,
                                       int32_t *status, cudaStream_t stream);

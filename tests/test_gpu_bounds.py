@@ -165,7 +165,7 @@ def test_padded_and_column_layouts(shape, dtype, launch_limit):
     dt = fp4._dtype_code(x)
     pad = lambda n, gsz: -(-n // gsz) * gsz  # noqa: E731
     refs = {"nv": fp4.nvfp4_quantize_padded(x), "mx": fp4.mxfp4_quantize_padded(x, fp4.MX_FLOOR)}
-    columns = (K * (2 if dtype == torch.bfloat16 else 4)) % 16 == 0  # a TMA row pitch of whole 16 bytes
+    columns = (K * (2 if dtype == torch.bfloat16 else 4)) % 4 == 0  # rows of whole 4-byte words
     refs["nva"] = refs["nv"]  # the same outputs from the _with_amax call
     if columns:
         refs["nvc"] = fp4.nvfp4_quantize_columns(x)

@@ -106,13 +106,13 @@ def check_columns(x):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("shape", [(16, 8), (20, 8), (64, 256), (100, 264), (129, 520), (300, 1032), (65, 4),
-                                   (256, 520), (192, 264)])
+                                   (256, 520), (192, 264), (33, 6), (70, 98), (257, 130), (31, 1), (40, 3)])
 def test_columns_parity(dtype, shape):
     R, C = shape
-    if dtype == torch.bfloat16 and C % 8:
-        # a bf16 row pitch that is not a multiple of 16 bytes cannot be
-        # described to the TMA unit: the documented answer is FP4_ERR_ALIGN,
-        # returned before anything is queued
+    if dtype == torch.bfloat16 and C % 2:
+        # an odd bf16 row is not a whole number of the 4-byte words the
+        # kernels read: the documented answer is FP4_ERR_ALIGN, returned
+        # before anything is queued
         xd = rand(R, C, dtype, seed=R * 5 + C).to(DEV)
         for call in (fp4.nvfp4_quantize_columns, fp4.mxfp4_quantize_columns):
             with pytest.raises(fp4.FP4Error) as e:
@@ -139,7 +139,7 @@ def test_columns_transpose_counterexample_of_the_page():
 
 
 def test_columns_argument_errors():
-    x = torch.randn(16, 12, device=DEV).bfloat16()  # 24-byte pitch
+    x = torch.randn(16, 13, device=DEV).bfloat16()  # 26-byte pitch: not whole 4-byte words
     with pytest.raises(fp4.FP4Error) as e:
         fp4.nvfp4_quantize_columns(x)
     assert e.value.status == fp4.ERR_ALIGN
