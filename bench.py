@@ -73,6 +73,7 @@ DEFAULT_WORKLOAD = MODEL_WEIGHTS
 KERNEL_SOURCES = ["block_scaled_fp4_reduce_b200/csrc/fp4_kernels.cuh",
                   "block_scaled_fp4_reduce_b200/csrc/fp4_codec.cuh",
                   "block_scaled_fp4_reduce_b200/csrc/fp4_grouped.cuh"]
+LAYOUT_SOURCES = ["block_scaled_fp4_reduce_b200/csrc/fp4_layouts.cuh"]
 OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize", "scale_search"]
 
 
@@ -86,9 +87,11 @@ def peaks() -> dict:
     return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(extra: tuple = ()) -> str:
+    """Hash of the kernel sources a traffic capture was taken from (the
+    layout workloads' kernels also live in LAYOUT_SOURCES)."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in list(KERNEL_SOURCES) + list(extra):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -848,7 +851,8 @@ def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict, n_cand: in
         with open(tpath) as f:
             t = json.load(f)
         ent = t.get("workloads", {}).get(w.name, {}).get(name)
-        if ent and ent.get("source_hash") == kernel_source_hash():
+        extra = tuple(LAYOUT_SOURCES) if w.name in LAYOUT_WORKLOADS else ()
+        if ent and ent.get("source_hash") == kernel_source_hash(extra):
             traffic = ent.get("bytes_per_launch")
     if name == "nvfp4_gemm" and gemm_mnk:
         # tensor-bound: 2 M N K flops per launch against the FP4 dense peak,
