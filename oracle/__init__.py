@@ -88,6 +88,9 @@ def lib() -> ctypes.CDLL:
             "oracle_search_candidate_code": (I, [F, F, I]),
             "oracle_nvfp4_scale_search": (I, [P, I, I64, I64, P, P, P, P]),
             "oracle_nvfp4_scale_search_with_g": (I, [P, I, I64, I64, F, P, P, P]),
+            "oracle_search_grid_code": (I, [F, F, I, I]),
+            "oracle_nvfp4_scale_search_grid": (I, [P, I, I64, I64, I, I, I, P, P, P, P]),
+            "oracle_nvfp4_scale_search_grid_with_g": (I, [P, I, I64, I64, F, I, I, I, P, P, P]),
             "oracle_nvfp4_artefact_loss": (I, [P, I, I64, I64, P, P, F, P]),
             "oracle_storage_bytes": (I64, [I64, I64, I64]),
             "oracle_padded_blocks": (I64, [I64, I64, I64]),
@@ -355,6 +358,37 @@ def nvfp4_scale_search(x: np.ndarray):
     _check(lib().oracle_nvfp4_scale_search(_ptr(x), dt, R, C, _ptr(packed), _ptr(scales),
                                            ctypes.byref(g), _ptr(loss)))
     return packed, scales, g.value, loss
+
+
+def search_grid_code(amax_b: float, g: float, num: int, q: int) -> int:
+    return lib().oracle_search_grid_code(float(amax_b), float(g), int(num), int(q))
+
+
+def nvfp4_scale_search_grid(x: np.ndarray, n: int, p: int, q: int):
+    """Brute force over the n candidates (p + k) / q x A_b / (6g), k < n,
+    of every block.  Returns (packed, scales, g, block_loss)."""
+    x, dt = _input(x)
+    R, C = _shape(x)
+    packed = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    loss = np.zeros((R, C // 16), np.float64)
+    g = ctypes.c_float()
+    _check(lib().oracle_nvfp4_scale_search_grid(_ptr(x), dt, R, C, int(n), int(p), int(q), _ptr(packed),
+                                                _ptr(scales), ctypes.byref(g), _ptr(loss)))
+    return packed, scales, g.value, loss
+
+
+def nvfp4_scale_search_grid_with_g(x: np.ndarray, g: float, n: int, p: int, q: int):
+    """The grid search at a given global scale.  Returns (packed, scales,
+    block_loss)."""
+    x, dt = _input(x)
+    R, C = _shape(x)
+    packed = np.zeros((R, C // 2), np.uint8)
+    scales = np.zeros((R, C // 16), np.uint8)
+    loss = np.zeros((R, C // 16), np.float64)
+    _check(lib().oracle_nvfp4_scale_search_grid_with_g(_ptr(x), dt, R, C, float(g), int(n), int(p), int(q),
+                                                       _ptr(packed), _ptr(scales), _ptr(loss)))
+    return packed, scales, loss
 
 
 def nvfp4_scale_search_with_g(x: np.ndarray, g: float):

@@ -46,7 +46,8 @@
  *     via frexp, clamped to [-127, 127]; an all-zero block clamps to -127.
  *   - Scale search: 64 candidates m_k * A_b / (6 g), m_k = (147 + k) / 210,
  *     k = 0..63 (0.70 .. 1.00 inclusive); loss of the emitted artefact,
- *     summed in double; exact ties go to the larger scale.
+ *     summed in double; exact ties go to the larger scale.  The grid form
+ *     takes m_k = (p + k) / q, k = 0..n-1, for any n, p, q up to 2^20.
  */
 #include <float.h>
 #include <math.h>
@@ -512,26 +513,36 @@ double oracle_nv_block_loss(const float *xb, int sc, float g)
     return loss;
 }
 
-/* Raw candidate k of a block: the E4M3 code nearest to the exact rational
- * (147 + k) A_b / (1260 g) = m_k * A_b / (6 g).  Numerator (<= 32 bits) and
- * denominator (<= 35 bits) are exact in double; one rounding follows. */
-int oracle_search_candidate_code(float amax_b, float g, int k)
+/* Raw candidate of numerator num over the grid denominator q: the E4M3
+ * code nearest to num A_b / (6 q g), the quotient rounded once to double.
+ * With num, q <= 2^20 the numerator (<= 44 bits) and the denominator
+ * (<= 47 bits) are exact in double. */
+int oracle_search_grid_code(float amax_b, float g, int num, int q)
 {
-    double t = ((double)(SEARCH_NUM0 + k) * (double)amax_b) /
-               (6.0 * SEARCH_DEN * (double)g);
+    double t = ((double)num * (double)amax_b) / (6.0 * (double)q * (double)g);
     return oracle_e4m3_encode(t);
 }
 
-/* Brute-force search over all 64 candidates of every block at a given
- * global scale g: the scale with the smallest loss wins, exact ties go to
- * the larger scale.  Emits packed codes, scale codes and (optionally) the
- * winning loss per block. */
-int oracle_nvfp4_scale_search_with_g(const void *x, int dtype, int64_t rows, int64_t cols,
-                                     float g, uint8_t *packed, uint8_t *scales,
-                                     double *block_loss)
+/* Raw candidate k of the fixed grid: m_k = (147 + k) / 210, i.e. the code
+ * nearest to (147 + k) A_b / (1260 g) = m_k * A_b / (6 g). */
+int oracle_search_candidate_code(float amax_b, float g, int k)
+{
+    return oracle_search_grid_code(amax_b, g, SEARCH_NUM0 + k, SEARCH_DEN);
+}
+
+/* Brute-force search over the n candidates m_k = (p + k) / q, k = 0..n-1,
+ * of every block at a given global scale g: the scale with the smallest
+ * loss wins, exact ties go to the larger scale.  Emits packed codes, scale
+ * codes and (optionally) the winning loss per block.  The fixed search is
+ * n = 64, p = 147, q = 210. */
+int oracle_nvfp4_scale_search_grid_with_g(const void *x, int dtype, int64_t rows, int64_t cols,
+                                          float g, int n, int p, int q, uint8_t *packed,
+                                          uint8_t *scales, double *block_loss)
 {
     if (cols % 16 || rows < 0 || cols < 0)
         return ORACLE_ERR_SHAPE;
+    if (n < 1 || p < 1 || q < 1 || p + (int64_t)n - 1 > (1 << 20) || q > (1 << 20))
+        return ORACLE_ERR_ARG;
     int64_t nblocks = rows * cols / 16;
     for (int64_t b = 0; b < nblocks; ++b) {
         float xb[16];
@@ -545,8 +556,8 @@ int oracle_nvfp4_scale_search_with_g(const void *x, int dtype, int64_t rows, int
         }
         int best = -1;
         double best_loss = 0.0;
-        for (int k = 0; k < SEARCH_N; ++k) {
-            int c = oracle_search_candidate_code(ab, g, k);
+        for (int k = 0; k < n; ++k) {
+            int c = oracle_search_grid_code(ab, g, p + k, q);
             double loss = oracle_nv_block_loss(xb, c, g);
             if (best < 0 || loss < best_loss ||
                 (loss == best_loss && oracle_e4m3_value(c) > oracle_e4m3_value(best))) {
@@ -562,6 +573,34 @@ int oracle_nvfp4_scale_search_with_g(const void *x, int dtype, int64_t rows, int
             block_loss[b] = best_loss;
     }
     return ORACLE_OK;
+}
+
+int oracle_nvfp4_scale_search_with_g(const void *x, int dtype, int64_t rows, int64_t cols,
+                                     float g, uint8_t *packed, uint8_t *scales,
+                                     double *block_loss)
+{
+    return oracle_nvfp4_scale_search_grid_with_g(x, dtype, rows, cols, g, SEARCH_N, SEARCH_NUM0,
+                                                 SEARCH_DEN, packed, scales, block_loss);
+}
+
+/* The full search over the grid (n, p, q): tensor amax -> g (as for
+ * NVFP4) -> per-block search. */
+int oracle_nvfp4_scale_search_grid(const void *x, int dtype, int64_t rows, int64_t cols, int n,
+                                   int p, int q, uint8_t *packed, uint8_t *scales, float *g_out,
+                                   double *block_loss)
+{
+    if (cols % 16 || rows < 0 || cols < 0)
+        return ORACLE_ERR_SHAPE;
+    float amax, g;
+    int st = oracle_tensor_amax(x, dtype, rows * cols, &amax);
+    if (st)
+        return st;
+    st = oracle_nv_global_scale(amax, &g);
+    if (st)
+        return st;
+    *g_out = g;
+    return oracle_nvfp4_scale_search_grid_with_g(x, dtype, rows, cols, g, n, p, q, packed, scales,
+                                                 block_loss);
 }
 
 /* The full search: tensor amax -> g (as for NVFP4) -> per-block search. */

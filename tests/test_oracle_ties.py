@@ -185,3 +185,57 @@ def test_four_over_six_matches_independent_model(oracle_mod):
         assert int(s[b]) == want
         n4 += want == c4 and c4 != c6
     assert 0 < n4 < xf.shape[0]
+
+
+# The search over a general grid m_k = (p + k) / q, k < n (the candidate grid
+# as a parameter of the call; the fixed search is n = 64, p = 147, q = 210).
+def model_grid_candidates(amax_b: float, g, n: int, p: int, q: int) -> list[int]:
+    return sorted({e4m3_code(Fraction(p + k, q) * Fraction(float(amax_b)) / (6 * Fraction(float(F32(g)))))
+                   for k in range(n)})
+
+
+def model_grid_search(xs, g, n, p, q):
+    amax_b = max(abs(float(F32(x))) for x in xs)
+    losses = {c: model_loss(xs, c, g) for c in model_grid_candidates(amax_b, g, n, p, q)}
+    best = min(losses, key=lambda c: (losses[c], -c))
+    rest = [v for c, v in losses.items() if c != best]
+    return best, losses[best], (min(rest) if rest else None)
+
+
+@pytest.mark.parametrize("grid", [(32, 16, 48), (8, 100, 100), (20, 40, 50), (5, 200, 160), (64, 147, 210)])
+def test_grid_search_argmin_matches_independent_model(oracle_mod, grid):
+    """Random blocks: the oracle's choice over the grid is the exact argmin
+    of the independent model over the same candidate set."""
+    n, p, q = grid
+    x = workloads.as_oracle_array(workloads.generate(workloads.with_shape(workloads.SEARCH_4K, 2, 512, 40 + n)))
+    xf = oracle_mod.bf16_to_f32(x).reshape(-1, 16)
+    packed, scales, g, loss = oracle_mod.nvfp4_scale_search_grid(x, n, p, q)
+    s, lo = scales.reshape(-1), loss.reshape(-1)
+    checked = 0
+    for b in range(xf.shape[0]):
+        xs = [float(v) for v in xf[b]]
+        best, best_loss, runner = model_grid_search(xs, g, n, p, q)
+        assert abs(Fraction(float(lo[b])) - best_loss) <= best_loss * Fraction(1, 10 ** 12)
+        if runner is not None and runner != best_loss and abs(runner - best_loss) <= best_loss * Fraction(1, 10 ** 12):
+            continue
+        assert int(s[b]) == best, f"grid {grid} block {b}: oracle chose {s[b]}, the exact argmin is {best}"
+        checked += 1
+    assert checked >= 48
+
+
+def test_grid_search_of_one_max_based_candidate_is_the_quantiser(oracle_mod):
+    """n = 1 with p = q leaves only the max-based scale A_b / (6g): the
+    search emits exactly the NVFP4 quantiser's codes and scales."""
+    x = workloads.as_oracle_array(workloads.generate(workloads.with_shape(workloads.ACT_8K, 3, 256, 41)))
+    for p in (1, 7, 210):
+        packed, scales, g, _ = oracle_mod.nvfp4_scale_search_grid(x, 1, p, p)
+        p0, s0, g0 = oracle_mod.nvfp4_quantize(x)
+        assert g == g0
+        assert np.array_equal(packed, p0) and np.array_equal(scales, s0)
+
+
+def test_grid_search_rejects_empty_and_oversized_grids(oracle_mod):
+    x = np.zeros((1, 16), np.float32)
+    for n, p, q in ((0, 147, 210), (64, 0, 210), (64, 147, 0), (2, 1 << 20, 4), (4, 16, (1 << 20) + 1)):
+        with pytest.raises(Exception):
+            oracle_mod.nvfp4_scale_search_grid(x, n, p, q)
