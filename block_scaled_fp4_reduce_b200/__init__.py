@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
             "fp4_dequantize": (I, [I, P, P, P, I64, I64, P, I, P]),
             "fp4_scale_search": (I, [P, I, I64, I64, P, P, P, P, P, SZ, P, P]),
             "fp4_scale_search_with_amax": (I, [P, I, I64, I64, P, P, P, P, P, P, P]),
+            "fp4_scale_search_grid": (I, [P, I, I64, I64, I, I, I, P, P, P, P, P, SZ, P, P]),
             "fp4_e2m1_round": (I, [P, P, I64, P]),
             "fp4_e2m1_roundtrip": (I, [P, P, I64, P]),
             "fp4_nv_encode_quotient": (I, [P, P, P, I64, P]),
@@ -542,7 +543,10 @@ def dequantize_grouped(qs, out_dtype=torch.bfloat16, outs=None, stream=None) -> 
     return ys
 
 
-def scale_search(x: torch.Tensor, with_loss: bool = True, workspace=None, status=None, stream=None) -> Quantized:
+def scale_search(x: torch.Tensor, with_loss: bool = True, workspace=None, status=None, stream=None,
+                 grid=None) -> Quantized:
+    """MSE scale search; `grid` = (n_cand, p, q) searches the candidates
+    (p + k) / q x A_b / (6g), k < n_cand (default: the fixed 64, 147, 210)."""
     R, C = _shape2(x)
     dev = x.device
     packed = torch.empty((R, C // 2), dtype=torch.uint8, device=dev)
@@ -551,7 +555,13 @@ def scale_search(x: torch.Tensor, with_loss: bool = True, workspace=None, status
     loss = torch.empty((R, C // 16), dtype=torch.float32, device=dev) if with_loss else None
     ws = workspace if workspace is not None else workspace_for(x)
     st = status if status is not None else new_status(dev)
-    _check(fp4_scale_search(x, packed, scales, g, loss, ws, st, stream), "fp4_scale_search")
+    if grid is None:
+        _check(fp4_scale_search(x, packed, scales, g, loss, ws, st, stream), "fp4_scale_search")
+    else:
+        n_cand, p, q = grid
+        _check(lib().fp4_scale_search_grid(_p(x), _dtype_code(x), R, C, int(n_cand), int(p), int(q), _p(packed),
+                                           _p(scales), _p(g), _p(loss), _p(ws), ws.numel() * ws.element_size(),
+                                           _p(st), _stream(stream)), "fp4_scale_search_grid")
     return Quantized(NVFP4, packed, scales, g, st, R, C, block_loss=loss)
 
 

@@ -91,16 +91,40 @@ fp4_status launch_block_kernel(K kernel, const T *x, int64_t n, const float *ama
     });
 }
 
+template <typename T, bool kFixed>
+fp4_status launch_search_t(const T *x, int64_t n, const float *amax, uint8_t *packed, uint8_t *scales,
+                           float *global_scale, float *block_loss, int32_t *status, cudaStream_t stream,
+                           int n_cand, int p, int q)
+{
+    uint2 *pk = reinterpret_cast<uint2 *>(packed);
+    auto kernel = fp4::scale_search_kernel<T, kFixed>;
+    return for_chunks(n / 16, [&](int64_t first, int count) {
+        const int grid = grid_for(kernel, count, kThreads);
+        if (grid <= 0)
+            return FP4_ERR_CUDA;
+        return launch(kernel, grid, stream, x + first * 16, count, amax, pk + first, scales + first, global_scale,
+                      block_loss ? block_loss + first : block_loss, status, p, p + n_cand - 1, q);
+    });
+}
+
+// n_cand = 0: the fixed grid of 64 candidates (147 + k) / 210.
 fp4_status launch_search(const void *x, fp4_dtype dtype, int64_t n, const float *amax,
                          uint8_t *packed, uint8_t *scales, float *global_scale,
-                         float *block_loss, int32_t *status, cudaStream_t stream)
+                         float *block_loss, int32_t *status, cudaStream_t stream,
+                         int n_cand = 0, int p = 0, int q = 0)
 {
-    if (dtype == FP4_BF16)
-        return launch_block_kernel(fp4::scale_search_kernel<uint16_t>,
-                                   static_cast<const uint16_t *>(x), n, amax, packed, scales,
-                                   global_scale, block_loss, status, stream);
-    return launch_block_kernel(fp4::scale_search_kernel<float>, static_cast<const float *>(x), n,
-                               amax, packed, scales, global_scale, block_loss, status, stream);
+    const bool bf = dtype == FP4_BF16;
+    const uint16_t *xb = static_cast<const uint16_t *>(x);
+    const float *xf = static_cast<const float *>(x);
+    if (n_cand == 0)
+        return bf ? launch_search_t<uint16_t, true>(xb, n, amax, packed, scales, global_scale, block_loss, status,
+                                                    stream, 0, 0, 0)
+                  : launch_search_t<float, true>(xf, n, amax, packed, scales, global_scale, block_loss, status,
+                                                 stream, 0, 0, 0);
+    return bf ? launch_search_t<uint16_t, false>(xb, n, amax, packed, scales, global_scale, block_loss, status,
+                                                 stream, n_cand, p, q)
+              : launch_search_t<float, false>(xf, n, amax, packed, scales, global_scale, block_loss, status,
+                                              stream, n_cand, p, q);
 }
 } // namespace
 
@@ -277,6 +301,34 @@ fp4_status fp4_scale_search(const void *x, fp4_dtype dtype, int64_t rows, int64_
         return st;
     return launch_search(x, dtype, n, amax, packed, scales, global_scale, block_loss, status,
                          stream);
+}
+
+fp4_status fp4_scale_search_grid(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols, int n_cand, int p,
+                                 int q, uint8_t *packed, uint8_t *scales, float *global_scale, float *block_loss,
+                                 void *workspace, size_t workspace_bytes, int32_t *status, cudaStream_t stream)
+{
+    if (n_cand < 1 || p < 16 || q < 1 || (int64_t)p + n_cand - 1 > (1 << 20) || q > (1 << 20))
+        return FP4_ERR_INVALID_ARG;
+    if (!global_scale || !status || !valid_dtype(dtype))
+        return FP4_ERR_INVALID_ARG;
+    fp4_status st = check_shape(rows, cols, 16);
+    if (st != FP4_OK)
+        return st;
+    const int64_t n = rows * cols;
+    if (n > 0 && (!x || !packed || !scales))
+        return FP4_ERR_INVALID_ARG;
+    if (!aligned(x, 32) || !aligned(packed, 16) || !aligned(block_loss, 4))
+        return FP4_ERR_ALIGN;
+    if (!workspace || workspace_bytes < fp4_workspace_bytes(FP4_NVFP4, rows, cols) ||
+        !aligned(workspace, 4))
+        return FP4_ERR_WORKSPACE;
+    uint32_t *ws = static_cast<uint32_t *>(workspace);
+    float *amax = reinterpret_cast<float *>(ws + kWsAmax);
+    st = launch_amax(x, dtype, n, ws, amax, status, stream);
+    if (st != FP4_OK)
+        return st;
+    return launch_search(x, dtype, n, amax, packed, scales, global_scale, block_loss, status, stream, n_cand,
+                         p, q);
 }
 
 fp4_status fp4_scale_search_with_amax(const void *x, fp4_dtype dtype, int64_t rows,

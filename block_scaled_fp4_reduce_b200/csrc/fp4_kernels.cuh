@@ -748,26 +748,41 @@ template <typename T> struct BlockSearch {
     }
 };
 
-template <typename T>
+// The candidate grid m_k = (p + k) / q, k = 0..n-1 (the fixed search: 64,
+// 147, 210) is passed as num_lo = p, num_hi = p + n - 1 and q; with p >= 16
+// consecutive raw candidates differ by a factor of at most 17/16, so they
+// hit every code from c_lo (k = 0) to c_hi (k = n - 1), as above.  num and
+// q are at most 2^20: num A_b and 6 q g are exact in double.  kFixed: the
+// fixed grid, compiled in (the arguments are ignored).
+constexpr int kSearchP = 147, kSearchQ = 210, kSearchN = 64;
+
+template <typename T, bool kFixed>
 __global__ void __launch_bounds__(kThreads, 4)
     scale_search_kernel(const T *__restrict__ x, int n_blocks, const float *amax,
                         uint2 *__restrict__ packed, uint8_t *__restrict__ scales,
-                        float *global_scale, float *__restrict__ block_loss, int32_t *status)
+                        float *global_scale, float *__restrict__ block_loss, int32_t *status,
+                        int num_lo_arg, int num_hi_arg, int q_arg)
 {
     pdl_begin();
     float g;
     if (!nv_prologue(amax, global_scale, status, g))
         return;
+    const int num_lo = kFixed ? kSearchP : num_lo_arg;
+    const int num_hi = kFixed ? kSearchP + kSearchN - 1 : num_hi_arg;
+    const int q = kFixed ? kSearchQ : q_arg;
     const NvScaleConsts sc = nv_scale_consts(g);
-    const double g1260 = 1260.0 * (double)g;      // exact: 9 + 24 significant bits
-    const float inv_lo = (float)(147.0 / g1260);  // RN32(0.7 / (6g))
+    const double den = 6.0 * (double)q * (double)g;      // exact: at most 23 + 24 significant bits
+    const float inv_lo = (float)((double)num_lo / den);  // RN32 of m_0 / (6g), within an ulp
+    const float inv_hi = (float)((double)num_hi / den);
+    const bool hi_is_max = kFixed || num_hi == q; // the largest candidate is the max-based scale
     const bool exact_always = !(g >= 0x1p-116f);
     const int stride = (int)(gridDim.x * blockDim.x);
     for (int blk = (int)(blockIdx.x * blockDim.x + threadIdx.x); blk < n_blocks; blk += stride) {
         BlockSearch<T> bs;
         const float amax_b = bs.setup(x, blk, g, exact_always);
-        const uint32_t c_hi = nv_scale_code_mg(amax_b, sc.inv6g, sc.g, 6.0f, sc.six_g);
-        bs.c_lo = nv_scale_code(amax_b, inv_lo, 147.0, g1260);
+        const uint32_t c_hi = hi_is_max ? nv_scale_code_mg(amax_b, sc.inv6g, sc.g, 6.0f, sc.six_g)
+                                        : nv_scale_code(amax_b, inv_hi, (double)num_hi, den);
+        bs.c_lo = nv_scale_code(amax_b, inv_lo, (double)num_lo, den);
         bs.best_c = c_hi;
         bs.next_c = c_hi;
         const Screen s0 = screen(bs.xk, c_hi, g, bs.k);

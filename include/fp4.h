@@ -199,6 +199,19 @@ fp4_status fp4_scale_search(const void *x, fp4_dtype dtype, int64_t rows, int64_
                             float *block_loss, void *workspace, size_t workspace_bytes,
                             int32_t *status, cudaStream_t stream);
 
+/* fp4_scale_search over a caller's candidate grid: m_k = (p + k) / q for
+ * k = 0..n_cand-1 (fp4_scale_search is n_cand = 64, p = 147, q = 210); each
+ * candidate the E4M3 code nearest to (p + k) A_b / (6 q g), the quotient
+ * rounded once to double, exactly as the fixed grid.  Requires n_cand >= 1,
+ * p >= 16 (then consecutive candidates lie within a factor 17/16, so every
+ * E4M3 code between the smallest and the largest candidate is one of
+ * them), p + n_cand - 1 <= 2^20 and 1 <= q <= 2^20; otherwise
+ * FP4_ERR_INVALID_ARG.  m_k may exceed 1 (scales above the max-based one,
+ * saturating at 448).  Everything else as fp4_scale_search. */
+fp4_status fp4_scale_search_grid(const void *x, fp4_dtype dtype, int64_t rows, int64_t cols, int n_cand, int p,
+                                 int q, uint8_t *packed, uint8_t *scales, float *global_scale, float *block_loss,
+                                 void *workspace, size_t workspace_bytes, int32_t *status, cudaStream_t stream);
+
 /* Scale search given a tensor amax already in device memory (e.g. from
  * fp4_tensor_amax, shared with fp4_nvfp4_quantize_with_amax so the tensor
  * is read once for both).  Same outputs and rules as fp4_scale_search with

@@ -445,3 +445,41 @@ def test_dequant_foreign_scale_bytes():
     torch.cuda.synchronize()
     assert_same_bits(yn, oracle.nvfp4_dequantize(packed.numpy(), s_nv.numpy(), g.item(), R, C), "NV foreign")
     assert_same_bits(ym, oracle.mxfp4_dequantize(packed.numpy(), s_mx.numpy(), R, C), "MX foreign")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("grid", [(32, 16, 48), (8, 100, 100), (20, 40, 50), (5, 200, 160), (64, 147, 210),
+                                  (1, 16, 16), (128, 16, 100), (3, 1000, 4096)])
+def test_scale_search_grid_parity(dtype, grid):
+    """The search over a caller's candidate grid (p + k) / q, k < n: codes,
+    scales, g and the per-block loss bit for bit against the oracle's brute
+    force over the same grid, including grids reaching above the max-based
+    scale (saturating at 448) and the single max-based candidate."""
+    w = workloads.with_shape(workloads.SEARCH_4K, 48, 512, 50 + grid[0])
+    x = workloads.generate(w).to(dtype)
+    q = fp4.scale_search(x.to(DEV), grid=grid)
+    torch.cuda.synchronize()
+    q.check()
+    p, s, g, loss = oracle.nvfp4_scale_search_grid(odata(x), *grid)
+    assert q.global_scale.item() == g
+    assert_same(q.scales, s, f"grid {grid} scales")
+    assert_same(q.packed, p, f"grid {grid} packed")
+    with np.errstate(over="ignore"):
+        loss32 = loss.astype(np.float32)
+    assert_same(q.block_loss, loss32, f"grid {grid} block loss")
+
+
+def test_scale_search_grid_arguments():
+    L = fp4.lib()
+    x = torch.randn(4, 64, device=DEV)
+    pk = torch.empty(4 * 32, dtype=torch.uint8, device=DEV)
+    sc = torch.empty(4 * 4, dtype=torch.uint8, device=DEV)
+    g = torch.empty(1, dtype=torch.float32, device=DEV)
+    ws = fp4.workspace_for(x)
+    st = fp4.new_status(DEV)
+    P = lambda t: t.data_ptr()  # noqa: E731
+    for n, p, q in ((0, 147, 210), (64, 15, 210), (64, 147, 0), (2, 1 << 20, 4), (4, 16, (1 << 20) + 1)):
+        assert L.fp4_scale_search_grid(P(x), fp4.F32, 4, 64, n, p, q, P(pk), P(sc), P(g), None, P(ws),
+                                       ws.numel() * ws.element_size(), P(st), None) == fp4.ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert st.item() == 0
