@@ -241,3 +241,15 @@ def test_with_amax_argument_errors():
         assert fn(P(x), fp4.F32, 8, 40, P(ab[1:]), P(pk), P(sc), P(g), P(st), None) == fp4.ERR_ALIGN
         assert fn(P(x), fp4.F32, 8, 40, P(a), P(pk), P(sc), None, P(st), None) == fp4.ERR_INVALID_ARG
     torch.cuda.synchronize()
+
+
+def test_with_amax_nonfinite_amax_sets_status():
+    """A non-finite amax handed in is a data error (NONFINITE in the status
+    word), as for the plain calls' own amax."""
+    x = rand(8, 40, torch.float32, seed=3).to(DEV)
+    for bad in (float("inf"), float("nan")):
+        a = torch.full((1,), bad, dtype=torch.float32, device=DEV)
+        for call in (fp4.nvfp4_quantize_padded, fp4.nvfp4_quantize_columns):
+            q = call(x, amax=a)
+            torch.cuda.synchronize()
+            assert q.status.item() == fp4.ERR_NONFINITE, (call.__name__, bad)
