@@ -36,19 +36,23 @@ fp4_status operand_map(const uint8_t *p, int64_t rows, int64_t K, CUtensorMap *m
     return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
 }
 
-// 2-D tensor map of an MMA scale layout viewed as uint32 [tiles, 128] (one
-// 512-byte tile per row; rows / 128 bands of K / 64 tiles): box 128 x 4, the
-// four tiles of one 256-element K step of one band.
-fp4_status scale_map(const uint8_t *sf, int64_t rows, int64_t K, CUtensorMap *map)
+// 4-D tensor maps of an MMA scale layout (rows / 128 bands of K / 64 tiles of
+// 512 bytes) that place every tile four times: dimension 0 the 128 words of
+// a tile, dimension 1 four replicas (stride 0), then the tile within its
+// band and the band (box 128 x 4 x 2 x 1, in the order the wide copy reads:
+// two tiles of one band for A, one tile of two bands for B).
+fp4_status scale_map_rep(const uint8_t *sf, int64_t rows, int64_t K, bool band_inner, CUtensorMap *map)
 {
     EncodeTiled enc = encode_tiled();
     if (!enc)
         return FP4_ERR_CUDA;
-    const cuuint64_t dims[2] = {128u, (cuuint64_t)((rows / 128) * (K / 64))};
-    const cuuint64_t strides[1] = {512u};
-    const cuuint32_t box[2] = {128u, 4u};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t *>(sf), dims, strides, box,
+    const cuuint64_t tiles = (cuuint64_t)(K / 64), bands = (cuuint64_t)(rows / 128);
+    const cuuint64_t band_stride = tiles * 512u;
+    const cuuint64_t dims[4] = {128u, 4u, band_inner ? bands : tiles, band_inner ? tiles : bands};
+    const cuuint64_t strides[3] = {0u, band_inner ? band_stride : 512u, band_inner ? 512u : band_stride};
+    const cuuint32_t box[4] = {128u, 4u, 2u, 1u};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<uint8_t *>(sf), dims, strides, box,
                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
@@ -127,7 +131,8 @@ fp4_status launch_pair(const uint8_t *packed_a, const uint8_t *sfa, const float 
     std::memset(&map_d, 0, sizeof(map_d));
     fp4_status st;
     if ((st = operand_map(packed_a, M, K, &map_a)) != FP4_OK || (st = operand_map(packed_b, N, K, &map_b)) != FP4_OK ||
-        (st = scale_map(sfa, M, K, &map_sfa)) != FP4_OK || (st = scale_map(sfb, N, K, &map_sfb)) != FP4_OK ||
+        (st = scale_map_rep(sfa, M, K, false, &map_sfa)) != FP4_OK ||
+        (st = scale_map_rep(sfb, N, K, true, &map_sfb)) != FP4_OK ||
         (st = out_map(d, M, N, &map_d)) != FP4_OK)
         return st;
     const int64_t tiles = (M / fp4::kPairTileM) * (N / fp4::kPairTileN);
@@ -228,14 +233,12 @@ fp4_status fp4_nvfp4_gemm_ex(const uint8_t *packed_a, const uint8_t *scales_a_mm
     const int sms = sm_count(dev);
     if (sms <= 0 || dev >= kMaxDevices)
         return FP4_ERR_CUDA;
-    // The pair kernel once its 256 x 256 tiles give every SM pair work and K
-    // is short enough that its persistent epilogue overlap pays; for long K
-    // the one-CTA kernel's deeper copy pipeline per SM (two CTAs x three
-    // stages) wins (measured on B200: 8192^3 3.08 against 2.86 PFLOP/s,
-    // 8192 x 4096 x 14336 3.15 against 3.23).
+    // The pair kernel once its 256 x 256 tiles give every SM pair work
+    // (measured on B200 with its wide scale copies: 8192 x 4096 x 14336 3.66
+    // against 3.18 PFLOP/s for the one-CTA kernel, 8192^3 3.60 against 2.86,
+    // 4096 x 4096 x 14336 3.24 against 2.77).
     if (kernel == FP4_GEMM_CTA_PAIR ||
-        (kernel == FP4_GEMM_AUTO && pair_shape && K <= 8192 &&
-         (M / fp4::kPairTileM) * (N / fp4::kPairTileN) >= sms / 2))
+        (kernel == FP4_GEMM_AUTO && pair_shape && (M / fp4::kPairTileM) * (N / fp4::kPairTileN) >= sms / 2))
         return launch_pair(packed_a, scales_a_mma, global_scale_a, packed_b, scales_b_mma, global_scale_b, M, N, K, d,
                            status, stream, dev);
     static bool attr_set[kMaxDevices] = {false};

@@ -462,12 +462,19 @@ __global__ void __launch_bounds__(128, 1)
 //
 // Roles (320 threads per CTA): warp 0 of both CTAs loads (2-D TMA, 128-byte
 // swizzle) this CTA's 128 rows of A and of B and the scale tiles (its own
-// 128 rows of A's, all 256 rows of B's) into a five-stage ring; every copy
+// 128 rows of A's, all 256 rows of B's) into a three-stage ring; every copy
 // completes on the leader CTA's "full" barrier, so the leader sees the
 // stage of both CTAs arrive.  Warp 1 of the leader issues: scale tiles to
 // tensor memory (tcgen05.cp, which reaches the same columns of both CTAs),
 // four K = 64 MMAs per stage, and a commit that arrives on the "empty"
-// barrier of the stage in both CTAs.  After a tile's last stage a commit
+// barrier of the stage in both CTAs.  A scale copy costs the tensor pipe
+// about the same per instruction whatever its width, so the scales go over
+// in six 128-lane x 256-bit copies per stage (A's for two K steps, or B's
+// two bands for one, each) rather than twelve 32-lane x 128-bit ones with
+// four-way replication: the stage holds every 512-byte scale tile four
+// times (one per 32-lane quarter of tensor memory), placed by TMA loads
+// from maps whose replica dimension has stride 0.  The copy writes exactly
+// the columns the 32x128b.warpx4 copies wrote.  After a tile's last stage a commit
 // arrives on "acc_full" in both CTAs.  Warps 2..9 of both CTAs drain the
 // accumulator: each reads its 32 lanes (warp % 4) and one 128-column half
 // into registers, releases the accumulator (an arrival on the leader's
@@ -484,10 +491,10 @@ __global__ void __launch_bounds__(128, 1)
 // ---------------------------------------------------------------------------
 constexpr int kPairTileM = 256;
 constexpr int kPairTileN = 256;
-constexpr int kPairStages = 5;
-constexpr int kPairSfaBytes = 4 * 512; // this CTA's 128 rows of A: four 4-block scale tiles
-constexpr int kPairSfbBytes = 8 * 512; // both 128-row bands of the B tile
-constexpr int kPairStageBytes = 2 * kGemmOpBytes + kPairSfaBytes + kPairSfbBytes; // 38 KB
+constexpr int kPairStages = 3;
+constexpr int kPairSfaBytes = 4 * 4 * 512; // this CTA's 128 rows of A: four scale tiles, each four times
+constexpr int kPairSfbBytes = 8 * 4 * 512; // both 128-row bands of the B tile: eight tiles, each four times
+constexpr int kPairStageBytes = 2 * kGemmOpBytes + kPairSfaBytes + kPairSfbBytes; // 56 KB
 constexpr int kPairOutBytes = 32 * 32 * 4; // one epilogue staging tile
 constexpr int kPairEpiWarps = 8;
 constexpr int kPairThreads = 320;
@@ -547,6 +554,16 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
                  : "memory");
 }
 
+// 4-D TMA tile load (pair form, completing on the leader's barrier).
+__device__ __forceinline__ void tma_load_4d_pair(void *dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
+                                                 uint32_t bar_cl)
+{
+    asm volatile("cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar_cl)
+                 : "memory");
+}
+
 // 2-D TMA store of a shared-memory box to (x = column, y = row); bulk group.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y)
 {
@@ -579,6 +596,21 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t cols)
 __device__ __forceinline__ void tc_copy_sf_pair(uint32_t taddr, uint64_t sdesc)
 {
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of a 128-row x 32-byte scale block for the wide
+// copy: two 2 KB halves (the first and second 16 bytes of every row), each
+// 128 rows x 16 bytes in 8-row core matrices 128 bytes apart; the halves
+// are 2 KB apart.
+__device__ __forceinline__ uint64_t smem_desc_sf_wide(uint32_t addr)
+{
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(2048 >> 4) << 16) | (8ull << 32) | (1ull << 46);
+}
+
+// 128 lanes x 256 bits into tensor memory: eight columns of every lane.
+__device__ __forceinline__ void tc_copy_sf_wide_pair(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 __device__ __forceinline__ void tc_mma_nvfp4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -678,10 +710,17 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                         mbar_expect_tx(&full[s], 2u * kPairStageBytes); // both CTAs' copies
                     tma_load_2d_pair(st, &map_a, k * 128, tm * kPairTileM + (int)rank * kGemmTile, bar);
                     tma_load_2d_pair(st + kGemmOpBytes, &map_b, k * 128, tn * kPairTileN + (int)rank * kGemmTile, bar);
-                    tma_load_2d_pair(sf, &map_sfa, 0, (tm * 2 + (int)rank) * sf_tiles_per_band + 4 * k, bar);
-                    tma_load_2d_pair(sf + kPairSfaBytes, &map_sfb, 0, (tn * 2) * sf_tiles_per_band + 4 * k, bar);
-                    tma_load_2d_pair(sf + kPairSfaBytes + 4 * 512, &map_sfb, 0,
-                                     (tn * 2 + 1) * sf_tiles_per_band + 4 * k, bar);
+                    // every scale tile four times (one copy per 32-lane quarter of
+                    // tensor memory), from maps whose replica dimension has stride
+                    // 0: A's tiles 2j, 2j + 1 as [tile 2j x4][tile 2j+1 x4] at
+                    // 4096 j, B's tile i of both bands as [band 0 x4][band 1 x4]
+                    // at 4096 i
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+                        tma_load_4d_pair(sf + 4096 * j, &map_sfa, 0, 0, 4 * k + 2 * j, tm * 2 + (int)rank, bar);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        tma_load_4d_pair(sf + kPairSfaBytes + 4096 * i, &map_sfb, 0, 0, tn * 2, 4 * k + i, bar);
                     issued_steps = it + 1;
                 }
                 __syncwarp();
@@ -715,16 +754,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                         const uint32_t sfb_addr = sfa_addr + kPairSfaBytes;
                         const uint32_t sfa_t = tmem + kPairTileN + (uint32_t)(it % kPairSfRing) * kPairSfCols;
                         const uint32_t sfb_t = sfa_t + 16;
+                        // A's scales for MMAs 2j and 2j + 1 in columns 8j..8j+3 and
+                        // 8j+4..8j+7; B's for MMA i: rows 0..127 in columns
+                        // 8i..8i+3, rows 128..255 in 8i+4..8i+7 -- one wide copy
+                        // each (the copies cost per instruction, not per byte)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j)
+                            tc_copy_sf_wide_pair(sfa_t + 8 * j, smem_desc_sf_wide(sfa_addr + 4096 * j));
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
-                            tc_copy_sf_pair(sfa_t + 4 * i, smem_desc_sf(sfa_addr + 512 * i));
-                        // B's scales for MMA i: rows 0..127 in columns 8i..8i+3,
-                        // rows 128..255 in 8i+4..8i+7
-#pragma unroll
-                        for (int b = 0; b < 2; ++b)
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                tc_copy_sf_pair(sfb_t + 8 * i + 4 * b, smem_desc_sf(sfb_addr + 512 * (4 * b + i)));
+                            tc_copy_sf_wide_pair(sfb_t + 8 * i, smem_desc_sf_wide(sfb_addr + 4096 * i));
 #pragma unroll
                         for (int i = 0; i < 4; ++i) // four MMAs of K = 64 (32 bytes of each 128-byte row)
                             tc_mma_nvfp4_pair(tmem, smem_desc_sw128(a_addr + 32 * i), smem_desc_sw128(b_addr + 32 * i),
