@@ -432,7 +432,10 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
     return d;
 }
 
-__device__ __forceinline__ uint32_t nv_encode8(const float (&x)[8], const NvRecip &q)
+// The bracket step alone: the codes of RN(x r_lo), and `exact` set when
+// they are not known to be v's (the brackets' codes differ, or d is
+// subnormal), i.e. when the eight IEEE quotients are needed.
+__device__ __forceinline__ uint32_t nv_bracket8(const float (&x)[8], const NvRecip &q, bool &exact)
 {
     float a[8], b[8];
     const uint64_t rlo = pack2(q.lo, q.lo), rhi = pack2(q.hi, q.hi);
@@ -442,15 +445,38 @@ __device__ __forceinline__ uint32_t nv_encode8(const float (&x)[8], const NvReci
         unpack2(mul2(xp, rlo), a[2 * j], a[2 * j + 1]);
         unpack2(mul2(xp, rhi), b[2 * j], b[2 * j + 1]);
     }
-    uint32_t ca = e2m1x8(a);
+    const uint32_t ca = e2m1x8(a);
     const uint32_t cb = e2m1x8(b);
-    if (ca != cb || q.exact_only) {
+    exact = ca != cb || q.exact_only;
+    return ca;
+}
+
+// E2M1 code (low nibble) of one value.
+__device__ __forceinline__ uint32_t e2m1_nibble(float v)
+{
+    uint32_t out;
+    asm("{\n\t"
+        ".reg .b8 b;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
+        "cvt.u32.u8 %0, b;\n\t"
+        "}"
+        : "=r"(out)
+        : "f"(v), "f"(0.0f));
+    return out & 15u;
+}
+
+__device__ __forceinline__ uint32_t nv_encode8(const float (&x)[8], const NvRecip &q)
+{
+    bool exact;
+    uint32_t c = nv_bracket8(x, q, exact);
+    if (exact) {
+        float a[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             a[i] = __fdiv_rn(x[i], q.d);
-        ca = e2m1x8(a);
+        c = e2m1x8(a);
     }
-    return ca;
+    return c;
 }
 
 // NVFP4 dequantised value fl32(fl32(p * s_b) * g); p * s_b is exact.

@@ -48,57 +48,15 @@
 
 #include <cuda.h>
 
+#include "fp4_async.cuh"
 #include "fp4_kernels.cuh"
 
 namespace fp4 {
 
 // ---------------------------------------------------------------------------
-// mbarrier and TMA helpers.  Every wait is bounded (kWaitTries polls); a
-// kernel whose wait runs out records FP4_ERR_TIMEOUT (kStatusTimeout).
+// TMA tile loads (the mbarrier helpers and the bounded wait are in
+// fp4_async.cuh).
 // ---------------------------------------------------------------------------
-constexpr int32_t kStatusTimeout = 8;
-constexpr uint32_t kWaitTries = 1u << 22;
-
-__device__ __forceinline__ uint32_t smem_addr(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-                 : "memory");
-}
-
-// Bounded wait for phase `parity` of the barrier; false when the tries run out.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
-{
-    for (uint32_t t = 0; t < kWaitTries; ++t) {
-        uint32_t done;
-        asm volatile("{\n\t"
-                     ".reg .pred p;\n\t"
-                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                     "selp.u32 %0, 1, 0, p;\n\t"
-                     "}"
-                     : "=r"(done)
-                     : "r"(smem_addr(bar)), "r"(parity)
-                     : "memory");
-        if (done)
-            return true;
-    }
-    return false;
-}
-
 // 2-D TMA tile load of box (x = column, y = row) into shared memory,
 // completing on `bar`.  x (the innermost coordinate) times the element size
 // is a multiple of 16 bytes.
@@ -219,14 +177,6 @@ __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t addr)
     return (uint64_t)((addr & 0x3FFFFu) >> 4) | (8ull << 32) | (1ull << 46);
 }
 
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_addr(dst)),
-                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
-                 : "memory");
-}
-
 __device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t cols)
 {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)),
@@ -333,7 +283,7 @@ __global__ void __launch_bounds__(128, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(&done, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_init_fence();
         consumed_steps = 0;
     }
     __syncwarp();
@@ -667,7 +617,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int tiles_m = M / kPairTileM;
     const int n_tiles = tiles_m * (N / kPairTileN);
     const int kt_steps = K / kGemmKStep;
-    const int sf_tiles_per_band = K / 64;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPairStages; ++s) {
@@ -677,7 +626,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         mbar_init(&acc_full, 1);
         mbar_init(&acc_empty, 2 * kPairEpiWarps);
         mbar_init(&mma_done, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_init_fence();
         issued_steps = 0;
         consumed_steps = 0;
     }

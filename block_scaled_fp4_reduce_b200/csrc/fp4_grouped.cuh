@@ -130,6 +130,37 @@ __device__ __forceinline__ void grouped_tiles(const Table &grp, Enter &&enter, L
     }
 }
 
+// As grouped_tiles, with the choice between a tile's two paths uniform
+// across the CTA: a tile all of whose kThreads * U units exist goes to
+// `whole(e, b0)` (this thread's units b0 + u * kThreads, u < U; all lanes of
+// every warp together, so the body may use warp collectives), the units of a
+// short tile one at a time to `one(e, b)`.
+template <int U, typename Table, typename Enter, typename Whole, typename One>
+__device__ __forceinline__ void grouped_tiles_cta(const Table &grp, Enter &&enter, Whole &&whole, One &&one)
+{
+    constexpr int kTile = kThreads * U;
+    const int tiles = grp.tile_first[grp.n];
+    int e = 0, cur = -1;
+    bool ok = false;
+    for (int t = (int)blockIdx.x; t < tiles; t += (int)gridDim.x) {
+        e = entry_from(grp.tile_first, t, e);
+        if (e != cur) {
+            cur = e;
+            ok = enter(e);
+        }
+        if (!ok)
+            continue;
+        const int nb = grp.first[e + 1] - grp.first[e];
+        const int first = (t - grp.tile_first[e]) * kTile;
+        if (first + kTile <= nb) {
+            whole(e, first + (int)threadIdx.x);
+        } else {
+            for (int b = first + (int)threadIdx.x; b < nb; b += kThreads)
+                one(e, b);
+        }
+    }
+}
+
 // Tiles of `units` units at U units per thread (host and device).
 __host__ __device__ constexpr int grouped_tile_count(int64_t units, int U)
 {
@@ -177,22 +208,57 @@ __global__ void __launch_bounds__(kThreads, kNvGroupedCtasPerSm)
     const T *x = nullptr;
     uint2 *packed = nullptr;
     uint8_t *scales = nullptr;
-    Blk<T, 16> blk[kNvGroupedU];
-    grouped_tiles<kNvGroupedU>(
-        grp,
-        [&](int e) {
-            int32_t err;
-            const float g = nv_global_scale(__ldcg(grp.amax[e]), err);
-            if (err)
-                return false;
-            sc = nv_scale_consts(g);
-            x = static_cast<const T *>(grp.x[e]);
-            packed = grp.packed[e];
-            scales = grp.scales[e];
-            return true;
-        },
-        [&](int u, int, int b) { load_blk(x, b, blk[u]); },
-        [&](int u, int, int b) { nv_quantize_block(blk[u], sc, packed + b, scales + b); });
+    constexpr int U = kNvGroupedU;
+    auto enter = [&](int e) {
+        int32_t err;
+        const float g = nv_global_scale(__ldcg(grp.amax[e]), err);
+        if (err)
+            return false;
+        sc = nv_scale_consts(g);
+        x = static_cast<const T *>(grp.x[e]);
+        packed = grp.packed[e];
+        scales = grp.scales[e];
+        return true;
+    };
+    auto one = [&](int, int b) {
+        Blk<T, 16> blk;
+        load_blk(x, b, blk);
+        nv_quantize_block(blk, sc, packed + b, scales + b);
+    };
+    if constexpr (sizeof(T) == 2) {
+        __shared__ NvExactQueue<U> queues[kThreads / 32];
+        NvExactQueue<U> &q = queues[threadIdx.x >> 5];
+        grouped_tiles_cta<U>(
+            grp, enter,
+            [&](int, int b0) {
+                Blk<T, 16> blk[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    load_blk(x, b0 + u * kThreads, blk[u]);
+                uint2 pk[U];
+                uint32_t code[U];
+                nv_quantize_warp(blk, sc, q, pk, code);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    packed[b0 + u * kThreads] = pk[u];
+                    scales[b0 + u * kThreads] = (uint8_t)code[u];
+                }
+            },
+            one);
+    } else {
+        grouped_tiles_cta<U>(
+            grp, enter,
+            [&](int e, int b0) {
+                Blk<T, 16> blk[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    load_blk(x, b0 + u * kThreads, blk[u]);
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    nv_quantize_block(blk[u], sc, packed + b0 + u * kThreads, scales + b0 + u * kThreads);
+            },
+            one);
+    }
 }
 
 // ---------------------------------------------------------------------------

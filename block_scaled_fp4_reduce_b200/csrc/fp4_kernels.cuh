@@ -167,6 +167,22 @@ __device__ __forceinline__ void stream_units(int n, Load &&load, Work &&work)
     }
 }
 
+// As stream_units, but the main loop's condition is taken for the warp's
+// last lane, so that all 32 lanes run it together (its body may use warp
+// collectives): `whole(i, stride)` takes units i + u * stride, u < U; the
+// units left over go one at a time to `one(i)`.
+template <int U, typename Whole, typename One>
+__device__ __forceinline__ void stream_units_warp(int n, Whole &&whole, One &&one)
+{
+    const int stride = (int)(gridDim.x * blockDim.x);
+    const int to_last_lane = 31 - (int)(threadIdx.x & 31u);
+    int i = (int)(blockIdx.x * blockDim.x + threadIdx.x);
+    for (; i + to_last_lane + (U - 1) * stride < n; i += U * stride)
+        whole(i, stride);
+    for (; i < n; i += stride)
+        one(i);
+}
+
 // Largest unit count one launch of a stream_units kernel takes.
 constexpr int64_t kMaxUnitsPerLaunch = (int64_t)1 << 30;
 
@@ -316,13 +332,110 @@ __device__ __forceinline__ uint2 nv_block_codes(const Blk<T, 16> &b, uint32_t c,
 // NVFP4 codes and scale byte of one loaded 16-block under the global scale
 // g (constants sc): written to *packed / *scale.
 template <typename T>
+__device__ __forceinline__ uint2 nv_block_quantize(const Blk<T, 16> &blk, const NvScaleConsts &sc,
+                                                   uint32_t &code)
+{
+    const float amax_b = __uint_as_float(absmax_bits(blk));
+    code = nv_scale_code_mg(amax_b, sc.inv6g, sc.g, 6.0f, sc.six_g);
+    return nv_block_codes(blk, code, sc.g);
+}
+
+template <typename T>
 __device__ __forceinline__ void nv_quantize_block(const Blk<T, 16> &blk, const NvScaleConsts &sc,
                                                   uint2 *packed, uint8_t *scale)
 {
-    const float amax_b = __uint_as_float(absmax_bits(blk));
-    const uint32_t code = nv_scale_code_mg(amax_b, sc.inv6g, sc.g, 6.0f, sc.six_g);
-    *packed = nv_block_codes(blk, code, sc.g);
+    uint32_t code;
+    *packed = nv_block_quantize(blk, sc, code);
     *scale = (uint8_t)code;
+}
+
+// ---------------------------------------------------------------------------
+// Warp-shared exact path (bf16 input).  A half-block whose bracket does not
+// settle its codes (nv_bracket8) needs its eight IEEE quotients x / d.  Done
+// by its own thread, the eight divisions run while the warp's other lanes
+// wait, and on tie-rich data (bf16 weights, where an element is often the
+// tensor amax times a power of two and a block scale of significand 1.5 or
+// 1.75 puts x / d on an E2M1 midpoint) about half the warps meet such a
+// half-block at every step.  Here the U blocks of every lane are first
+// bracketed; flagged half-blocks go to a per-warp queue in shared memory
+// (their eight elements and d); then the whole warp works the queue off with
+// one element per lane (eight lanes per half-block, four half-blocks per
+// pass, the nibbles gathered by three shuffles), and each owner reads its
+// code word back.  The codes are those of the per-thread path bit for bit:
+// the same quotients, the same conversion.  All 32 lanes of the warp must
+// call it together.
+// ---------------------------------------------------------------------------
+template <int U> struct NvExactQueue {
+    static constexpr int kCap = 32 * 2 * U; // every half-block of the warp
+    uint4 x[kCap];     // the eight bf16 elements
+    uint32_t d[kCap];  // bits of d = fl32(s_b g); after the pass, the code word
+};
+
+template <int U>
+__device__ __forceinline__ void nv_quantize_warp(const Blk<uint16_t, 16> (&blk)[U],
+                                                 const NvScaleConsts &sc, NvExactQueue<U> &q,
+                                                 uint2 (&pk)[U], uint32_t (&code)[U])
+{
+    const int lane = (int)(threadIdx.x & 31u);
+    const uint32_t below = (1u << lane) - 1u;
+    int count = 0;
+    uint32_t cw[U][2];
+    int slot[U][2];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const float amax_b = __uint_as_float(absmax_bits(blk[u]));
+        code[u] = nv_scale_code_mg(amax_b, sc.inv6g, sc.g, 6.0f, sc.six_g);
+        const NvRecip r = nv_recip(__fmul_rn(e4m3_pos_to_f32(code[u]), sc.g));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float x[8];
+            elems8(blk[u], 8 * h, x);
+            bool exact;
+            cw[u][h] = nv_bracket8(x, r, exact);
+            exact = exact && code[u] != 0u; // a zero scale gives zero codes
+            slot[u][h] = -1;
+            const uint32_t m = __ballot_sync(0xFFFFFFFFu, exact);
+            if (m) {
+                if (exact) {
+                    const int s = count + __popc(m & below);
+                    q.x[s] = make_uint4(blk[u].w[4 * h], blk[u].w[4 * h + 1], blk[u].w[4 * h + 2],
+                                        blk[u].w[4 * h + 3]);
+                    q.d[s] = __float_as_uint(r.d);
+                    slot[u][h] = s;
+                }
+                count += __popc(m);
+            }
+        }
+    }
+    if (count) {
+        __syncwarp();
+        const int i = lane & 7;
+        for (int q0 = 0; q0 < count; q0 += 4) {
+            const int s = q0 + (lane >> 3);
+            uint32_t nib = 0;
+            if (s < count) {
+                const uint32_t w = reinterpret_cast<const uint32_t *>(&q.x[s])[i >> 1];
+                const float xv = __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
+                nib = e2m1_nibble(__fdiv_rn(xv, __uint_as_float(q.d[s]))) << (4 * i);
+            }
+            nib |= __shfl_xor_sync(0xFFFFFFFFu, nib, 1);
+            nib |= __shfl_xor_sync(0xFFFFFFFFu, nib, 2);
+            nib |= __shfl_xor_sync(0xFFFFFFFFu, nib, 4);
+            if (i == 0 && s < count)
+                q.d[s] = nib;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                if (slot[u][h] >= 0)
+                    cw[u][h] = q.d[slot[u][h]];
+        __syncwarp();
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+        pk[u] = code[u] ? make_uint2(cw[u][0], cw[u][1]) : make_uint2(0u, 0u);
 }
 
 template <typename T>
@@ -336,10 +449,37 @@ __global__ void __launch_bounds__(kThreads)
     if (!nv_prologue(amax, global_scale, status, g))
         return;
     const NvScaleConsts sc = nv_scale_consts(g);
-    Blk<T, 16> blk[4];
-    stream_units<4>(
-        n_blocks, [&](int u, int b) { load_blk(x, b, blk[u]); },
-        [&](int u, int b) { nv_quantize_block(blk[u], sc, packed + b, scales + b); });
+    constexpr int U = 4;
+    if constexpr (sizeof(T) == 2) {
+        __shared__ NvExactQueue<U> queues[kThreads / 32];
+        NvExactQueue<U> &q = queues[threadIdx.x >> 5];
+        stream_units_warp<U>(
+            n_blocks,
+            [&](int b0, int stride) {
+                Blk<T, 16> blk[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    load_blk(x, b0 + u * stride, blk[u]);
+                uint2 pk[U];
+                uint32_t code[U];
+                nv_quantize_warp(blk, sc, q, pk, code);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    packed[b0 + u * stride] = pk[u];
+                    scales[b0 + u * stride] = (uint8_t)code[u];
+                }
+            },
+            [&](int b) {
+                Blk<T, 16> blk;
+                load_blk(x, b, blk);
+                nv_quantize_block(blk, sc, packed + b, scales + b);
+            });
+    } else {
+        Blk<T, 16> blk[U];
+        stream_units<U>(
+            n_blocks, [&](int u, int b) { load_blk(x, b, blk[u]); },
+            [&](int u, int b) { nv_quantize_block(blk[u], sc, packed + b, scales + b); });
+    }
 }
 
 // ---------------------------------------------------------------------------

@@ -51,21 +51,70 @@ int sm_count(int &dev)
     return n;
 }
 
+// Per-device facts about a kernel, cached by the kernel's address (kernels
+// of different instantiations can share a function type).
+struct KernelFacts {
+    const void *kernel;
+    int dev;
+    int resident;   // resident CTAs per SM (0: not queried yet)
+    bool smem_set;  // dynamic shared-memory limit raised
+};
+
+KernelFacts &kernel_facts(const void *kernel, int dev)
+{
+    static std::mutex mu;
+    static KernelFacts table[256];
+    static int used = 0;
+    static KernelFacts spare;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (table[i].kernel == kernel && table[i].dev == dev)
+            return table[i];
+    if (used == 256) { // more kernels x devices than this library has: no caching
+        spare = KernelFacts{kernel, dev, 0, false};
+        return spare;
+    }
+    table[used] = KernelFacts{kernel, dev, 0, false};
+    return table[used++];
+}
+
 // Resident CTAs per SM of `kernel` at `block` threads and `smem` bytes of
-// dynamic shared memory (cached per device and kernel instantiation; a
-// kernel is always queried with the same block and smem).
+// dynamic shared memory (cached per device and kernel; a kernel is always
+// queried with the same block and smem).
 template <typename K> int resident_ctas(K kernel, int dev, int block = kThreads, size_t smem = 0)
 {
-    static int cache[kMaxDevices] = {0};
-    if (dev < kMaxDevices && cache[dev] > 0)
-        return cache[dev];
+    KernelFacts &f = kernel_facts(reinterpret_cast<const void *>(kernel), dev);
+    if (f.resident > 0)
+        return f.resident;
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, smem) != cudaSuccess ||
-        n <= 0)
+        n <= 0) {
+        (void)cudaGetLastError();
         n = 1;
-    if (dev < kMaxDevices)
-        cache[dev] = n;
+    }
+    f.resident = n;
     return n;
+}
+
+// Lets `kernel` launch with `bytes` of dynamic shared memory on the current
+// device (above the default 48 KB); false on a CUDA error.
+template <typename K> bool smem_attr(K kernel, int bytes)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    KernelFacts &f = kernel_facts(reinterpret_cast<const void *>(kernel), dev);
+    if (f.smem_set)
+        return true;
+    if (cudaFuncSetAttribute(reinterpret_cast<const void *>(kernel), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    f.smem_set = true;
+    return true;
 }
 
 // Persistent grid: enough CTAs for `work` items at `per_cta` items each,
