@@ -170,14 +170,47 @@ __global__ void __launch_bounds__(kThreads)
     const NvScaleConsts sc = nv_scale_consts(g);
     const char *x_end = reinterpret_cast<const char *>(x + (int64_t)nbp.div(n_blocks) * K);
     constexpr int U = pad_units<16>();
-    PadWin<T, 16> pw[U];
-    stream_units<U>(
-        n_blocks, [&](int u, int b) { pad_win_load(x, x_end, b, nbp, K, pw[u]); },
-        [&](int u, int b) {
-            Blk<T, 16> blk;
-            pad_win_block(pw[u], blk);
-            nv_quantize_block(blk, sc, packed + b, scales + b);
-        });
+    if constexpr (sizeof(T) == 2) {
+        // whole warp steps take the warp-shared exact path
+        __shared__ NvExactQueue<U> queues[kThreads / 32];
+        NvExactQueue<U> &q = queues[threadIdx.x >> 5];
+        stream_units_warp<U>(
+            n_blocks,
+            [&](int b0, int stride) {
+                PadWin<T, 16> pw[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    pad_win_load(x, x_end, b0 + u * stride, nbp, K, pw[u]);
+                Blk<T, 16> blk[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    pad_win_block(pw[u], blk[u]);
+                uint2 pk[U];
+                uint32_t code[U];
+                nv_quantize_warp(blk, sc, q, pk, code);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    packed[b0 + u * stride] = pk[u];
+                    scales[b0 + u * stride] = (uint8_t)code[u];
+                }
+            },
+            [&](int b) {
+                PadWin<T, 16> pw;
+                pad_win_load(x, x_end, b, nbp, K, pw);
+                Blk<T, 16> blk;
+                pad_win_block(pw, blk);
+                nv_quantize_block(blk, sc, packed + b, scales + b);
+            });
+    } else {
+        PadWin<T, 16> pw[U];
+        stream_units<U>(
+            n_blocks, [&](int u, int b) { pad_win_load(x, x_end, b, nbp, K, pw[u]); },
+            [&](int u, int b) {
+                Blk<T, 16> blk;
+                pad_win_block(pw[u], blk);
+                nv_quantize_block(blk, sc, packed + b, scales + b);
+            });
+    }
 }
 
 template <typename T, bool kCeil>
@@ -458,6 +491,7 @@ __global__ void __launch_bounds__(kThreads, kNvColCtasPerSm)
     constexpr int kScaleRow = 20;                // staged scale bytes per output row (16 + 4 of padding)
     __shared__ __align__(16) uint8_t st_packed[2][kTileCols * 128];
     __shared__ __align__(16) uint8_t st_scales[2][kTileCols * kScaleRow];
+    __shared__ NvExactQueue<kPerWord> queues[sizeof(T) == 2 ? kThreads / 32 : 1];
     pdl_begin();
     float g;
     if (!nv_prologue(amax, global_scale, status, g))
@@ -475,6 +509,8 @@ __global__ void __launch_bounds__(kThreads, kNvColCtasPerSm)
         const int w = strip * 32 + lane;                     // word column of W
         const int r0 = band * kNvColRows + warp * 32;      // this warp's first row
         if (w < Cw && r0 < R) {
+            // all 32 lanes here (the strip is whole): the warp-shared exact path
+            const bool whole_warp = strip * 32 + 32 <= Cw;
             uint32_t sb2[kPerWord]; // the two scale bytes of each column
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -490,25 +526,40 @@ __global__ void __launch_bounds__(kThreads, kNvColCtasPerSm)
                     for (int i = 0; i < 16; ++i, src += Cw)
                         v[i] = rh + i < R ? __ldcg(src) : 0u;
                 }
+                Blk<T, 16> b[kPerWord];
 #pragma unroll
                 for (int p = 0; p < kPerWord; ++p) {
-                    Blk<T, 16> b;
                     if constexpr (sizeof(T) == 2) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            b.w[i] = __byte_perm(v[2 * i], v[2 * i + 1], p ? 0x7632 : 0x5410);
+                            b[p].w[i] = __byte_perm(v[2 * i], v[2 * i + 1], p ? 0x7632 : 0x5410);
                     } else {
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            b.w[i] = v[i];
+                            b[p].w[i] = v[i];
                     }
-                    uint2 q;
-                    uint8_t sbyte;
-                    nv_quantize_block(b, sc, &q, &sbyte);
+                }
+                uint2 q[kPerWord];
+                uint32_t sbyte[kPerWord];
+                if constexpr (sizeof(T) == 2) {
+                    if (whole_warp) {
+                        nv_quantize_warp(b, sc, queues[warp], q, sbyte);
+                    } else {
+#pragma unroll
+                        for (int p = 0; p < kPerWord; ++p)
+                            q[p] = nv_block_quantize(b[p], sc, sbyte[p]);
+                    }
+                } else {
+#pragma unroll
+                    for (int p = 0; p < kPerWord; ++p)
+                        q[p] = nv_block_quantize(b[p], sc, sbyte[p]);
+                }
+#pragma unroll
+                for (int p = 0; p < kPerWord; ++p) {
                     const int cl = lane * kPerWord + p;
                     const int chunk = (2 * warp + h) ^ col_swizzle<kPerWord>(cl);
-                    *reinterpret_cast<uint2 *>(&st_packed[s][cl * 128 + 8 * chunk]) = q;
-                    sb2[p] = h ? sb2[p] | ((uint32_t)sbyte << 8) : (uint32_t)sbyte;
+                    *reinterpret_cast<uint2 *>(&st_packed[s][cl * 128 + 8 * chunk]) = q[p];
+                    sb2[p] = h ? sb2[p] | (sbyte[p] << 8) : sbyte[p];
                 }
             }
 #pragma unroll

@@ -19,7 +19,7 @@ next to midpoints:
   (the queue holds every half-block of every warp step).
 
 Codes and scale bytes must equal the oracle's bit for bit, for the
-single-tensor call and for the grouped call."""
+single-tensor, grouped, padded (ragged rows) and column-wise calls."""
 import numpy as np
 import pytest
 import torch
@@ -74,6 +74,14 @@ def midpoint_fraction(x: torch.Tensor) -> float:
     return float(near.mean())
 
 
+def check_q(q, p, s, g):
+    torch.cuda.synchronize()
+    assert q.status.item() == 0
+    assert q.global_scale.item() == g
+    assert_same(q.scales, s, "scales")
+    assert_same(q.packed, p, "packed")
+
+
 def check_single(x: torch.Tensor):
     xo = odata(x)
     p, s, g = oracle.nvfp4_quantize(xo)
@@ -109,3 +117,15 @@ def test_tie_rich_grouped():
         assert nv[i].global_scale.item() == g, f"item {i} g"
         assert_same(nv[i].scales, s, f"item {i} scales")
         assert_same(nv[i].packed, p, f"item {i} packed")
+
+
+def test_tie_rich_padded():
+    x = tie_rich(2048, 4096, seed=40)[:, :4095].contiguous()
+    check_q(fp4.nvfp4_quantize_padded(x.to(DEV)), *oracle.nvfp4_quantize_padded(odata(x)))
+
+
+def test_tie_rich_columns():
+    x = tie_rich(4096, 2048, seed=41)
+    xt = x.t().contiguous()
+    assert midpoint_fraction(xt[:256]) > 0.02  # ties along the columns too
+    check_q(fp4.nvfp4_quantize_columns(x.to(DEV)), *oracle.nvfp4_quantize_columns(odata(x)))
