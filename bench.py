@@ -397,9 +397,34 @@ class GroupedPath:
             (L.fp4_dequantize_grouped, (fp4.MXFP4, cp(self.d_mx), k, fp4.BF16, st)),
         ]
         self.results = [self.nv_p, self.nv_s, self.nv_g, self.mx_p, self.mx_s, self.status]
+        # The same five calls per layer (the layer's seven matrices), for the
+        # end-to-end run that streams the set layer by layer: the elements
+        # [e0, e1) of x that the layer holds, and its calls.
+        per = len(workloads.MODEL_MATRICES)
+        self.layers = []
+        e0 = 0
+        for li in range(0, k, per):
+            e1 = e0 + sum(sizes[li:li + per])
+            n_l = min(per, k - li)
+            sl = lambda a, j=li: ctypes.c_void_p(ctypes.addressof(a) + j * ctypes.sizeof(a._type_))  # noqa: E731
+            calls = [
+                (L.fp4_tensor_amax_grouped, (sl(self.q_nv), n_l, fp4.BF16, ws, self.ws.numel(), stp, st)),
+                (L.fp4_nvfp4_quantize_grouped_with_amax, (sl(self.q_nv), n_l, fp4.BF16, ws, stp, st)),
+                (L.fp4_mxfp4_quantize_grouped, (sl(self.q_mx), n_l, fp4.BF16, stp, st)),
+                (L.fp4_dequantize_grouped, (fp4.NVFP4, sl(self.d_nv), n_l, fp4.BF16, st)),
+                (L.fp4_dequantize_grouped, (fp4.MXFP4, sl(self.d_mx), n_l, fp4.BF16, st)),
+            ]
+            self.layers.append((e0, e1, calls))
+            e0 = e1
 
     step = Path.step
     check_status = Path.check_status
+
+    def layer_outputs(self, e0: int, e1: int):
+        """(device tensor, slice) of every per-element result of elements
+        [e0, e1): the NVFP4 and MXFP4 packed codes and scale bytes."""
+        return [(self.nv_p, slice(e0 // 2, e1 // 2)), (self.nv_s, slice(e0 // 16, e1 // 16)),
+                (self.mx_p, slice(e0 // 2, e1 // 2)), (self.mx_s, slice(e0 // 32, e1 // 32))]
 
 
 class LayoutPath:
@@ -598,6 +623,62 @@ def e2e_pipelined(path, x, x_host, steps: int) -> tuple[float, str]:
                         "from pinned host memory, every result downloaded; no L2 flush between steps")
 
 
+def e2e_layered(path, x, x_host, steps: int) -> tuple[float, str]:
+    """Milliseconds for `steps` steps over the weight set, each streamed layer
+    by layer the way a caller quantising a model feeds it: layer l's
+    matrices are uploaded on an upload stream, their five grouped calls run
+    on the compute stream once the upload is in, and their packed codes and
+    scale bytes go back on a download stream, so that uploads, kernels and
+    downloads of different layers overlap (the link is full duplex).  Every
+    step uploads the whole set from pinned host memory and downloads every
+    result (the per-matrix g and the status word after the last layer); one
+    event pair on the device spans each step, and the steps are timed one
+    after another."""
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in path.results]
+    host_of = {id(t): h for t, h in zip(path.results, host_out)}
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    n_layers = len(path.layers)
+
+    def one() -> float:
+        ev_up = [torch.cuda.Event() for _ in range(n_layers)]
+        ev_c = [torch.cuda.Event() for _ in range(n_layers)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(up)
+        comp.wait_event(start)
+        down.wait_event(start)
+        for l, (e0, e1, calls) in enumerate(path.layers):
+            with torch.cuda.stream(up):
+                x[e0:e1].copy_(x_host[e0:e1], non_blocking=True)
+            ev_up[l].record(up)
+            comp.wait_event(ev_up[l])
+            for fn, args in calls:
+                st = fn(*args)
+                if st != 0:
+                    raise path.fp4.FP4Error(st, fn.__name__)
+            ev_c[l].record(comp)
+            down.wait_event(ev_c[l])
+            with torch.cuda.stream(down):
+                for t, sl in path.layer_outputs(e0, e1):
+                    host_of[id(t)][sl].copy_(t[sl], non_blocking=True)
+        with torch.cuda.stream(down):
+            for t in (path.nv_g, path.status):
+                host_of[id(t)].copy_(t, non_blocking=True)
+        end.record(down)
+        end.synchronize()
+        if int(host_of[id(path.status)].item()) != 0:
+            raise RuntimeError("device status set during the end-to-end run")
+        return start.elapsed_time(end)
+
+    one()  # warm-up: streams, pinned buffers
+    ms = sum(one() for _ in range(steps))
+    return ms, ("layer-streamed: each step uploads the set layer by layer (upload stream), runs the five grouped "
+                "calls on each layer's seven matrices once its upload is in (compute stream) and downloads the "
+                "layer's codes and scale bytes (download stream), so that the three overlap across layers; every "
+                "element uploaded from pinned host memory and every result downloaded each step")
+
+
 def max_over_ranks(values: list[float], device, world: int) -> list[float]:
     """Element-wise max of per-rank timings (one all-reduce; identity at N=1)."""
     if world == 1:
@@ -721,7 +802,9 @@ def run_ours(args, rank: int, world: int, local: int):
     # ---- end to end through the same calls from pinned host memory ---------
     h2d = x.numel() * x.element_size()
     d2h = sum(t.numel() * t.element_size() for t in path.results)
-    if hasattr(path, "twin"):
+    if hasattr(path, "layers"):
+        e2e_ms, e2e_schedule = e2e_layered(path, x, x_host, Ke)
+    elif hasattr(path, "twin"):
         e2e_ms, e2e_schedule = e2e_pipelined(path, x, x_host, Ke)
     else:
         e2e_ms, e2e_schedule = e2e_serial(path, x, x_host, Ke, flush_l2)
