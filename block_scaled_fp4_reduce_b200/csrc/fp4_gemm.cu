@@ -70,23 +70,6 @@ bool set_smem_attr(const void *kernel, int bytes, bool (&done)[kMaxDevices], int
     return true;
 }
 
-// 2-D tensor map of D [M, N] fp32: box 32 x 32 with 128-byte swizzle (the
-// pair kernel's epilogue staging tiles).
-fp4_status out_map(float *d, int64_t M, int64_t N, CUtensorMap *map)
-{
-    EncodeTiled enc = encode_tiled();
-    if (!enc)
-        return FP4_ERR_CUDA;
-    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-    const cuuint64_t strides[1] = {(cuuint64_t)N * 4u};
-    const cuuint32_t box[2] = {32u, 32u};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, d, dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? FP4_OK : FP4_ERR_CUDA;
-}
-
 // Clusters of two CTAs of the pair kernel that fit on the device at once.
 int pair_clusters(int dev)
 {
@@ -123,17 +106,15 @@ fp4_status launch_pair(const uint8_t *packed_a, const uint8_t *sfa, const float 
     const int clusters = pair_clusters(dev);
     if (clusters <= 0)
         return FP4_ERR_CUDA;
-    CUtensorMap map_a, map_b, map_sfa, map_sfb, map_d;
+    CUtensorMap map_a, map_b, map_sfa, map_sfb;
     std::memset(&map_a, 0, sizeof(map_a));
     std::memset(&map_b, 0, sizeof(map_b));
     std::memset(&map_sfa, 0, sizeof(map_sfa));
     std::memset(&map_sfb, 0, sizeof(map_sfb));
-    std::memset(&map_d, 0, sizeof(map_d));
     fp4_status st;
     if ((st = operand_map(packed_a, M, K, &map_a)) != FP4_OK || (st = operand_map(packed_b, N, K, &map_b)) != FP4_OK ||
         (st = scale_map_rep(sfa, M, K, false, &map_sfa)) != FP4_OK ||
-        (st = scale_map_rep(sfb, N, K, true, &map_sfb)) != FP4_OK ||
-        (st = out_map(d, M, N, &map_d)) != FP4_OK)
+        (st = scale_map_rep(sfb, N, K, true, &map_sfb)) != FP4_OK)
         return st;
     const int64_t tiles = (M / fp4::kPairTileM) * (N / fp4::kPairTileN);
     const int64_t pairs = tiles < clusters ? tiles : clusters;
@@ -151,7 +132,7 @@ fp4_status launch_pair(const uint8_t *packed_a, const uint8_t *sfa, const float 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, fp4::nvfp4_gemm_pair_kernel, map_a, map_b, map_sfa, map_sfb, map_d, g_a, g_b,
+    if (cudaLaunchKernelEx(&cfg, fp4::nvfp4_gemm_pair_kernel, map_a, map_b, map_sfa, map_sfb, d, g_a, g_b,
                            (int)M, (int)N, (int)K, status) != cudaSuccess) {
         (void)cudaGetLastError();
         return FP4_ERR_CUDA;

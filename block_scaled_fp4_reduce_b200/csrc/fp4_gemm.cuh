@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(128, 1)
 //
 // Roles (320 threads per CTA): warp 0 of both CTAs loads (2-D TMA, 128-byte
 // swizzle) this CTA's 128 rows of A and of B and the scale tiles (its own
-// 128 rows of A's, all 256 rows of B's) into a three-stage ring; every copy
+// 128 rows of A's, all 256 rows of B's) into a four-stage ring; every copy
 // completes on the leader CTA's "full" barrier, so the leader sees the
 // stage of both CTAs arrive.  Warp 1 of the leader issues: scale tiles to
 // tensor memory (tcgen05.cp, which reaches the same columns of both CTAs),
@@ -428,9 +428,11 @@ __global__ void __launch_bounds__(128, 1)
 // arrives on "acc_full" in both CTAs.  Warps 2..9 of both CTAs drain the
 // accumulator: each reads its 32 lanes (warp % 4) and one 128-column half
 // into registers, releases the accumulator (an arrival on the leader's
-// "acc_empty", 16 per tile), and only then scales and stores -- through a
-// swizzled 32 x 32 staging tile and a TMA store -- so the next tile's MMAs
-// run while the stores drain.  The grid is persistent: cluster p takes
+// "acc_empty", 16 per tile), and only then scales and stores: each lane
+// writes its row's 128 columns (512 contiguous bytes, whole 128-byte lines)
+// straight from registers with 32- or 16-byte stores, so the next tile's
+// MMAs run while the stores drain, and no shared memory goes to staging
+// (it holds a fourth stage instead).  The grid is persistent: cluster p takes
 // tiles p, p + P, ... (M-tile fastest).  Tensor memory (512 columns,
 // allocated by the pair): the accumulator in columns 0..255, then a ring of
 // four scale column sets (16 for A, 32 for B).  All waits are bounded; on
@@ -441,21 +443,19 @@ __global__ void __launch_bounds__(128, 1)
 // ---------------------------------------------------------------------------
 constexpr int kPairTileM = 256;
 constexpr int kPairTileN = 256;
-constexpr int kPairStages = 3;
+constexpr int kPairStages = 4;
 constexpr int kPairSfaBytes = 4 * 4 * 512; // this CTA's 128 rows of A: four scale tiles, each four times
 constexpr int kPairSfbBytes = 8 * 4 * 512; // both 128-row bands of the B tile: eight tiles, each four times
 constexpr int kPairStageBytes = 2 * kGemmOpBytes + kPairSfaBytes + kPairSfbBytes; // 56 KB
-constexpr int kPairOutBytes = 32 * 32 * 4; // one epilogue staging tile
 constexpr int kPairEpiWarps = 8;
 constexpr int kPairThreads = 320;
-constexpr int kPairOutOffset = kPairStages * kPairStageBytes;
-constexpr int kPairSmem = kPairOutOffset + kPairEpiWarps * kPairOutBytes + 1024;
+constexpr int kPairSmem = kPairStages * kPairStageBytes + 1024; // + alignment to 1024 bytes
 constexpr uint32_t kPairSfCols = 16 + 32; // A: 4 columns per MMA; B (256 rows): 8
 constexpr uint32_t kPairSfRing = 4;
 constexpr uint32_t kPairTmemCols = 512;
 static_assert(kPairTileN + kPairSfRing * kPairSfCols <= kPairTmemCols, "tensor memory");
 static_assert(kPairStageBytes % 1024 == 0, "stages stay 1024-byte aligned");
-static_assert(kPairSmem <= 232448 - 512, "shared memory");
+static_assert(kPairSmem <= 232448 - 256, "shared memory (with the static barriers)");
 // M = 256 (bits 24..28 = M / 16), N = 256 (bits 17..22 = N / 8), E2M1 x E2M1,
 // UE4M3 scales, K-major, dense.
 constexpr uint32_t kPairIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kPairTileN / 8) << 17) |
@@ -513,20 +513,6 @@ __device__ __forceinline__ void tma_load_4d_pair(void *dst, const CUtensorMap *m
                  "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar_cl)
                  : "memory");
 }
-
-// 2-D TMA store of a shared-memory box to (x = column, y = row); bulk group.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y)
-{
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y), "r"(smem_addr(src))
-                 : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// This thread's bulk stores have read their shared memory / have finished.
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot, uint32_t cols)
 {
@@ -593,15 +579,17 @@ __device__ __forceinline__ void tc_commit_own(uint64_t *bar)
 }
 
 // map_a / map_b: the packed operands as in nvfp4_gemm_kernel.  map_sfa /
-// map_sfb: the MMA scale layouts viewed as uint32 [tiles, 128] (one 512-byte
-// tile per row, K/64 tiles per 128-row band), box 128 x 4: one K step of
-// one band.  map_d: D fp32, box 32 x 32, 128-byte swizzle.  M and N
-// multiples of 256, K of 256; grid = 2 x pairs, cluster 2.
+// map_sfb: the MMA scale layouts as 4-D uint32 maps (the 128 words of a
+// 512-byte tile, four replicas at stride 0, then K steps and bands: for A
+// K steps inner, for B bands inner), box 128 x 4 x 2 x 1: two tiles (two K
+// steps of A's band, or B's two bands at one K step), each four times.  d:
+// D fp32 row-major (16-byte aligned; 32-byte stores when it is 32-byte
+// aligned).  M and N multiples of 256, K of 256; grid = 2 x pairs, cluster 2.
 __global__ void __launch_bounds__(kPairThreads, 1)
     nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                            const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
-                           const __grid_constant__ CUtensorMap map_d, const float *g_a, const float *g_b, int M, int N,
-                           int K, int32_t *status)
+                           float *__restrict__ d, const float *g_a, const float *g_b, int M, int N, int K,
+                           int32_t *status)
 {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kPairStages], empty[kPairStages], acc_full, acc_empty, mma_done;
@@ -740,11 +728,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 timed_out = true;
         }
     } else {
-        // epilogue, both CTAs: lanes of warp % 4, columns 128 h .. 128 h + 127
+        // epilogue, both CTAs: lanes of warp % 4, columns 128 h .. 128 h + 127;
+        // lane l stores row 32 q + l of this CTA's half of the tile
         const int q = warp & 3, h = (warp - 2) >> 2;
         const float gg = __fmul_rn(__ldcg(g_a), __ldcg(g_b));
         const uint32_t release = cluster_addr(&acc_empty, 0);
-        uint8_t *stg = smem + kPairOutOffset + (warp - 2) * kPairOutBytes;
+        const bool wide = (reinterpret_cast<uintptr_t>(d) & 31u) == 0; // 32-byte stores
         int j = 0;
         for (int t = pair; t < n_tiles; t += n_pairs, ++j) {
             if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full, (uint32_t)j & 1u))) {
@@ -761,29 +750,26 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             if (lane == 0)
                 mbar_arrive_cluster(release); // the accumulator may be overwritten now
             const int tm = t % tiles_m, tn = t / tiles_m;
-            const int row0 = tm * kPairTileM + (int)rank * kGemmTile + q * 32;
-            // 32 x 32 chunks through this warp's staging tile: lane l writes
-            // row l, its 16-byte unit u at unit u ^ (l % 8) (the 128-byte
-            // swizzle; eight lanes cover all banks), then lane 0 stores the
-            // tile with TMA once the previous store has read it.
+            const int row = tm * kPairTileM + (int)rank * kGemmTile + q * 32 + lane;
+            float *drow = d + (int64_t)row * N + tn * kPairTileN + h * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                if (lane == 0)
-                    bulk_wait_read();
-                __syncwarp();
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    *reinterpret_cast<float4 *>(stg + lane * 128 + 16 * (u ^ (lane & 7))) =
-                        make_float4(__fmul_rn(v[c][4 * u], gg), __fmul_rn(v[c][4 * u + 1], gg),
-                                    __fmul_rn(v[c][4 * u + 2], gg), __fmul_rn(v[c][4 * u + 3], gg));
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0)
-                    tma_store_2d(&map_d, stg, tn * kPairTileN + h * 128 + c * 32, row0);
+                for (int u = 0; u < 4; ++u) {
+                    uint32_t o[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        o[i] = __float_as_uint(__fmul_rn(v[c][8 * u + i], gg));
+                    float *p = drow + c * 32 + 8 * u;
+                    if (wide) {
+                        stg_v8(p, o);
+                    } else {
+                        *reinterpret_cast<uint4 *>(p) = make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4 *>(p + 4) = make_uint4(o[4], o[5], o[6], o[7]);
+                    }
+                }
             }
         }
-        if (lane == 0)
-            bulk_wait_all(); // the stores have finished before the CTA ends
     }
     if (timed_out)
         raise_status(status, kStatusTimeout);

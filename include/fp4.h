@@ -346,8 +346,8 @@ fp4_status fp4_scales_to_mma_layout(const uint8_t *scales, int64_t rows, int64_t
  * weight stored N x K) with scales_b_mma; global scales as the quantisers
  * write them.  M and N multiples of 128, K a multiple of 256 (else
  * FP4_ERR_SHAPE); packed, scales and d 16-byte aligned.  One kernel: the
- * CTA-pair kernel (below) when M and N are multiples of 256, K <= 8192 and
- * its 256 x 256 tiles number at least half the SMs, else one CTA per 128 x
+ * CTA-pair kernel (below) when M and N are multiples of 256 and its
+ * 256 x 256 tiles number at least half the SMs, else one CTA per 128 x
  * 128 tile.
  * A copy that never completes ends the kernel with FP4_ERR_TIMEOUT in
  * *status.  The accumulation order inside the tensor core is the
