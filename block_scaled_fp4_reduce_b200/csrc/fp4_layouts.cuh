@@ -236,22 +236,23 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // Dequantise a row-padded layout into the logical [R, K] output.  Unit i is
-// 16 codes of the padded matrix (row i / nup, columns (i % nup) * 16 ..); a
-// warp takes a chunk of 32 consecutive units.  The outputs of consecutive
-// units are contiguous in y, and every unit of a row starts at the same
-// offset s within a 32-byte vector (units are 16 elements apart).  A chunk
-// whose 32 units are whole (16 logical elements each) and lie in one row is
-// written as whole aligned vectors: lane L assembles the vector(s) that
-// start s bytes before its unit from the tail of unit L-1 (moved over by a
-// shuffle) and its own head, and writes them with 256-bit stores; lane 0
-// writes its own head and lane 31 its own tail -- the parts of the chunk's
-// two edge vectors that are theirs -- with the fewest aligned stores that
-// cover them (at most one each of 2, 4, 8 and 16 bytes).  Every store is an
-// L2 write request, and requests are what this kernel runs out of: written
-// element by element, the edges took 89 against 63 us without them on
-// 8192 x 14335.  Any other chunk (a row boundary, a partial unit, the end
-// of the launch) writes each unit's logical elements one by one.  Every
-// output element is written once.
+// 16 codes of the padded matrix (row i / nup, columns (i % nup) * 16 ..).
+// The outputs of consecutive units are contiguous in y, and every unit of a
+// row starts at the same offset s within a 32-byte vector (units are 16
+// elements apart), so the aligned vector(s) that start s bytes before unit u
+// hold the tail of unit u - 1 and the head of unit u.  A warp takes a chunk
+// of 31 units, u = 31 c .. 31 c + 30, and its 32 lanes decode units 31 c - 1
+// .. 31 c + 30: lane L >= 1 moves the tail of lane L - 1's unit over with a
+// shuffle, joins it to its own head and writes the whole vector(s) with
+// 256-bit stores; lane 0 only supplies its unit's tail.  So every vector
+// inside a run of such chunks is written once, whole, by one lane (no
+// partial edge stores: every store is an L2 write request, and the partial
+// stores at both edges of 32-unit chunks cost 3.03 M requests against 1.84 M
+// for the row dequantiser on 8192 x 14335).  A chunk whose 32 decoded units
+// are not all whole (16 logical elements) in one row -- a row boundary, a
+// partial unit, the first chunk of a launch, the end of the launch -- writes
+// every decoded unit's logical elements one by one; the bytes it shares with
+// a neighbouring chunk's vectors are then written twice with the same values.
 template <int K4, int W>
 __device__ __forceinline__ void pad_join(const uint32_t (&q)[2 * W], uint32_t sh, uint32_t *out)
 {
@@ -269,55 +270,8 @@ template <typename TOut> __device__ __forceinline__ void pad_store_elem(TOut *y,
         y[e] = __uint_as_float(word);
 }
 
-// Bytes [LO, HI) of the 32-byte-aligned span p, whose image is the words w,
-// in the fewest aligned stores.
-template <int LO, int HI>
-__device__ __forceinline__ void store_range(uint8_t *p, const uint32_t *w)
-{
-    if constexpr (LO < HI) {
-        constexpr int a = (LO % 32 == 0 && LO + 32 <= HI)   ? 32
-                          : (LO % 16 == 0 && LO + 16 <= HI) ? 16
-                          : (LO % 8 == 0 && LO + 8 <= HI)   ? 8
-                          : (LO % 4 == 0 && LO + 4 <= HI)   ? 4
-                                                            : 2;
-        constexpr int k = LO / 4;
-        if constexpr (a == 32)
-            stg_v8(p + LO, w + k);
-        else if constexpr (a == 16)
-            *reinterpret_cast<uint4 *>(p + LO) = make_uint4(w[k], w[k + 1], w[k + 2], w[k + 3]);
-        else if constexpr (a == 8)
-            *reinterpret_cast<uint2 *>(p + LO) = make_uint2(w[k], w[k + 1]);
-        else if constexpr (a == 4)
-            *reinterpret_cast<uint32_t *>(p + LO) = w[k];
-        else
-            *reinterpret_cast<uint16_t *>(p + LO) = (uint16_t)(w[k] >> (8 * (LO % 4)));
-        store_range<LO + a, HI>(p, w);
-    }
-}
-
-// The head [sb, span) or the tail [0, sb) of a span of 4 W bytes, for a
-// warp-uniform sb (a multiple of the element size, 0 < sb < 32).
-template <int W, bool kHead>
-__device__ __forceinline__ void store_edge(uint8_t *p, const uint32_t *w, int sb)
-{
-    constexpr int S = 4 * W;
-#define FP4_EDGE(SB)                                                                                 \
-    case SB:                                                                                         \
-        if constexpr (kHead)                                                                         \
-            store_range<SB, S>(p, w);                                                                \
-        else                                                                                         \
-            store_range<0, SB>(p, w);                                                                \
-        break;
-    switch (sb) {
-        FP4_EDGE(2) FP4_EDGE(4) FP4_EDGE(6) FP4_EDGE(8) FP4_EDGE(10) FP4_EDGE(12) FP4_EDGE(14)
-        FP4_EDGE(16) FP4_EDGE(18) FP4_EDGE(20) FP4_EDGE(22) FP4_EDGE(24) FP4_EDGE(26) FP4_EDGE(28)
-        FP4_EDGE(30)
-    default: break;
-    }
-#undef FP4_EDGE
-}
-
-constexpr int kPadDqChunks = 4; // chunks of 32 units per warp whose loads go out together
+constexpr int kPadDqChunks = 4; // chunks per warp whose loads go out together
+constexpr int kPadDqStep = 31;  // units a chunk stores (its 32 lanes decode one unit more)
 
 template <bool kNv, typename TOut>
 __global__ void __launch_bounds__(kThreads)
@@ -331,36 +285,39 @@ __global__ void __launch_bounds__(kThreads)
     const float g = kNv ? __ldcg(global_scale) : 1.0f;
     const uint64_t g2 = pack2(g, g);
     const int lane = (int)(threadIdx.x & 31u);
-    const int warp_stride = (int)(gridDim.x * (blockDim.x >> 5)) * 32;
     constexpr int U = kPadDqChunks;
+    const int n_warps = (int)(gridDim.x * (blockDim.x >> 5));
+    const int n_chunks = (n_units + kPadDqStep - 1) / kPadDqStep;
     uint2 pkv[U];
     uint32_t sbv[U];
-    int chunk = 0;
-    for (int base = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 32; base < n_units;
-         base += warp_stride, chunk = (chunk + 1) % U) {
+    int slot = 0;
+    for (int c = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)); c < n_chunks;
+         c += n_warps, slot = (slot + 1) % U) {
         // the codes and scale bytes of the next U chunks, loaded together
-        if (chunk == 0) {
+        if (slot == 0) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int iu = base + u * warp_stride + lane;
-                if (iu < n_units) {
+                const int cu = c + u * n_warps;
+                const int iu = cu * kPadDqStep - 1 + lane;
+                if (cu < n_chunks && iu >= 0 && iu < n_units) {
                     pkv[u] = __ldcg(packed + iu);
                     sbv[u] = __ldcg(scales + (kNv ? iu : (iu >> 1)));
                 }
             }
         }
-        const int i = base + lane;
+        const int i = c * kPadDqStep - 1 + lane; // lane 0: the unit before the chunk
+        const bool valid = i >= 0 && i < n_units;
         int cnt = 0;
         int row = -1;
         int64_t f = 0;
         uint32_t o[kW];
-        if (i < n_units) {
+        if (valid) {
             f = pad_block_start(i, nup, K, 16, cnt, row);
             uint2 pk = pkv[0];
             uint32_t sbyte = sbv[0];
 #pragma unroll
             for (int u = 1; u < U; ++u)
-                if (chunk == u) {
+                if (slot == u) {
                     pk = pkv[u];
                     sbyte = sbv[u];
                 }
@@ -377,14 +334,16 @@ __global__ void __launch_bounds__(kThreads)
             }
         }
         const int row0 = __shfl_sync(0xFFFFFFFFu, row, 0);
-        if (__all_sync(0xFFFFFFFFu, cnt == 16 && row == row0)) {
+        if (__all_sync(0xFFFFFFFFu, valid && cnt == 16 && row == row0)) {
             const uintptr_t start = reinterpret_cast<uintptr_t>(y + f);
             const int sb = (int)(start & 31u); // the same in every lane
             uint8_t *vec = reinterpret_cast<uint8_t *>(start - (uintptr_t)sb);
             if (sb == 0) {
+                if (lane > 0) {
 #pragma unroll
-                for (int v = 0; v < kW / 8; ++v)
-                    stg_v8(vec + 32 * v, o + 8 * v);
+                    for (int v = 0; v < kW / 8; ++v)
+                        stg_v8(vec + 32 * v, o + 8 * v);
+                }
                 continue;
             }
             uint32_t q[2 * kW];
@@ -393,7 +352,7 @@ __global__ void __launch_bounds__(kThreads)
                 q[k] = __shfl_up_sync(0xFFFFFFFFu, o[k], 1);
                 q[kW + k] = o[k];
             }
-            uint32_t out[kW]; // the image of the span at vec (lane 0: its own bytes only)
+            uint32_t out[kW]; // the aligned vector(s) holding the tail of unit L-1 and the head of unit L
             const uint32_t sh = (uint32_t)((32 - sb) & 3) * 8u;
             switch ((sb + 3) >> 2) { // words of unit L-1 in the first vector
             case 1: pad_join<1, kW>(q, sh, out); break;
@@ -409,29 +368,8 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
                 for (int v = 0; v < kW / 8; ++v)
                     stg_v8(vec + 32 * v, out + 8 * v);
-            } else {
-                store_edge<kW, true>(vec, out, sb);
             }
-            if (lane == 31) {
-                // the bytes past the span: the image of the next span holds
-                // this unit's last sb bytes first
-                uint32_t tail[kW];
-#pragma unroll
-                for (int k = 0; k < kW; ++k)
-                    q[k] = o[k];
-                switch ((sb + 3) >> 2) {
-                case 1: pad_join<1, kW>(q, sh, tail); break;
-                case 2: pad_join<2, kW>(q, sh, tail); break;
-                case 3: pad_join<3, kW>(q, sh, tail); break;
-                case 4: pad_join<4, kW>(q, sh, tail); break;
-                case 5: pad_join<5, kW>(q, sh, tail); break;
-                case 6: pad_join<6, kW>(q, sh, tail); break;
-                case 7: pad_join<7, kW>(q, sh, tail); break;
-                default: pad_join<8, kW>(q, sh, tail); break;
-                }
-                store_edge<kW, false>(vec + 4 * kW, tail, sb);
-            }
-        } else if (i < n_units) {
+        } else if (valid) {
 #pragma unroll
             for (int e = 0; e < 16; ++e)
                 if (e < cnt)
