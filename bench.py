@@ -334,6 +334,19 @@ class ShardedPath(Path):
         sharded_step(local_amax, all_reduce_max, rest)
 
 
+def layer_spans(sizes: list[int], per: int) -> list[tuple[int, int, int, int]]:
+    """The weight set's layers for the layer-streamed end-to-end run: per
+    layer (first item, items, first element, end element) of consecutive
+    groups of `per` items (the last group may be short), items laid out one
+    after another in element order."""
+    spans, e0 = [], 0
+    for li in range(0, len(sizes), per):
+        e1 = e0 + sum(sizes[li:li + per])
+        spans.append((li, min(per, len(sizes) - li), e0, e1))
+        e0 = e1
+    return spans
+
+
 class GroupedPath:
     """The whole 7B-class weight set (32 layers x 4 x 4096^2 + 3 x 4096x14336
     bf16 matrices, each generated from its own seed) in one flat device
@@ -400,12 +413,8 @@ class GroupedPath:
         # The same five calls per layer (the layer's seven matrices), for the
         # end-to-end run that streams the set layer by layer: the elements
         # [e0, e1) of x that the layer holds, and its calls.
-        per = len(workloads.MODEL_MATRICES)
         self.layers = []
-        e0 = 0
-        for li in range(0, k, per):
-            e1 = e0 + sum(sizes[li:li + per])
-            n_l = min(per, k - li)
+        for li, n_l, e0, e1 in layer_spans(sizes, len(workloads.MODEL_MATRICES)):
             sl = lambda a, j=li: ctypes.c_void_p(ctypes.addressof(a) + j * ctypes.sizeof(a._type_))  # noqa: E731
             calls = [
                 (L.fp4_tensor_amax_grouped, (sl(self.q_nv), n_l, fp4.BF16, ws, self.ws.numel(), stp, st)),
@@ -415,7 +424,6 @@ class GroupedPath:
                 (L.fp4_dequantize_grouped, (fp4.MXFP4, sl(self.d_mx), n_l, fp4.BF16, st)),
             ]
             self.layers.append((e0, e1, calls))
-            e0 = e1
 
     step = Path.step
     check_status = Path.check_status

@@ -84,3 +84,17 @@ def test_search_candidate_count_matches_its_definition():
         t_lo = float(torch.tensor(a * 147.0 / (1260.0 * g), dtype=torch.float32))
         want += nearest(t_hi) - nearest(t_lo) + 1
     assert bench.search_candidate_count(x, g) == want
+
+
+def test_layer_spans_cover_the_weight_set_once():
+    sizes = [r * c for r, c in workloads.MODEL_MATRICES] * workloads.MODEL_LAYERS
+    per = len(workloads.MODEL_MATRICES)
+    spans = bench.layer_spans(sizes, per)
+    assert len(spans) == workloads.MODEL_LAYERS
+    assert spans[0][0] == 0 and spans[0][2] == 0 and spans[-1][3] == workloads.model_numel()
+    for (li, n, e0, e1), nxt in zip(spans, spans[1:] + [None]):
+        assert n == per and e1 - e0 == sum(sizes[li:li + n])
+        if nxt is not None:
+            assert nxt[0] == li + n and nxt[2] == e1  # contiguous, no gap, no overlap
+    # a short last group
+    assert bench.layer_spans([3, 4, 5, 6, 7], 2) == [(0, 2, 0, 7), (2, 2, 7, 18), (4, 1, 18, 25)]
