@@ -74,6 +74,7 @@ KERNEL_SOURCES = ["block_scaled_fp4_reduce_b200/csrc/fp4_kernels.cuh",
                   "block_scaled_fp4_reduce_b200/csrc/fp4_codec.cuh",
                   "block_scaled_fp4_reduce_b200/csrc/fp4_grouped.cuh"]
 LAYOUT_SOURCES = ["block_scaled_fp4_reduce_b200/csrc/fp4_layouts.cuh"]
+GEMM_SOURCES = ["block_scaled_fp4_reduce_b200/csrc/fp4_gemm.cuh", "block_scaled_fp4_reduce_b200/csrc/fp4_gemm.cu"]
 OPS = ["amax", "nvfp4_quantize", "mxfp4_quantize", "nvfp4_dequantize", "mxfp4_dequantize", "scale_search"]
 
 
@@ -89,7 +90,8 @@ def peaks() -> dict:
 
 def kernel_source_hash(extra: tuple = ()) -> str:
     """Hash of the kernel sources a traffic capture was taken from (the
-    layout workloads' kernels also live in LAYOUT_SOURCES)."""
+    layout and GEMM workloads' kernels also live in the sources
+    traffic_sources names)."""
     h = hashlib.sha256()
     for rel in list(KERNEL_SOURCES) + list(extra):
         with open(os.path.join(ROOT, rel), "rb") as f:
@@ -932,6 +934,16 @@ def search_candidate_count(x: torch.Tensor, g: float) -> int:
 SEARCH_OPS_PER_EVAL = 7
 
 
+def traffic_sources(workload: str) -> tuple:
+    """Sources beyond KERNEL_SOURCES whose kernels a workload's traffic
+    figures were captured from (the layout and GEMM kernels)."""
+    if workload in LAYOUT_WORKLOADS:
+        return tuple(LAYOUT_SOURCES)
+    if workload == GEMM_WORKLOAD:
+        return tuple(GEMM_SOURCES)
+    return ()
+
+
 def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict, n_cand: int | None = None,
                  gemm_mnk=None) -> dict:
     # DRAM bytes per launch from an ncu capture (profiles/traffic.json), used
@@ -942,8 +954,7 @@ def roofline_for(name: str, k: dict, w: workloads.Workload, pk: dict, n_cand: in
         with open(tpath) as f:
             t = json.load(f)
         ent = t.get("workloads", {}).get(w.name, {}).get(name)
-        extra = tuple(LAYOUT_SOURCES) if w.name in LAYOUT_WORKLOADS else ()
-        if ent and ent.get("source_hash") == kernel_source_hash(extra):
+        if ent and ent.get("source_hash") == kernel_source_hash(traffic_sources(w.name)):
             traffic = ent.get("bytes_per_launch")
     if name == "nvfp4_gemm" and gemm_mnk:
         # tensor-bound: 2 M N K flops per launch against the FP4 dense peak,
