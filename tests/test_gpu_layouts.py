@@ -253,3 +253,34 @@ def test_with_amax_nonfinite_amax_sets_status():
             q = call(x, amax=a)
             torch.cuda.synchronize()
             assert q.status.item() == fp4.ERR_NONFINITE, (call.__name__, bad)
+
+
+def test_padded_full_size_ragged_sampled_rows():
+    """The 8192 x 14335 bf16 ragged-row workload as the benchmark runs it
+    (the step's amax handed to the NVFP4 call): padded NVFP4 / MXFP4 codes
+    and scales, and both bf16 dequantisations cut back to 14335 columns,
+    checked against the oracle on sampled rows (first and last included)."""
+    w = workloads.RAGGED_8K
+    x = workloads.generate(w)
+    xd = x.to(DEV)
+    amax, _ = fp4.tensor_amax(xd)
+    nv = fp4.nvfp4_quantize_padded(xd, amax=amax)
+    mx = fp4.mxfp4_quantize_padded(xd)
+    ynv = fp4.dequantize_padded(nv, torch.bfloat16)
+    ymx = fp4.dequantize_padded(mx, torch.bfloat16)
+    torch.cuda.synchronize()
+    nv.check()
+    mx.check()
+    g = oracle.nv_global_scale(x.abs().amax().float().item())
+    assert nv.global_scale.item() == g
+    R, K = x.shape
+    rows = workloads.sample_rows(R, 16, seed=5)
+    sub = odata(x[rows].contiguous())
+    p, s = oracle.nvfp4_quantize_with_g(oracle.pad_rows(sub, 16), g)
+    assert_same(nv.packed[rows], p, "NV padded packed (sampled rows)")
+    assert_same(nv.scales[rows], s, "NV padded scales (sampled rows)")
+    assert_same_bits(ynv[rows], oracle.nvfp4_dequantize_padded(p, s, g, len(rows), K), "NV padded dequant (sampled)")
+    p, s = oracle.mxfp4_quantize_padded(sub)
+    assert_same(mx.packed[rows], p, "MX padded packed (sampled rows)")
+    assert_same(mx.scales[rows], s, "MX padded scales (sampled rows)")
+    assert_same_bits(ymx[rows], oracle.mxfp4_dequantize_padded(p, s, len(rows), K), "MX padded dequant (sampled)")
