@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
             "fp4_e2m1_round": (I, [P, P, I64, P]),
             "fp4_e2m1_roundtrip": (I, [P, P, I64, P]),
             "fp4_nv_encode_quotient": (I, [P, P, P, I64, P]),
+            "fp4_test_bounded_wait": (I, [ctypes.c_uint32, P, P, P]),
             "fp4_grouped_workspace_bytes": (SZ, [I]),
             "fp4_nvfp4_quantize_grouped": (I, [P, I, I, P, SZ, P, P]),
             "fp4_tensor_amax_grouped": (I, [P, I, I, P, SZ, P, P]),
@@ -304,6 +305,10 @@ def fp4_e2m1_roundtrip(v, out, stream=None) -> int:
 
 def fp4_nv_encode_quotient(x, d, codes, stream=None) -> int:
     return lib().fp4_nv_encode_quotient(_p(x), _p(d), _p(codes), x.numel(), _stream(stream))
+
+
+def fp4_test_bounded_wait(tries: int, status, elapsed_ns, stream=None) -> int:
+    return lib().fp4_test_bounded_wait(tries, _p(status), _p(elapsed_ns), _stream(stream))
 
 
 # ------------------------------------------------- allocating helpers ------

@@ -11,6 +11,7 @@
 
 #include "fp4.h"
 #include "fp4_kernels.cuh"
+#include "fp4_async.cuh"
 #include "fp4_launch.cuh"
 
 namespace fp4_launch {
@@ -405,6 +406,14 @@ fp4_status fp4_e2m1_roundtrip(const float *v, float *out, int64_t n, cudaStream_
     if (grid <= 0)
         return FP4_ERR_CUDA;
     return launch(fp4::e2m1_roundtrip_kernel, grid, stream, v, out, n);
+}
+
+fp4_status fp4_test_bounded_wait(uint32_t tries, int32_t *status, int64_t *elapsed_ns, cudaStream_t stream)
+{
+    if (tries < 1 || tries > fp4::kWaitTries || !status || !elapsed_ns)
+        return FP4_ERR_INVALID_ARG;
+    return launch_cfg(fp4::bounded_wait_test_kernel, dim3(1), 32, 0, stream, tries, status,
+                      reinterpret_cast<long long *>(elapsed_ns));
 }
 
 fp4_status fp4_nv_encode_quotient(const float *x, const float *d, uint8_t *codes, int64_t n,

@@ -490,6 +490,16 @@ fp4_status fp4_e2m1_roundtrip(const float *v, float *out, int64_t n, cudaStream_
 fp4_status fp4_nv_encode_quotient(const float *x, const float *d, uint8_t *codes, int64_t n,
                                   cudaStream_t stream);
 
+/* Bounded wait alone, for tests: one warp waits on a shared-memory barrier
+ * that nothing arrives on, for `tries` polls (1 .. 2^18; every wait of the
+ * kernels that copy with TMA is bounded the same way, at 2^18 polls of about
+ * 4 us each, i.e. about a second).  When the
+ * wait runs out the kernel records FP4_ERR_TIMEOUT in *status (first error
+ * sticks) and returns, leaving the context usable; *elapsed_ns (device
+ * int64) receives the wait's duration on the GPU's global timer.
+ * FP4_ERR_INVALID_ARG for other tries or NULL pointers. */
+fp4_status fp4_test_bounded_wait(uint32_t tries, int32_t *status, int64_t *elapsed_ns, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
